@@ -1,0 +1,358 @@
+"""Benchmark: one content-adaptive block-sparse attention layer at the Wan-14B
+720p shape (40 heads, d=128, 21x48x80 tokens, thr=0.1 unioned with the +-1
+STA window), seeded synthetic inputs.
+
+A step is one pass of the whole path on one layer's inputs: fractal flatten of
+Q, K, V -> block mean pooling -> reduced softmax + CDF selection + STA union +
+CSR -> block-sparse attention (O, LSE) -> unflatten of O.  `value` is ms per
+layer (lower is better); with N GPUs every rank runs its own layer (weak
+scaling, no collective on the data path) and value = max-over-ranks time / N.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+`--impl reference` times the CPU oracle (the plain fp64 restatement under
+oracle/) on a bounded sample of the same workload, extrapolated to one layer.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "wan14b-720p"
+METRIC = "ms/attention layer and kept-tile TFLOP/s at Wan-14B 720p shape, thr=0.1"
+UNIT = "ms/layer"
+L2_FLUSH_BYTES = 256 << 20
+PROFILE = os.path.join(ROOT, "profiles", "sparse_attn_fwd_wan14b.md")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="vsa", choices=["vsa", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["bf16_tflops"], p["hbm_gbs"], "measured"
+    except Exception:
+        return 1590.0, 6650.0, "fallback"
+
+
+def profile_traffic(kernel_src: str):
+    """DRAM bytes per attention launch from the committed ncu summary, if it was
+    taken on the current kernel source (same hash); else None."""
+    try:
+        text = open(PROFILE).read()
+    except OSError:
+        return None
+    h = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
+    b = re.search(r"dram_bytes_per_launch_full:\s*([0-9.eE+]+)", text)
+    if not h or not b:
+        return None
+    cur = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
+    return float(b.group(1)) if cur.startswith(h.group(1)) else None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = [r.split(",") for r in self.out.strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = np.array([float(r[1]) for r in rows])
+        mx = float(rows[0][2])
+        power = np.array([float(r[3]) for r in rows if r[3].strip() not in ("", "[N/A]")] or [0.0])
+        loaded = sm[power >= np.percentile(power, 50)] if power.size == sm.size else sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i]})
+        return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- GPU arm
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import content_adaptive_block_fractal_b200 as vsa
+    from content_adaptive_block_fractal_b200 import workloads
+
+    torch.cuda.set_device(local_rank)
+    wl = workloads.get(args.workload)
+    shape = vsa.Shape.of(wl)
+    params = vsa.MaskParams(wl.thr, wl.use_sta, wl.sta)
+
+    q, k, v = workloads.make_qkv(wl)                       # host bf16, raster order
+    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+    qd, kd, vd = (x.cuda() for x in (qh, kh, vh))
+    stream = torch.cuda.current_stream()
+    qf, kf, vf = (torch.empty_like(qd) for _ in range(3))
+    layer = vsa.Layer(shape, params, qd.device)
+    o_raster = torch.empty_like(qd)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=qd.device)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
+    launches_per_step = 3 + 1 + 3 + 2 + 1   # flatten x3, pool, mask x3, plan+attn, unflatten
+
+    def step(record=False):
+        if record: ev[0].record(stream)
+        vsa.fractal_flatten(qd, shape, out=qf)
+        vsa.fractal_flatten(kd, shape, out=kf)
+        vsa.fractal_flatten(vd, shape, out=vf)
+        if record: ev[1].record(stream)
+        vsa.pool_qk(qf, kf, shape, out=(layer.qp, layer.kp))
+        if record: ev[2].record(stream)
+        vsa.block_mask(layer.qp, layer.kp, shape, params, out=layer.csr, workspace=layer.ws_mask)
+        if record: ev[3].record(stream)
+        vsa.sparse_attn_fwd(qf, kf, vf, layer.csr.row_ptr, layer.csr.col_idx, shape, 0.0,
+                            out=(layer.o, layer.lse), workspace=layer.ws_attn)
+        if record: ev[4].record(stream)
+        vsa.fractal_unflatten(layer.o, shape, out=o_raster)
+        if record: ev[5].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    vsa.device_status()
+    kept = int(layer.csr.row_ptr[-1].item())
+    rows = shape.B * shape.heads * shape.Nb
+    kept_frac = kept / (rows * shape.Nb)
+    flop_per_tile = 4 * 64 * 64 * shape.d
+    kept_flop = kept * flop_per_tile
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    parts = np.zeros(5)
+    total = 0.0
+    with ClockSampler(local_rank) as clk:
+        for _ in range(args.steps):
+            flush.zero_()
+            step(record=True)
+            ev[5].synchronize()
+            t = [ev[i].elapsed_time(ev[i + 1]) for i in range(5)]
+            parts += t
+            total += ev[0].elapsed_time(ev[5])
+    torch.cuda.synchronize()
+    vsa.device_status()
+    ms = total / args.steps
+    parts /= args.steps
+
+    # end to end through the public API with host buffers: H2D of raster
+    # Q, K, V from pinned memory, the whole path, D2H of O and LSE
+    e2e = None
+    if not args.no_e2e:
+        o_host = torch.empty(qh.shape, dtype=torch.bfloat16, pin_memory=True)
+        lse_host = torch.empty(layer.lse.shape, dtype=torch.float32, pin_memory=True)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, min(args.steps, 10))
+
+        def e2e_step():
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            step()
+            o_host.copy_(o_raster, non_blocking=True)
+            lse_host.copy_(layer.lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / n_e2e
+        e2e = {"value": e2e_ms, "unit": UNIT,
+               "h2d_bytes_per_step": 3 * qh.numel() * 2,
+               "d2h_bytes_per_step": o_host.numel() * 2 + lse_host.numel() * 4}
+
+    if world > 1:
+        t = torch.tensor([ms, e2e["value"] if e2e else 0.0], device=qd.device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t[0])
+        if e2e:
+            e2e["value"] = float(t[1]) / world
+    value = ms / world
+    peak_tf, peak_gbs, peak_src = measured_peaks()
+    attn_ms = parts[3]
+    achieved_tf = kept_flop / (attn_ms * 1e-3) / 1e12
+    traffic = profile_traffic(os.path.join(ROOT, "content_adaptive_block_fractal_b200", "csrc", "k_attn.cu"))
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {**wl.describe(), "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "256 MiB flush written between timed steps; Q/K/V 2.5 GB > L2",
+                   "step": "flatten q,k,v + pool + mask + sparse attention + unflatten o"},
+        "kept_tile_tflops": achieved_tf,
+        "kept_tile_tflops_layer": kept_flop / (ms * 1e-3) / 1e12,
+        "kept_fraction": kept_frac,
+        "kept_tiles": kept,
+        "breakdown_ms": {"flatten_qkv": parts[0], "pool": parts[1], "mask": parts[2],
+                         "sparse_attn": parts[3], "unflatten_o": parts[4]},
+        "roofline": {"bound": "tensor", "kernel": "sparse_attn_kernel<128>",
+                     "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": achieved_tf / peak_tf, "traffic": traffic,
+                     "peak_source": f"{peak_src} bf16 (burst)",
+                     "flop_per_kept_tile": flop_per_tile},
+        "mask_path_gbs": (shape.B * shape.heads * shape.N * shape.d * 2 * 2
+                          + 2 * rows * shape.d * 8) / ((parts[1] + parts[2]) * 1e-3) / 1e9,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if e2e:
+        result["e2e"] = e2e
+    return result, (q, k, v, wl)
+
+
+# --------------------------------------------------------------------------- CPU oracle
+def oracle_sample(wl, heads, n_qblocks, seed=0):
+    """Time the oracle on `heads` (flatten, pool, mask in full; attention on
+    n_qblocks sampled query blocks per head) and extrapolate to one layer."""
+    import oracle
+    from content_adaptive_block_fractal_b200 import workloads
+    oracle.lib()
+    t_perm = t_pool = t_mask = t_attn = 0.0
+    kept_total = kept_sampled = 0
+    for h in heads:
+        q, k, v = workloads.make_qkv(wl, heads=[h])
+        t0 = time.perf_counter()
+        qf, kf, vf = (oracle.flatten(x, wl.T, wl.H, wl.W) for x in (q, k, v))
+        t1 = time.perf_counter()
+        qp, kp = oracle.pool(qf), oracle.pool(kf)
+        t2 = time.perf_counter()
+        keep, _ = oracle.block_mask(qp, kp, wl.Hb, wl.Wb, float(np.float32(wl.thr)), wl.use_sta, wl.sta)
+        rp, ci = oracle.mask_to_csr(keep)
+        t3 = time.perf_counter()
+        rng = np.random.default_rng(seed + h)
+        qb = rng.choice(wl.Nb, n_qblocks, replace=False)
+        oracle.sparse_attention(qf, kf, vf, rp, ci, qblocks=qb)
+        t4 = time.perf_counter()
+        cnt = np.diff(rp)
+        t_perm += (t1 - t0) * 4.0 / 3.0            # unflatten of O costs one more permute
+        t_pool += t2 - t1
+        t_mask += t3 - t2
+        t_attn += t4 - t3
+        kept_total += int(cnt.sum())
+        kept_sampled += int(cnt[qb].sum())
+    nh = len(heads)
+    scale_heads = wl.B * wl.heads / nh
+    ms = 1e3 * ((t_perm + t_pool + t_mask) * scale_heads
+                + t_attn * (kept_total / max(kept_sampled, 1)) * scale_heads)
+    work_s = t_perm + t_pool + t_mask + t_attn
+    sample = (f"{nh} of {wl.B * wl.heads} heads: flatten/pool/mask in full, attention on "
+              f"{n_qblocks} query blocks per head; extrapolated by heads and by kept tiles")
+    return ms, work_s, sample
+
+
+def run_reference(args):
+    import oracle
+    from content_adaptive_block_fractal_b200 import workloads
+    wl = workloads.get(args.workload)
+    cores = oracle.num_threads()
+    vals = []
+    for i in range(args.warmup + args.steps):
+        ms, _, sample = oracle_sample(wl, [i % wl.heads], 16, seed=i)
+        if i >= args.warmup:
+            vals.append(ms)
+    value = float(np.mean(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": value,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": wl.describe(),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        result, _ = run_gpu(args, rank, world, local_rank)
+        if rank == 0:
+            if not args.no_cpu_baseline:
+                import oracle
+                wl = __import__("content_adaptive_block_fractal_b200.workloads",
+                                fromlist=["get"]).get(args.workload)
+                ms, work_s, sample = oracle_sample(wl, [0, 1, 2, 3], 96)
+                result["cpu_baseline"] = {"value": ms, "unit": UNIT, "cores": oracle.num_threads(),
+                                          "kind": "oracle", "sample": sample,
+                                          "cpu_seconds_measured": work_s}
+            print(json.dumps(result), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

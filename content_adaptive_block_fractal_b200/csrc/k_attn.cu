@@ -1,0 +1,644 @@
+// k_attn.cu -- block-sparse attention forward over kept 64 x 64 tiles
+// (NABLA, Methodology item 2, "expansion": the block mask decides which
+// N x N tiles are computed; Sparse VideoGen2 section 2C: contiguous query
+// blocks are computed densely while key/value blocks are loaded sparsely).
+//
+// Blackwell mapping.  A work item is a 128-row query tile made of two 64-token
+// query blocks of one (batch, head): the same patch in frames 2t and 2t+1,
+// whose kept lists overlap most (time pairing).  The item walks the merged,
+// ascending union of both lists two key blocks (128 keys) per step:
+//   S  = Q K^T   tcgen05.mma M=128, N=64*nb, K=d   (SMEM x SMEM -> TMEM fp32)
+//   P  = online softmax of S, per row only over the blocks kept by that row's
+//        query block, written to SMEM as bf16
+//   O += P V     tcgen05.mma M=128, N=d, K=64*nb   (SMEM x SMEM -> TMEM fp32)
+// Warp roles (192 threads, one CTA per SM, persistent):
+//   warp 0      producer: takes items from an atomic counter over an LPT work
+//               list, merges the two CSR lists, issues TMA loads of Q and of
+//               the K/V blocks into a 2-stage ring (128B-swizzled boxes);
+//   warp 1      allocates TMEM; one lane issues all MMAs and commits;
+//   warps 2..5  one thread per query row: softmax, lazy O rescale (only when
+//               the running max grows by more than 2^8), epilogue O / l -> bf16
+//               and LSE.
+// Every mbarrier wait is bounded; a wait that gives up records an error code
+// and the CTA winds down instead of hanging.
+#include "vsa_device.cuh"
+#include "vsa_internal.h"
+
+#include <cmath>
+#include <mutex>
+
+namespace vsa {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kStages = 2;
+constexpr int kListWin = 512;          // CSR entries staged per list in SMEM
+constexpr uint32_t kTmemCols = 256;    // O: [0, 128), S: [128, 256)
+constexpr uint32_t kTmemS = 128;
+
+struct StepMeta {
+  int32_t blk0, blk1;  // key blocks of this step (blk1 = -1 when nb == 1)
+  int32_t nb;          // 1 or 2 key blocks; 0 = empty item; -1 = no more work
+  uint32_t flags;      // bit0/1: blk0 kept by query block 0/1; bit2/3: blk1
+  int32_t bh, r0, r1;  // head slice and query blocks (r1 = -1 if absent)
+  int32_t first_last;  // bit0: first step of the item, bit1: last step
+};
+
+template <int D>
+struct Smem {
+  static constexpr int kQBytes = 128 * D * 2;             // two query blocks
+  static constexpr int kKVHalf = 2 * 64 * D * 2;          // K (or V) of two key blocks
+  static constexpr int kStageBytes = 2 * kKVHalf;         // K + V
+  static constexpr int kPBytes = 128 * 128 * 2;           // P tile, 128 keys
+  static constexpr int kQOff = 0;
+  static constexpr int kKVOff = kQOff + kQBytes;
+  static constexpr int kPOff = kKVOff + kStages * kStageBytes;
+  static constexpr int kMetaOff = kPOff + kPBytes;
+  static constexpr int kListOff = kMetaOff + kStages * static_cast<int>(sizeof(StepMeta));
+  static constexpr int kBarOff = kListOff + 2 * kListWin * 4;
+  static constexpr int kNumBars = 2 * kStages + 6;
+  static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kTmemSlotOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;            // room to align to 1 KiB
+};
+
+struct AttnArgs {
+  const int64_t *row_ptr;
+  const int32_t *col_idx;
+  __nv_bfloat16 *o;
+  float *lse;
+  const int32_t *order;   // LPT-ordered work items
+  int *counter;           // next position in `order`
+  unsigned *err;
+  int64_t items;          // total work items
+  int64_t N;              // tokens per head
+  int Nb, T, HW;          // blocks per head, frames, patches per frame
+  int pairs_per_head;
+  float c;                // scale * log2(e)
+  float lse_scale;        // ln(2)
+};
+
+// item -> (bh, r0, r1): the same patch in frames 2t and 2t+1.
+__device__ __forceinline__ void decode_item(int item, const AttnArgs &a, int &bh, int &r0,
+                                            int &r1) {
+  bh = item / a.pairs_per_head;
+  const int p = item % a.pairs_per_head;
+  const int t2 = p / a.HW, sp = p % a.HW;
+  r0 = 2 * t2 * a.HW + sp;
+  r1 = (2 * t2 + 1 < a.T) ? r0 + a.HW : -1;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    sparse_attn_kernel(const __grid_constant__ CUtensorMap tq,
+                       const __grid_constant__ CUtensorMap tk,
+                       const __grid_constant__ CUtensorMap tv, const AttnArgs a) {
+  using L = Smem<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *smem = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  StepMeta *meta = reinterpret_cast<StepMeta *>(smem + L::kMetaOff);
+  int32_t *list0 = reinterpret_cast<int32_t *>(smem + L::kListOff);
+  int32_t *list1 = list0 + kListWin;
+  const uint32_t bar = sbase + L::kBarOff;
+  auto kv_full = [&](int s) { return bar + 8u * s; };
+  auto kv_empty = [&](int s) { return bar + 8u * (kStages + s); };
+  const uint32_t q_full = bar + 8u * (2 * kStages + 0);
+  const uint32_t q_empty = bar + 8u * (2 * kStages + 1);
+  const uint32_t s_full = bar + 8u * (2 * kStages + 2);
+  const uint32_t p_full = bar + 8u * (2 * kStages + 3);
+  const uint32_t o_full = bar + 8u * (2 * kStages + 4);
+  const uint32_t o_empty = bar + 8u * (2 * kStages + 5);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemSlotOff);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(kv_full(s), 1);
+      mbar_init(kv_empty(s), 1);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(o_full, 1);
+    mbar_init(o_empty, 128);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tq);
+      tma_prefetch_desc(&tk);
+      tma_prefetch_desc(&tv);
+    }
+    int stage = 0;
+    uint32_t kv_phase = 0;   // bit s: parity to wait on kv_empty[s]
+    uint32_t q_phase = 0;
+    bool ok = true;
+    int nitems = 0;
+    // Waits until stage `stage` is free, publishes the step and loads it.
+    auto emit = [&](const StepMeta &m) -> bool {
+      if (!mbar_wait(kv_empty(stage), ((kv_phase >> stage) & 1u) ^ 1u, a.err, kErrWaitMma))
+        return false;
+      kv_phase ^= 1u << stage;
+      if (lane == 0) {
+        meta[stage] = m;
+        const int nb = m.nb > 0 ? m.nb : 0;
+        mbar_arrive_expect_tx(kv_full(stage), static_cast<uint32_t>(nb * 2 * 64 * D * 2));
+        const uint32_t kbase = sbase + L::kKVOff + stage * L::kStageBytes;
+        const uint32_t vbase = kbase + L::kKVHalf;
+        for (int j = 0; j < nb; ++j) {
+          const int row = static_cast<int>(static_cast<int64_t>(m.bh) * a.N) +
+                          (j ? m.blk1 : m.blk0) * 64;
+          for (int dh = 0; dh < D / 64; ++dh) {
+            const uint32_t off = dh * (2 * 64 * 128) + j * (64 * 128);
+            tma_load_2d(kbase + off, &tk, kv_full(stage), dh * 64, row);
+            tma_load_2d(vbase + off, &tv, kv_full(stage), dh * 64, row);
+          }
+        }
+      }
+      __syncwarp();
+      stage = (stage + 1) % kStages;
+      return true;
+    };
+    while (ok) {
+      int item = 0;
+      if (lane == 0) item = atomicAdd(a.counter, 1);
+      item = __shfl_sync(0xFFFFFFFFu, item, 0);
+      if (item >= a.items) {
+        StepMeta m{};
+        m.nb = -1;
+        emit(m);
+        break;
+      }
+      item = a.order[item];
+      int bh, r0, r1;
+      decode_item(item, a, bh, r0, r1);
+      // Q tile: query block r0 -> rows 0..63, r1 -> rows 64..127
+      if (nitems > 0) {
+        if (!mbar_wait(q_empty, q_phase, a.err, kErrWaitMma)) break;
+        q_phase ^= 1u;
+      }
+      ++nitems;
+      if (lane == 0) {
+        const int nq = r1 >= 0 ? 2 : 1;
+        mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(nq * 64 * D * 2));
+        for (int j = 0; j < nq; ++j) {
+          const int row = static_cast<int>(static_cast<int64_t>(bh) * a.N) + (j ? r1 : r0) * 64;
+          for (int dh = 0; dh < D / 64; ++dh)
+            tma_load_2d(sbase + L::kQOff + dh * (128 * 128) + j * (64 * 128), &tq, q_full,
+                        dh * 64, row);
+        }
+      }
+      // merge the two ascending lists, two union entries per step
+      const int64_t g0 = static_cast<int64_t>(bh) * a.Nb + r0;
+      const int64_t b0 = a.row_ptr[g0], n0 = a.row_ptr[g0 + 1] - b0;
+      int64_t b1 = 0, n1 = 0;
+      if (r1 >= 0) {
+        b1 = a.row_ptr[g0 + a.HW];
+        n1 = a.row_ptr[g0 + a.HW + 1] - b1;
+      }
+      int64_t i0 = 0, i1 = 0, w0 = -kListWin, w1 = -kListWin;
+      StepMeta pend{};
+      pend.bh = bh; pend.r0 = r0; pend.r1 = r1;
+      pend.nb = 0; pend.first_last = 1;
+      bool have_pending = false;
+      StepMeta cur = pend;
+      cur.nb = 0; cur.flags = 0; cur.blk0 = cur.blk1 = -1;
+      while (i0 < n0 || i1 < n1) {
+        if (i0 < n0 && i0 >= w0 + kListWin) {
+          w0 = i0;
+          __syncwarp();
+          for (int j = lane; j < kListWin && w0 + j < n0; j += 32) list0[j] = a.col_idx[b0 + w0 + j];
+          __syncwarp();
+        }
+        if (i1 < n1 && i1 >= w1 + kListWin) {
+          w1 = i1;
+          __syncwarp();
+          for (int j = lane; j < kListWin && w1 + j < n1; j += 32) list1[j] = a.col_idx[b1 + w1 + j];
+          __syncwarp();
+        }
+        const int c0 = i0 < n0 ? list0[i0 - w0] : 0x7FFFFFFF;
+        const int c1 = i1 < n1 ? list1[i1 - w1] : 0x7FFFFFFF;
+        const int c = c0 < c1 ? c0 : c1;
+        const uint32_t f = (c0 == c ? 1u : 0u) | (c1 == c ? 2u : 0u);
+        i0 += (c0 == c);
+        i1 += (c1 == c);
+        if (c < 0 || c >= a.Nb) {  // invalid index: skip it, record once
+          if (lane == 0) atomicOr(a.err, kErrBadIndex);
+          continue;
+        }
+        if (cur.nb == 0) {
+          cur.blk0 = c;
+          cur.flags = f;
+          cur.nb = 1;
+        } else {
+          cur.blk1 = c;
+          cur.flags |= f << 2;
+          cur.nb = 2;
+          if (have_pending && !(ok = emit(pend))) break;
+          pend = cur;
+          pend.first_last = have_pending ? 0 : 1;
+          have_pending = true;
+          cur.nb = 0; cur.flags = 0; cur.blk0 = cur.blk1 = -1;
+        }
+      }
+      if (!ok) break;
+      if (cur.nb > 0) {
+        if (have_pending && !(ok = emit(pend))) break;
+        const int first = have_pending ? 0 : 1;
+        pend = cur;
+        pend.first_last = first;
+        have_pending = true;
+      }
+      if (!have_pending) {  // empty item: one step without blocks
+        pend.nb = 0; pend.flags = 0; pend.blk0 = pend.blk1 = -1;
+        pend.first_last = 1;
+      }
+      pend.first_last |= 2;
+      if (!(ok = emit(pend))) break;
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    int stage = 0;
+    uint32_t kv_phase = 0, q_phase = 0, p_phase = 0, oe_phase = 0;
+    bool first_item = true;
+    constexpr uint32_t kIdescO = idesc_bf16(128, D, false, true);
+    while (true) {
+      if (!mbar_wait(kv_full(stage), (kv_phase >> stage) & 1u, a.err, kErrWaitTma)) break;
+      kv_phase ^= 1u << stage;
+      const StepMeta m = meta[stage];
+      if (m.nb < 0) break;
+      const bool first = m.first_last & 1, last = m.first_last & 2;
+      if (first) {
+        if (!mbar_wait(q_full, q_phase, a.err, kErrWaitTma)) break;
+        q_phase ^= 1u;
+      }
+      tc_fence_after();
+      const uint32_t qb = sbase + L::kQOff;
+      const uint32_t kb = sbase + L::kKVOff + stage * L::kStageBytes;
+      const uint32_t vb = kb + L::kKVHalf;
+      const uint32_t pb = sbase + L::kPOff;
+      if (lane == 0 && m.nb > 0) {
+        const uint32_t idesc_s = idesc_bf16(128, 64 * m.nb, false, false);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint64_t ad = smem_desc(qb + (k >> 2) * (128 * 128) + (k & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc(kb + (k >> 2) * (2 * 64 * 128) + (k & 3) * 32, 16, 1024);
+          mma_bf16_ss(tmem + kTmemS, ad, bd, idesc_s, k > 0);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mma_commit(s_full);
+        if (last) mma_commit(q_empty);
+      }
+      __syncwarp();
+      if (!mbar_wait(p_full, p_phase, a.err, kErrWaitSoftmax)) break;
+      p_phase ^= 1u;
+      if (first) {
+        if (!first_item) {
+          if (!mbar_wait(o_empty, oe_phase, a.err, kErrWaitSoftmax)) break;
+          oe_phase ^= 1u;
+        }
+        first_item = false;
+      }
+      tc_fence_after();
+      if (lane == 0 && m.nb > 0) {
+        for (int k = 0; k < 4 * m.nb; ++k) {
+          const uint64_t ad = smem_desc(pb + (k >> 2) * (128 * 128) + (k & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc(vb + k * 2048, 2 * 64 * 128, 1024);
+          mma_bf16_ss(tmem, ad, bd, kIdescO, !(first && k == 0));
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mma_commit(kv_empty(stage));
+        if (last) mma_commit(o_full);
+      }
+      __syncwarp();
+      stage = (stage + 1) % kStages;
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int quarter = warp & 3;              // TMEM lane quarter of this warp
+    const int row = quarter * 32 + lane;       // query row within the tile
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t sel = row >= 64 ? 1u : 0u;
+    unsigned char *prow = smem + L::kPOff + (row >> 3) * 1024 + (row & 7) * 128;
+    int stage = 0;
+    uint32_t kv_phase = 0, s_phase = 0, o_phase = 0;
+    float m_run = -INFINITY, l_run = 0.0f;
+    while (true) {
+      if (!mbar_wait(kv_full(stage), (kv_phase >> stage) & 1u, a.err, kErrWaitTma)) break;
+      kv_phase ^= 1u << stage;
+      const StepMeta m = meta[stage];
+      if (m.nb < 0) break;
+      const bool first = m.first_last & 1, last = m.first_last & 2;
+      if (first) {
+        m_run = -INFINITY;
+        l_run = 0.0f;
+      }
+      if (!mbar_wait(s_full, s_phase, a.err, kErrWaitMma)) break;
+      s_phase ^= 1u;
+      tc_fence_after();
+      float x[128];
+      const bool v0 = (m.flags >> sel) & 1u;
+      const bool v1 = (m.flags >> (2 + sel)) & 1u;
+      float mx = -INFINITY;
+      if (m.nb > 0) {
+        tmem_ld32(lane_addr + kTmemS + 0, &x[0]);
+        tmem_ld32(lane_addr + kTmemS + 32, &x[32]);
+        if (m.nb > 1) {
+          tmem_ld32(lane_addr + kTmemS + 64, &x[64]);
+          tmem_ld32(lane_addr + kTmemS + 96, &x[96]);
+        }
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          x[j] = v0 ? x[j] * a.c : -INFINITY;
+          mx = fmaxf(mx, x[j]);
+        }
+        if (m.nb > 1) {
+#pragma unroll
+          for (int j = 64; j < 128; ++j) {
+            x[j] = v1 ? x[j] * a.c : -INFINITY;
+            mx = fmaxf(mx, x[j]);
+          }
+        }
+      }
+      // lazy rescale: move the reference max only when it grows by > 8 (2^8)
+      float alpha = 1.0f;
+      bool resc = false;
+      if (mx > m_run + 8.0f) {
+        if (m_run != -INFINITY) {
+          alpha = ex2(m_run - mx);
+          resc = !first;
+        }
+        l_run *= alpha;
+        m_run = mx;
+      }
+      const float mref = m_run == -INFINITY ? 0.0f : m_run;
+      float rs = 0.0f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (h < m.nb) {
+          unsigned char *dst = prow + h * (128 * 128);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float p0 = ex2(x[h * 64 + j * 8 + 2 * e] - mref);
+              const float p1 = ex2(x[h * 64 + j * 8 + 2 * e + 1] - mref);
+              rs += p0 + p1;
+              w[e] = pack_bf16x2(p0, p1);
+            }
+            *reinterpret_cast<uint4 *>(dst + ((j ^ (row & 7)) << 4)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+      l_run += rs;
+      if (__any_sync(0xFFFFFFFFu, resc)) {
+#pragma unroll 1
+        for (int cc = 0; cc < D; cc += 32) {
+          float ov[32];
+          tmem_ld32(lane_addr + cc, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ov[j] *= alpha;
+          tmem_st32(lane_addr + cc, ov);
+        }
+        tmem_wait_st();
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full);
+      if (last) {
+        if (!mbar_wait(o_full, o_phase, a.err, kErrWaitMma)) break;
+        o_phase ^= 1u;
+        tc_fence_after();
+        const int rblk = sel ? m.r1 : m.r0;
+        const bool store = rblk >= 0;
+        const bool has_keys = l_run > 0.0f;
+        const float inv = has_keys ? 1.0f / l_run : 0.0f;
+        const int64_t tok = static_cast<int64_t>(m.bh) * a.N + static_cast<int64_t>(rblk) * 64 +
+                            (row & 63);
+        uint4 *orow = reinterpret_cast<uint4 *>(a.o + tok * D);
+#pragma unroll 1
+        for (int cc = 0; cc < D; cc += 32) {
+          float ov[32];
+          tmem_ld32(lane_addr + cc, ov);
+          tmem_wait_ld();
+          if (store) {
+            if (!has_keys) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) ov[j] = 0.0f;
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint4 u;
+              u.x = pack_bf16x2(ov[8 * j + 0] * inv, ov[8 * j + 1] * inv);
+              u.y = pack_bf16x2(ov[8 * j + 2] * inv, ov[8 * j + 3] * inv);
+              u.z = pack_bf16x2(ov[8 * j + 4] * inv, ov[8 * j + 5] * inv);
+              u.w = pack_bf16x2(ov[8 * j + 6] * inv, ov[8 * j + 7] * inv);
+              orow[cc / 8 + j] = u;
+            }
+          }
+        }
+        if (store)
+          a.lse[tok] = has_keys ? (m_run + log2f(l_run)) * a.lse_scale : -INFINITY;
+        tc_fence_before();
+        mbar_arrive(o_empty);
+      }
+      stage = (stage + 1) % kStages;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Work list: per head, items sorted by descending cost (kept blocks of both
+// query blocks), heads in order so that each head's K/V stays L2-resident.
+// One CTA per head; also resets the scheduler counter.
+__global__ void __launch_bounds__(1024) plan_kernel(const int64_t *__restrict__ row_ptr, int Nb,
+                                                    int T, int HW, int pairs, int32_t *order,
+                                                    int *counter) {
+  extern __shared__ unsigned long long keys[];
+  const int bh = blockIdx.x;
+  if (bh == 0 && threadIdx.x == 0) *counter = 0;
+  int n2 = 1;
+  while (n2 < pairs) n2 <<= 1;
+  for (int p = threadIdx.x; p < n2; p += blockDim.x) {
+    unsigned long long k = ~0ull;
+    if (p < pairs) {
+      const int t2 = p / HW, sp = p % HW;
+      const int r0 = 2 * t2 * HW + sp;
+      const int64_t g = static_cast<int64_t>(bh) * Nb + r0;
+      int64_t cost = row_ptr[g + 1] - row_ptr[g];
+      if (2 * t2 + 1 < T) cost += row_ptr[g + HW + 1] - row_ptr[g + HW];
+      if (cost > 0x7FFFFFFF) cost = 0x7FFFFFFF;
+      k = (static_cast<unsigned long long>(0x7FFFFFFFu - static_cast<uint32_t>(cost)) << 32) |
+          static_cast<uint32_t>(p);
+    }
+    keys[p] = k;
+  }
+  __syncthreads();
+  for (int size = 2; size <= n2; size <<= 1)
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < n2; i += blockDim.x) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool up = (i & size) == 0;
+          const unsigned long long x = keys[i], y = keys[j];
+          if ((x > y) == up) {
+            keys[i] = y;
+            keys[j] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  for (int p = threadIdx.x; p < pairs; p += blockDim.x)
+    order[static_cast<int64_t>(bh) * pairs + p] =
+        bh * pairs + static_cast<int32_t>(keys[p] & 0xFFFFFFFFu);
+}
+
+// Fallback order (no per-head sort) for very large heads.
+__global__ void identity_order_kernel(int32_t *order, int64_t n, int *counter) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i == 0) *counter = 0;
+  if (i < n) order[i] = static_cast<int32_t>(i);
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                              const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                              const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn() {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  });
+  return fn;
+}
+
+bool make_map(CUtensorMap *m, const void *base, int64_t rows, int d) {
+  EncodeFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  const cuuint32_t box[2] = {64, 64};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+struct AttnLayout {
+  int pairs, HW;
+  int64_t items;
+  size_t order_off, counter_off, total;
+};
+
+AttnLayout attn_layout(const Geometry &g) {
+  AttnLayout L;
+  L.HW = g.Hb * g.Wb;
+  L.pairs = ((g.T + 1) / 2) * L.HW;
+  L.items = g.BH * L.pairs;
+  L.counter_off = 0;
+  L.order_off = 256;
+  L.total = L.order_off + ((static_cast<size_t>(L.items) * 4 + 255) & ~static_cast<size_t>(255));
+  return L;
+}
+
+}  // namespace
+
+size_t sparse_attn_workspace_bytes(const Geometry &g) { return attn_layout(g).total; }
+
+cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
+                               const int64_t *row_ptr, const int32_t *col_idx,
+                               const Geometry &g, float scale, void *o, float *lse, void *ws,
+                               unsigned *err, cudaStream_t st, const char **why) {
+  const AttnLayout L = attn_layout(g);
+  if (L.items == 0) return cudaSuccess;
+  if (L.items > 0x7FFFFFFF || g.BH * g.N > 0x7FFFFFFF) {
+    *why = "sparse attention: too many tokens for 32-bit TMA row coordinates";
+    return cudaErrorInvalidValue;
+  }
+  CUtensorMap mq, mk, mv;
+  const int64_t rows = g.BH * g.N;
+  if (!make_map(&mq, qf, rows, g.d) || !make_map(&mk, kf, rows, g.d) ||
+      !make_map(&mv, vf, rows, g.d)) {
+    *why = "sparse attention: cuTensorMapEncodeTiled failed";
+    return cudaErrorInvalidValue;
+  }
+  unsigned char *w = static_cast<unsigned char *>(ws);
+  int *counter = reinterpret_cast<int *>(w + L.counter_off);
+  int32_t *order = reinterpret_cast<int32_t *>(w + L.order_off);
+  int n2 = 1;
+  while (n2 < L.pairs) n2 <<= 1;
+  cudaError_t e;
+  if (n2 <= 4096) {
+    plan_kernel<<<static_cast<int>(g.BH), 1024, n2 * 8, st>>>(row_ptr, static_cast<int>(g.Nb),
+                                                              g.T, L.HW, L.pairs, order, counter);
+  } else {
+    identity_order_kernel<<<static_cast<int>((L.items + 255) / 256), 256, 0, st>>>(order, L.items,
+                                                                                 counter);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  AttnArgs a;
+  a.row_ptr = row_ptr; a.col_idx = col_idx;
+  a.o = static_cast<__nv_bfloat16 *>(o); a.lse = lse;
+  a.order = order; a.counter = counter; a.err = err;
+  a.items = L.items; a.N = g.N; a.Nb = static_cast<int>(g.Nb); a.T = g.T; a.HW = L.HW;
+  a.pairs_per_head = L.pairs;
+  a.c = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  a.lse_scale = 0.6931471805599453f;
+  int grid = num_sms();
+  if (L.items < grid) grid = static_cast<int>(L.items);
+  if (g.d == 128) {
+    const int smem = Smem<128>::kAlloc;
+    if ((e = cudaFuncSetAttribute(sparse_attn_kernel<128>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+      return e;
+    sparse_attn_kernel<128><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+  } else {
+    const int smem = Smem<64>::kAlloc;
+    if ((e = cudaFuncSetAttribute(sparse_attn_kernel<64>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+      return e;
+    sparse_attn_kernel<64><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace vsa

@@ -1,0 +1,474 @@
+// k_mask.cu -- content-adaptive block mask (NABLA, Methodology item 2:
+// reduced attention over pooled blocks and the per-row CDF threshold; item 3:
+// union with the sliding-tile window; Sparse VideoGen2 section 2B: top-p).
+//
+// Three kernels:
+//   mask_select_kernel  persistent; one work item = 64 query blocks of one
+//                       (batch, head).  Phase A forms the 64 x Nb pooled
+//                       scores with fp64 tensor-core MMAs (m8n8k4) in column
+//                       tiles of 128, keeps each tile's row maxima in fp64 and
+//                       writes 2^(t - tile max) as fp32 to a CTA-private slab
+//                       that stays in L2.  Phase B, one warp per row, rescales
+//                       the slab to the row maximum, finds the CDF cut by
+//                       bisection on the fp32 bit pattern (mass tests in fp64,
+//                       candidates compacted once the range is narrow), breaks
+//                       ties by index, ORs in the STA window and writes a
+//                       kept-bit row and its count.
+//   scan_counts_kernel  exclusive scan of the counts into row_ptr (int64).
+//   expand_bits_kernel  kept bits -> ascending col_idx lists.
+//
+// Precision: scores are exact fp64 dot products of exact pooled means; each
+// probability carries a relative error of a few 1e-7 (fp32 storage and the
+// hardware exp2 on a reduced argument), so the kept set equals the exact one
+// except for rows whose cut is within that of 1 - thr or of a tie.
+#include "vsa_device.cuh"
+#include "vsa_internal.h"
+
+#include <cmath>
+
+namespace vsa {
+namespace {
+
+constexpr int kRT = 64;       // query blocks per work item
+constexpr int kCT = 128;      // key blocks per phase-A column tile
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kPad = 4;       // fp64 padding per smem row (conflict-free fragments)
+constexpr int kCand = 256;    // per-warp candidate list capacity
+constexpr int kMaxGrid = 160; // slabs in the workspace
+
+struct MaskArgs {
+  const double *qp, *kp;
+  int64_t BH;
+  int Nb, d, Hb, Wb;
+  float thr;
+  int use_sta, rt, rh, rw;
+  double c;          // scale * log2(e)
+  float *slab;       // [grid][kRT][ld_slab]
+  double *tmax;      // [grid][kRT][ntiles]
+  int ld_slab, ntiles;
+  uint32_t *bits;    // [BH*Nb][words]
+  int words;
+  int32_t *counts;   // [BH*Nb]
+  int64_t items, tiles_per_head;
+};
+
+__device__ __forceinline__ void dmma(double (&c)[2], double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+               : "+d"(c[0]), "+d"(c[1])
+               : "d"(a), "d"(b));
+}
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool valid) {
+  const uint32_t s = smem_u32(smem);
+  const int n = valid ? 16 : 0;  // src size 0 -> zero fill
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem), "r"(n)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_max(double v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmax(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+__device__ __forceinline__ int warp_sum_i(int v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+// 2^x for x <= 0 in fp64 argument, fp32 result with relative error ~2e-7:
+// split x = n + f with f in [0, 1), hardware exp2 of f, exact scaling by 2^n.
+__device__ __forceinline__ float exp2_split(double x) {
+  if (!(x > -126.0)) return 0.0f;  // also maps -inf / NaN to 0
+  const double n = floor(x);
+  const float f = static_cast<float>(x - n);
+  return ex2(f) * __int_as_float((static_cast<int>(n) + 127) << 23);
+}
+
+__device__ __forceinline__ bool sta_keep(int r, int c, const MaskArgs &a) {
+  const int hw = a.Hb * a.Wb;
+  const int tr = r / hw, yr = (r / a.Wb) % a.Hb, xr = r % a.Wb;
+  const int tc = c / hw, yc = (c / a.Wb) % a.Hb, xc = c % a.Wb;
+  return abs(tr - tc) <= a.rt && abs(yr - yc) <= a.rh && abs(xr - xc) <= a.rw;
+}
+
+// Phase B for one row: selection and kept bits.  ebuf: this warp's Nb floats.
+__device__ void select_row(const MaskArgs &a, int64_t grow, int r, const float *slab_row,
+                           const double *tmax_row, float *ebuf, uint32_t *cand_key,
+                           int32_t *cand_idx, double *tscale) {
+  const int lane = threadIdx.x & 31;
+  const int Nb = a.Nb;
+  // row maximum over the tile maxima, per-tile rescale factors in fp64
+  double M = -INFINITY;
+  for (int t = lane; t < a.ntiles; t += 32) M = fmax(M, tmax_row[t]);
+  M = warp_max(M);
+  for (int t = lane; t < a.ntiles; t += 32) tscale[t] = exp2(tmax_row[t] - M);
+  __syncwarp();
+  double z = 0.0;
+  uint32_t kmax = 0;
+  for (int c = lane; c < Nb; c += 32) {
+    const float e = static_cast<float>(static_cast<double>(slab_row[c]) * tscale[c / kCT]);
+    ebuf[c] = e;
+    z += static_cast<double>(e);
+    kmax = max(kmax, __float_as_uint(e));
+  }
+  z = warp_sum(z);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) kmax = max(kmax, __shfl_xor_sync(0xFFFFFFFFu, kmax, o));
+  __syncwarp();
+
+  bool keep_all = !(a.thr > 0.0f);
+  uint32_t vkey = 0;
+  int need_ties = 0;
+  if (!keep_all) {
+    const double target = (1.0 - static_cast<double>(a.thr)) * z;
+    // Invariant: the cut key lies in [lo, hi); mass(key >= hi) = base < target.
+    uint32_t lo = 0, hi = kmax + 1;
+    double base = 0.0;
+    int ncand = -1;  // -1: scan the whole row
+    for (int it = 0; hi - lo > 1; ++it) {
+      const uint32_t mid = lo + ((hi - lo) >> 1);
+      double up = 0.0;
+      if (ncand < 0) {
+        for (int c = lane; c < Nb; c += 32) {
+          const float e = ebuf[c];
+          const uint32_t k = __float_as_uint(e);
+          if (k >= mid && k < hi) up += static_cast<double>(e);
+        }
+      } else {
+        for (int i = lane; i < ncand; i += 32) {
+          const uint32_t k = cand_key[i];
+          if (k >= mid && k < hi) up += static_cast<double>(__uint_as_float(k));
+        }
+      }
+      up = warp_sum(up);
+      if (base + up >= target) {
+        lo = mid;
+      } else {
+        base += up;
+        hi = mid;
+      }
+      if (ncand < 0 && it >= 5) {
+        int cnt = 0;
+        for (int c = lane; c < Nb; c += 32) {
+          const uint32_t k = __float_as_uint(ebuf[c]);
+          cnt += (k >= lo && k < hi);
+        }
+        cnt = warp_sum_i(cnt);
+        if (cnt <= kCand) {
+          int pos = 0;
+          for (int c0 = 0; c0 < Nb; c0 += 32) {
+            const int c = c0 + lane;
+            const uint32_t k = c < Nb ? __float_as_uint(ebuf[c]) : 0u;
+            const bool in = c < Nb && k >= lo && k < hi;
+            const uint32_t m = __ballot_sync(0xFFFFFFFFu, in);
+            if (in) {
+              const int p = pos + __popc(m & ((1u << lane) - 1u));
+              cand_key[p] = k;
+              cand_idx[p] = c;
+            }
+            pos += __popc(m);
+          }
+          ncand = pos;
+          __syncwarp();
+        }
+      }
+    }
+    vkey = lo;
+    if (vkey == 0u) {
+      keep_all = true;  // the sums never reach 1 - thr: keep every block
+    } else {
+      const double v = static_cast<double>(__uint_as_float(vkey));
+      int j = static_cast<int>(ceil((target - base) / v));
+      if (j < 1) j = 1;
+      while (j > 1 && base + (j - 1) * v >= target) --j;
+      while (base + j * v < target && j < Nb) ++j;
+      need_ties = j;
+    }
+  }
+
+  // kept bits: above the cut, the first need_ties equal keys in index order,
+  // or the STA window
+  int ties_seen = 0, count = 0;
+  uint32_t *out = a.bits + grow * a.words;
+  for (int w = 0; w < a.words; ++w) {
+    const int c = w * 32 + lane;
+    const bool valid = c < Nb;
+    const uint32_t k = valid ? __float_as_uint(ebuf[c]) : 0u;
+    bool kept = valid && (keep_all || k > vkey);
+    const bool tie = valid && !keep_all && k == vkey;
+    const uint32_t tm = __ballot_sync(0xFFFFFFFFu, tie);
+    if (tie && ties_seen + __popc(tm & ((1u << lane) - 1u)) < need_ties) kept = true;
+    ties_seen += __popc(tm);
+    if (valid && a.use_sta && sta_keep(r, c, a)) kept = true;
+    const uint32_t word = __ballot_sync(0xFFFFFFFFu, kept);
+    if (lane == 0) out[w] = word;
+    count += __popc(word);
+  }
+  if (lane == 0) a.counts[grow] = count;
+  __syncwarp();
+}
+
+__global__ void __launch_bounds__(kThreads, 1) mask_select_kernel(const MaskArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  double *sQ = reinterpret_cast<double *>(smem_raw);
+  const int ld = a.d + kPad;
+  double *sK = sQ + kRT * ld;
+  __shared__ double sRed[kRT][4];
+  __shared__ double sTileMax[kRT];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, tq = lane & 3;
+  const int wm = warp >> 2, wn = warp & 3;
+  float *slab = a.slab + static_cast<int64_t>(blockIdx.x) * kRT * a.ld_slab;
+  double *tmax = a.tmax + static_cast<int64_t>(blockIdx.x) * kRT * a.ntiles;
+  const int vec_per_row = a.d / 2;  // 16-byte chunks per fp64 row
+
+  for (int64_t item = blockIdx.x; item < a.items; item += gridDim.x) {
+    const int64_t bh = item / a.tiles_per_head;
+    const int r0 = static_cast<int>(item % a.tiles_per_head) * kRT;
+    const double *qsrc = a.qp + (bh * a.Nb + r0) * a.d;
+    const double *ksrc = a.kp + bh * a.Nb * a.d;
+
+    // ---- phase A: scores, tile maxima, exp2 slab
+    for (int i = tid; i < kRT * vec_per_row; i += kThreads) {
+      const int row = i / vec_per_row, ch = i % vec_per_row;
+      const bool ok = r0 + row < a.Nb;
+      cp_async16(sQ + row * ld + ch * 2, ok ? qsrc + row * a.d + ch * 2 : a.qp, ok);
+    }
+    for (int ct = 0; ct < a.ntiles; ++ct) {
+      const int c0 = ct * kCT;
+      for (int i = tid; i < kCT * vec_per_row; i += kThreads) {
+        const int row = i / vec_per_row, ch = i % vec_per_row;
+        const bool ok = c0 + row < a.Nb;
+        cp_async16(sK + row * ld + ch * 2,
+                   ok ? ksrc + static_cast<int64_t>(c0 + row) * a.d + ch * 2 : a.kp, ok);
+      }
+      cp_async_wait_all();
+      __syncthreads();
+
+      double acc[4][4][2];
+#pragma unroll
+      for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni) acc[mi][ni][0] = acc[mi][ni][1] = 0.0;
+      const double *qa = sQ + (wm * 32 + g) * ld + tq;
+      const double *kb = sK + (wn * 32 + g) * ld + tq;
+#pragma unroll 2
+      for (int k = 0; k < a.d; k += 4) {
+        double af[4], bf[4];
+#pragma unroll
+        for (int mi = 0; mi < 4; ++mi) af[mi] = qa[mi * 8 * ld + k];
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni) bf[ni] = kb[ni * 8 * ld + k];
+#pragma unroll
+        for (int mi = 0; mi < 4; ++mi)
+#pragma unroll
+          for (int ni = 0; ni < 4; ++ni) dmma(acc[mi][ni], af[mi], bf[ni]);
+      }
+      // scaled log2 scores; columns past Nb do not exist
+#pragma unroll
+      for (int mi = 0; mi < 4; ++mi) {
+        double m = -INFINITY;
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int col = c0 + wn * 32 + ni * 8 + 2 * tq + j;
+            acc[mi][ni][j] = col < a.Nb ? acc[mi][ni][j] * a.c : -INFINITY;
+            m = fmax(m, acc[mi][ni][j]);
+          }
+        m = fmax(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+        m = fmax(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+        if (tq == 0) sRed[wm * 32 + mi * 8 + g][wn] = m;
+      }
+      __syncthreads();
+      if (tid < kRT) {
+        const double m = fmax(fmax(sRed[tid][0], sRed[tid][1]), fmax(sRed[tid][2], sRed[tid][3]));
+        sTileMax[tid] = m;
+        tmax[tid * a.ntiles + ct] = m;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int mi = 0; mi < 4; ++mi) {
+        const int row = wm * 32 + mi * 8 + g;
+        const double m = sTileMax[row];
+#pragma unroll
+        for (int ni = 0; ni < 4; ++ni) {
+          const int col = c0 + wn * 32 + ni * 8 + 2 * tq;
+          if (col < a.Nb) {
+            float2 e;
+            e.x = exp2_split(acc[mi][ni][0] - m);
+            e.y = exp2_split(acc[mi][ni][1] - m);
+            *reinterpret_cast<float2 *>(slab + row * a.ld_slab + col) = e;
+          }
+        }
+      }
+      __syncthreads();  // sK is overwritten by the next tile
+    }
+    __threadfence_block();
+    __syncthreads();
+
+    // ---- phase B: one warp per row
+    unsigned char *wbase = smem_raw + warp * (static_cast<size_t>(a.Nb) * 4 + kCand * 8 +
+                                              static_cast<size_t>(a.ntiles) * 8 + 16);
+    float *ebuf = reinterpret_cast<float *>(wbase);
+    uint32_t *cand_key = reinterpret_cast<uint32_t *>(ebuf + a.Nb);
+    int32_t *cand_idx = reinterpret_cast<int32_t *>(cand_key + kCand);
+    double *tscale = reinterpret_cast<double *>(
+        (reinterpret_cast<uintptr_t>(cand_idx + kCand) + 15) & ~static_cast<uintptr_t>(15));
+    for (int row = warp; row < kRT; row += kWarps) {
+      const int r = r0 + row;
+      if (r >= a.Nb) break;
+      select_row(a, bh * a.Nb + r, r, slab + row * a.ld_slab, tmax + row * a.ntiles, ebuf,
+                 cand_key, cand_idx, tscale);
+    }
+    __syncthreads();  // smem and slab are reused by the next item
+  }
+}
+
+// Exclusive scan of n counts into row_ptr[0..n] by one CTA of 1024 threads.
+__global__ void __launch_bounds__(1024) scan_counts_kernel(const int32_t *__restrict__ counts,
+                                                           int64_t n,
+                                                           int64_t *__restrict__ row_ptr) {
+  __shared__ int64_t warp_tot[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t per = (n + 1023) / 1024;
+  const int64_t b = tid * per, e = b + per < n ? b + per : n;
+  int64_t s = 0;
+  for (int64_t i = b; i < e; ++i) s += counts[i];
+  int64_t x = s;  // inclusive warp scan
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int64_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int64_t w = warp_tot[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t y = __shfl_up_sync(0xFFFFFFFFu, w, o);
+      if (lane >= o) w += y;
+    }
+    warp_tot[lane] = w;
+  }
+  __syncthreads();
+  int64_t run = x - s + (warp ? warp_tot[warp - 1] : 0);
+  for (int64_t i = b; i < e; ++i) {
+    row_ptr[i] = run;
+    run += counts[i];
+  }
+  if (tid == 1023) row_ptr[n] = warp_tot[31];
+}
+
+__global__ void __launch_bounds__(256) expand_bits_kernel(const uint32_t *__restrict__ bits,
+                                                          int words, int64_t rows,
+                                                          const int64_t *__restrict__ row_ptr,
+                                                          int32_t *__restrict__ col_idx) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < rows;
+       r += warps) {
+    int64_t pos = row_ptr[r];
+    const uint32_t *rb = bits + r * words;
+    for (int w0 = 0; w0 < words; w0 += 32) {
+      const uint32_t mine = w0 + lane < words ? rb[w0 + lane] : 0u;
+      for (int i = 0; i < 32 && w0 + i < words; ++i) {
+        const uint32_t word = __shfl_sync(0xFFFFFFFFu, mine, i);
+        if ((word >> lane) & 1u) col_idx[pos + __popc(word & ((1u << lane) - 1u))] = (w0 + i) * 32 + lane;
+        pos += __popc(word);
+      }
+    }
+  }
+}
+
+struct MaskLayout {
+  int ld_slab, ntiles, words, grid;
+  size_t slab_off, tmax_off, bits_off, counts_off, total;
+  size_t smem;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+MaskLayout mask_layout(const Geometry &g, int grid) {
+  MaskLayout L;
+  L.ld_slab = static_cast<int>((g.Nb + 3) & ~3LL);
+  L.ntiles = static_cast<int>((g.Nb + kCT - 1) / kCT);
+  L.words = static_cast<int>((g.Nb + 31) / 32);
+  L.grid = grid;
+  size_t off = 0;
+  L.slab_off = off;
+  off = align256(off + static_cast<size_t>(kMaxGrid) * kRT * L.ld_slab * 4);
+  L.tmax_off = off;
+  off = align256(off + static_cast<size_t>(kMaxGrid) * kRT * L.ntiles * 8);
+  L.bits_off = off;
+  off = align256(off + static_cast<size_t>(g.BH * g.Nb) * L.words * 4);
+  L.counts_off = off;
+  off = align256(off + static_cast<size_t>(g.BH * g.Nb) * 4);
+  L.total = off;
+  const size_t phase_a = static_cast<size_t>(kRT + kCT) * (g.d + kPad) * 8;
+  const size_t phase_b =
+      static_cast<size_t>(kWarps) * (static_cast<size_t>(g.Nb) * 4 + kCand * 8 + L.ntiles * 8 + 16);
+  L.smem = phase_a > phase_b ? phase_a : phase_b;
+  return L;
+}
+
+}  // namespace
+
+size_t block_mask_workspace_bytes(const Geometry &g) { return mask_layout(g, kMaxGrid).total; }
+
+size_t block_mask_smem_bytes(const Geometry &g) { return mask_layout(g, kMaxGrid).smem; }
+
+cudaError_t launch_block_mask(const double *qp, const double *kp, const Geometry &g,
+                              const vsa_mask_params &p, int64_t *row_ptr, int32_t *col_idx,
+                              int32_t *kept_count, void *ws, unsigned *err, cudaStream_t st) {
+  (void)err;
+  const int64_t rows = g.BH * g.Nb;
+  if (rows == 0) {
+    return cudaMemsetAsync(row_ptr, 0, sizeof(int64_t), st);
+  }
+  const int64_t tiles_per_head = (g.Nb + kRT - 1) / kRT;
+  const int64_t items = g.BH * tiles_per_head;
+  int grid = num_sms();
+  if (grid > kMaxGrid) grid = kMaxGrid;
+  if (items < grid) grid = static_cast<int>(items);
+  MaskLayout L = mask_layout(g, grid);
+  unsigned char *w = static_cast<unsigned char *>(ws);
+  MaskArgs a;
+  a.qp = qp; a.kp = kp; a.BH = g.BH; a.Nb = static_cast<int>(g.Nb); a.d = g.d;
+  a.Hb = g.Hb; a.Wb = g.Wb; a.thr = p.thr; a.use_sta = p.use_sta != 0;
+  a.rt = p.sta_t; a.rh = p.sta_h; a.rw = p.sta_w;
+  a.c = 1.4426950408889634 / std::sqrt(static_cast<double>(g.d));
+  a.slab = reinterpret_cast<float *>(w + L.slab_off);
+  a.tmax = reinterpret_cast<double *>(w + L.tmax_off);
+  a.ld_slab = L.ld_slab; a.ntiles = L.ntiles;
+  a.bits = reinterpret_cast<uint32_t *>(w + L.bits_off);
+  a.words = L.words;
+  a.counts = kept_count ? kept_count : reinterpret_cast<int32_t *>(w + L.counts_off);
+  a.items = items; a.tiles_per_head = tiles_per_head;
+  cudaError_t e = cudaFuncSetAttribute(mask_select_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(L.smem));
+  if (e != cudaSuccess) return e;
+  mask_select_kernel<<<grid, kThreads, L.smem, st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  scan_counts_kernel<<<1, 1024, 0, st>>>(a.counts, rows, row_ptr);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int64_t want = (rows + 7) / 8;
+  const int eg = static_cast<int>(want < 16LL * num_sms() ? want : 16LL * num_sms());
+  expand_bits_kernel<<<eg, 256, 0, st>>>(a.bits, a.words, rows, row_ptr, col_idx);
+  return cudaGetLastError();
+}
+
+}  // namespace vsa

@@ -1,0 +1,235 @@
+// vsa_api.cu -- the extern "C" entry points of libvsa (declared in
+// include/vsa.h): host-side validation, launch, error reporting.
+#include "vsa_internal.h"
+
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+namespace vsa {
+size_t block_mask_smem_bytes(const Geometry &g);
+}
+
+namespace {
+
+thread_local std::string g_last_error;
+
+// Per-device error word written by bounded device waits (bit flags).
+__device__ unsigned g_device_error;
+
+constexpr int kMaxDevices = 64;
+constexpr size_t kMaxSmem = 232448;  // opt-in dynamic shared memory per block on sm_100
+
+vsa_status fail(vsa_status st, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+vsa_status cuda_fail(cudaError_t e, const char *what) {
+  return fail(VSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+unsigned *device_error_word(cudaError_t *err) {
+  static unsigned *addr[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if ((*err = cudaGetDevice(&dev)) != cudaSuccess) return nullptr;
+  if (dev < 0 || dev >= kMaxDevices) {
+    *err = cudaErrorInvalidDevice;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void *p = nullptr;
+    if ((*err = cudaGetSymbolAddress(&p, g_device_error)) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<unsigned *>(p);
+  }
+  return addr[dev];
+}
+
+// Shape checks shared by every entry point.
+vsa_status check_shape(const vsa_shape &s) {
+  if (s.B < 0 || s.heads < 0 || s.T < 0 || s.H < 0 || s.W < 0 || s.d <= 0 || s.P <= 0)
+    return fail(VSA_ERR_INVALID_ARG, "negative or zero size in shape (B=%d heads=%d T=%d H=%d W=%d d=%d P=%d)",
+                s.B, s.heads, s.T, s.H, s.W, s.d, s.P);
+  if (s.P * s.P != 64)
+    return fail(VSA_ERR_UNSUPPORTED, "patch size P=%d: blocks must be P*P = 64 tokens (P = 8)", s.P);
+  if (s.H % s.P || s.W % s.P)
+    return fail(VSA_ERR_UNSUPPORTED, "grid H=%d W=%d is not a multiple of P=%d", s.H, s.W, s.P);
+  if (s.d != 64 && s.d != 128)
+    return fail(VSA_ERR_UNSUPPORTED, "head dim d=%d: only 64 and 128 are implemented", s.d);
+  const long long n = 1LL * s.B * s.heads * s.T * s.H * s.W;
+  if (n > (1LL << 31) - 1)
+    return fail(VSA_ERR_UNSUPPORTED, "B*heads*N = %lld exceeds 2^31-1 tokens", n);
+  return VSA_OK;
+}
+
+bool empty(const vsa_shape &s) { return 1LL * s.B * s.heads * s.T * s.H * s.W == 0; }
+
+}  // namespace
+
+namespace vsa {
+int num_sms() {
+  static int cache[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+}  // namespace vsa
+
+extern "C" {
+
+const char *vsa_version(void) { return "0.1.0"; }
+
+const char *vsa_last_error(void) { return g_last_error.c_str(); }
+
+static vsa_status permute(const void *src, void *dst, vsa_shape s, void *stream, bool inverse) {
+  vsa_status st = check_shape(s);
+  if (st != VSA_OK) return st;
+  if (empty(s)) return VSA_OK;
+  if (!src || !dst) return fail(VSA_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(src) || !aligned16(dst))
+    return fail(VSA_ERR_UNSUPPORTED, "tensor pointers must be 16-byte aligned");
+  const vsa::Geometry g = vsa::geometry(s);
+  const size_t bytes = static_cast<size_t>(g.BH * g.N) * g.d * 2;
+  const char *a = static_cast<const char *>(src);
+  const char *b = static_cast<const char *>(dst);
+  if (a < b + bytes && b < a + bytes)
+    return fail(VSA_ERR_INVALID_ARG, "source and destination overlap");
+  cudaError_t e = vsa::launch_fractal_permute(src, dst, g, inverse,
+                                              static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? VSA_OK : cuda_fail(e, "fractal permute launch");
+}
+
+vsa_status vsa_fractal_flatten(const void *x, void *y, vsa_shape s, void *stream) {
+  return permute(x, y, s, stream, false);
+}
+
+vsa_status vsa_fractal_unflatten(const void *y, void *x, vsa_shape s, void *stream) {
+  return permute(y, x, s, stream, true);
+}
+
+vsa_status vsa_pool_qk(const void *qf, const void *kf, double *qp, double *kp, vsa_shape s,
+                       void *stream) {
+  vsa_status st = check_shape(s);
+  if (st != VSA_OK) return st;
+  if (empty(s)) return VSA_OK;
+  if (!qf || !kf || !qp || !kp) return fail(VSA_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(qf) || !aligned16(kf) || !aligned16(qp) || !aligned16(kp))
+    return fail(VSA_ERR_UNSUPPORTED, "tensor pointers must be 16-byte aligned");
+  cudaError_t e = vsa::launch_pool_qk(qf, kf, qp, kp, vsa::geometry(s),
+                                      static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? VSA_OK : cuda_fail(e, "pool launch");
+}
+
+size_t vsa_block_mask_workspace_size(vsa_shape s) {
+  if (check_shape(s) != VSA_OK) return 0;
+  return vsa::block_mask_workspace_bytes(vsa::geometry(s));
+}
+
+vsa_status vsa_block_mask(const double *qp, const double *kp, vsa_shape s, vsa_mask_params p,
+                          int64_t *row_ptr, int32_t *col_idx, int64_t col_capacity,
+                          int32_t *kept_count, void *workspace, size_t workspace_bytes,
+                          void *stream) {
+  vsa_status st = check_shape(s);
+  if (st != VSA_OK) return st;
+  if (!(p.thr >= 0.0f && p.thr < 1.0f))
+    return fail(VSA_ERR_INVALID_ARG, "thr=%g outside [0, 1)", static_cast<double>(p.thr));
+  if (p.use_sta && (p.sta_t < 0 || p.sta_h < 0 || p.sta_w < 0))
+    return fail(VSA_ERR_INVALID_ARG, "negative STA radius (%d, %d, %d)", p.sta_t, p.sta_h, p.sta_w);
+  if (!row_ptr) return fail(VSA_ERR_INVALID_ARG, "null row_ptr");
+  const vsa::Geometry g = vsa::geometry(s);
+  const int64_t need = g.BH * g.Nb * g.Nb;
+  if (col_capacity < need)
+    return fail(VSA_ERR_CAPACITY, "col_capacity %lld < B*heads*Nb*Nb = %lld",
+                static_cast<long long>(col_capacity), static_cast<long long>(need));
+  if (empty(s)) {
+    cudaError_t e = cudaMemsetAsync(row_ptr, 0, sizeof(int64_t), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? VSA_OK : cuda_fail(e, "row_ptr reset");
+  }
+  if (!qp || !kp || !col_idx || !workspace)
+    return fail(VSA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(qp) || !aligned16(kp) || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      (reinterpret_cast<uintptr_t>(row_ptr) & 7u) || (reinterpret_cast<uintptr_t>(col_idx) & 3u) ||
+      (kept_count && (reinterpret_cast<uintptr_t>(kept_count) & 3u)))
+    return fail(VSA_ERR_UNSUPPORTED, "misaligned pointer (tensors 16 B, workspace 256 B)");
+  const size_t ws = vsa::block_mask_workspace_bytes(g);
+  if (workspace_bytes < ws)
+    return fail(VSA_ERR_CAPACITY, "block mask workspace %zu < %zu bytes", workspace_bytes, ws);
+  if (vsa::block_mask_smem_bytes(g) > kMaxSmem)
+    return fail(VSA_ERR_UNSUPPORTED, "Nb=%lld blocks per head exceeds the mask kernel's shared memory",
+                static_cast<long long>(g.Nb));
+  cudaError_t e;
+  unsigned *err = device_error_word(&e);
+  if (!err) return cuda_fail(e, "device error word");
+  e = vsa::launch_block_mask(qp, kp, g, p, row_ptr, col_idx, kept_count, workspace, err,
+                             static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? VSA_OK : cuda_fail(e, "block mask launch");
+}
+
+size_t vsa_sparse_attn_workspace_size(vsa_shape s) {
+  if (check_shape(s) != VSA_OK) return 0;
+  return vsa::sparse_attn_workspace_bytes(vsa::geometry(s));
+}
+
+vsa_status vsa_sparse_attn_fwd(const void *qf, const void *kf, const void *vf,
+                               const int64_t *row_ptr, const int32_t *col_idx, vsa_shape s,
+                               float scale, void *o, float *lse, void *workspace,
+                               size_t workspace_bytes, void *stream) {
+  vsa_status st = check_shape(s);
+  if (st != VSA_OK) return st;
+  if (empty(s)) return VSA_OK;
+  if (!qf || !kf || !vf || !row_ptr || !col_idx || !o || !lse || !workspace)
+    return fail(VSA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(qf) || !aligned16(kf) || !aligned16(vf) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      (reinterpret_cast<uintptr_t>(row_ptr) & 7u) || (reinterpret_cast<uintptr_t>(col_idx) & 3u))
+    return fail(VSA_ERR_UNSUPPORTED, "misaligned pointer (tensors 16 B, workspace 256 B)");
+  if (!(scale == scale)) return fail(VSA_ERR_INVALID_ARG, "scale is NaN");
+  const vsa::Geometry g = vsa::geometry(s);
+  const size_t ws = vsa::sparse_attn_workspace_bytes(g);
+  if (workspace_bytes < ws)
+    return fail(VSA_ERR_CAPACITY, "attention workspace %zu < %zu bytes", workspace_bytes, ws);
+  if (scale <= 0.0f) scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(s.d)));
+  cudaError_t e;
+  unsigned *err = device_error_word(&e);
+  if (!err) return cuda_fail(e, "device error word");
+  const char *why = nullptr;
+  e = vsa::launch_sparse_attn(qf, kf, vf, row_ptr, col_idx, g, scale, o, lse, workspace, err,
+                              static_cast<cudaStream_t>(stream), &why);
+  if (e != cudaSuccess)
+    return why ? fail(VSA_ERR_UNSUPPORTED, "%s", why) : cuda_fail(e, "sparse attention launch");
+  return VSA_OK;
+}
+
+vsa_status vsa_device_status(void *stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  unsigned *err = device_error_word(&e);
+  if (!err) return cuda_fail(e, "device error word");
+  unsigned v = 0;
+  if ((e = cudaMemcpy(&v, err, sizeof v, cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(e, "read device error word");
+  if (v == 0) return VSA_OK;
+  const unsigned zero = 0;
+  if ((e = cudaMemcpy(err, &zero, sizeof zero, cudaMemcpyHostToDevice)) != cudaSuccess)
+    return cuda_fail(e, "clear device error word");
+  return fail(VSA_ERR_DEVICE_TIMEOUT,
+              "device error word 0x%x (1: TMA wait, 2: MMA wait, 4: softmax wait, 8: bad block index)",
+              v);
+}
+
+}  // extern "C"

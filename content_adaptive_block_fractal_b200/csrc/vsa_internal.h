@@ -1,0 +1,51 @@
+// vsa_internal.h -- launch functions shared between the C-ABI layer and the
+// kernel translation units of libvsa.  Host-side only; not part of the ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/vsa.h"
+
+namespace vsa {
+
+struct Geometry {
+  int64_t BH;   // batch * heads
+  int64_t N;    // tokens per (batch, head)
+  int64_t Nb;   // 64-token blocks per (batch, head)
+  int T, H, W, d, P, Hb, Wb;
+};
+
+inline Geometry geometry(const vsa_shape &s) {
+  Geometry g;
+  g.BH = static_cast<int64_t>(s.B) * s.heads;
+  g.N = static_cast<int64_t>(s.T) * s.H * s.W;
+  g.Nb = g.N / 64;
+  g.T = s.T; g.H = s.H; g.W = s.W; g.d = s.d; g.P = s.P;
+  g.Hb = s.P ? s.H / s.P : 0;
+  g.Wb = s.P ? s.W / s.P : 0;
+  return g;
+}
+
+int num_sms();   // SM count of the current device (cached per device)
+
+cudaError_t launch_fractal_permute(const void *src, void *dst, const Geometry &g, bool inverse,
+                                   cudaStream_t st);
+cudaError_t launch_pool_qk(const void *qf, const void *kf, double *qp, double *kp,
+                           const Geometry &g, cudaStream_t st);
+
+// Block mask: workspace carve-up and launch.
+size_t block_mask_workspace_bytes(const Geometry &g);
+cudaError_t launch_block_mask(const double *qp, const double *kp, const Geometry &g,
+                              const vsa_mask_params &p, int64_t *row_ptr, int32_t *col_idx,
+                              int32_t *kept_count, void *ws, unsigned *err, cudaStream_t st);
+
+// Sparse attention: workspace carve-up and launch.
+size_t sparse_attn_workspace_bytes(const Geometry &g);
+cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
+                               const int64_t *row_ptr, const int32_t *col_idx,
+                               const Geometry &g, float scale, void *o, float *lse, void *ws,
+                               unsigned *err, cudaStream_t st, const char **why);
+
+}  // namespace vsa

@@ -1,0 +1,148 @@
+/*
+ * vsa.h -- C ABI of the content-adaptive block-sparse video attention library
+ * (libvsa.so, hand-written CUDA for sm_100a).
+ *
+ * The method (NABLA: Neighborhood Adaptive Block-Level Attention, gist.science
+ * summary of arXiv 2507.13546, "Methodology" items 1-3; the same top-p block
+ * selection appears in Sparse VideoGen2, arXiv 2505.18875 summary, section 2B,
+ * and in DynamicRad's dynamic-threshold mode, arXiv 2604.20470 summary,
+ * section 2A) runs in five steps, one entry point each:
+ *   1. vsa_fractal_flatten       reorder a T x H x W token grid so each P x P
+ *                                spatial patch is a contiguous run of 64 tokens;
+ *   2. vsa_pool_qk               mean-pool Q and K over those 64-token blocks;
+ *   3.-4. vsa_block_mask         reduced softmax of pooled scores, per-row CDF
+ *                                (top-p) selection, optional union with a
+ *                                sliding-tile (STA) window, compacted to CSR;
+ *   5. vsa_sparse_attn_fwd       attention forward over the kept 64 x 64 tiles,
+ *                                returning O and the log-sum-exp;
+ *   and vsa_fractal_unflatten    to bring O back to raster order.
+ *
+ * Conventions shared by every entry point
+ *   - Pointers marked "device" are CUDA device pointers on the current device;
+ *     the caller allocates and frees every buffer, the library allocates
+ *     nothing.  Tensors are dense and contiguous, bf16 = IEEE bfloat16 stored
+ *     as uint16, layout [B, heads, N, d] (d fastest).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is
+ *     asynchronous on that stream and never synchronises the host.
+ *   - Arguments are validated on the host before anything is launched; a
+ *     non-OK status means nothing was enqueued.  vsa_last_error() returns a
+ *     message for the last non-OK status of the calling thread.
+ *   - Kernels never trap.  A bounded device-side wait that gives up records a
+ *     code in a per-device error word; vsa_device_status() synchronises the
+ *     stream, reports and clears it.
+ */
+#ifndef VSA_H
+#define VSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    VSA_OK = 0,
+    VSA_ERR_INVALID_ARG = 1,     /* null pointer, negative size, thr outside [0,1) ... */
+    VSA_ERR_UNSUPPORTED = 2,     /* valid but not implemented: d not 64/128, P*P != 64,
+                                    H or W not a multiple of P, misaligned pointer */
+    VSA_ERR_CAPACITY = 3,        /* an output or workspace buffer is too small */
+    VSA_ERR_CUDA = 4,            /* a CUDA runtime call failed (message has the reason) */
+    VSA_ERR_DEVICE_TIMEOUT = 5   /* a device-side wait gave up (see vsa_device_status) */
+} vsa_status;
+
+/* Token grid and head geometry.  N = T*H*W tokens per (batch, head);
+ * blocks of P*P = 64 tokens; Nb = N/64 blocks per (batch, head). */
+typedef struct {
+    int32_t B, heads, T, H, W, d, P;
+} vsa_shape;
+
+/* Block-selection parameters.
+ * thr     : CDF threshold in [0, 1).  Each row keeps the smallest set of its
+ *           highest-probability blocks whose mass reaches 1 - thr (equal
+ *           probabilities: lower block index first); thr = 0 keeps all blocks.
+ * use_sta : non-zero to union the kept set with the STA window.
+ * sta_t, sta_h, sta_w : STA radii in frames, patch rows and patch columns
+ *           (Chebyshev window, clipped at the grid edges); >= 0. */
+typedef struct {
+    float thr;
+    int32_t use_sta;
+    int32_t sta_t, sta_h, sta_w;
+} vsa_mask_params;
+
+/* 1. Fractal flattening (NABLA, Methodology item 1).
+ * y[b,h,f(n),:] = x[b,h,n,:] with raster n = (t*H + y)*W + x and
+ * f(n) = t*H*W + ((y/P)*(W/P) + x/P)*P*P + (y%P)*P + x%P.
+ * x, y : device bf16 [B,heads,N,d], must not overlap.  P must be 8. */
+vsa_status vsa_fractal_flatten(const void *x, void *y, vsa_shape s, void *stream);
+
+/* Inverse permutation: x[b,h,n,:] = y[b,h,f(n),:]. */
+vsa_status vsa_fractal_unflatten(const void *y, void *x, vsa_shape s, void *stream);
+
+/* 2. Block mean pooling (NABLA, Methodology item 2, "downsampling").
+ * qp[b,h,r,:] = (1/64) * sum_{i<64} qf[b,h,64r+i,:], same for k.
+ * qf, kf : device bf16 [B,heads,N,d] in flattened order.
+ * qp, kp : device fp64 [B,heads,Nb,d].  The sum of 64 bf16 values is exact in
+ *          fp64 and the division by 64 is exact, so each pooled value is the
+ *          exact block mean. */
+vsa_status vsa_pool_qk(const void *qf, const void *kf, double *qp, double *kp,
+                       vsa_shape s, void *stream);
+
+/* 3.-4. Block mask (NABLA, Methodology items 2-3).
+ * For every (b, h) and query block r: A[r,:] = softmax(qp_r . kp_c / sqrt(d))
+ * over the Nb key blocks c, CDF selection at thr, union with the STA window
+ * when enabled, and the kept blocks listed in ascending order:
+ *   row_ptr : device int64 [B*heads*Nb + 1]; row g = (b*heads + h)*Nb + r;
+ *             row_ptr[0] = 0, row_ptr[g+1] - row_ptr[g] = kept count of row g.
+ *   col_idx : device int32 [col_capacity]; key block indices within the head.
+ *             col_capacity must be >= B*heads*Nb*Nb (the worst case), so no
+ *             host read-back of the kept count is ever needed.
+ *   kept_count : optional device int32 [B*heads*Nb] (may be NULL).
+ *   workspace  : device scratch of at least vsa_block_mask_workspace_size(s)
+ *                bytes, 256-byte aligned; its contents need no initialisation.
+ * Pooled scores are formed in fp64; probabilities carry a relative error
+ * below 1e-6, so only rows whose cut lies within that of 1 - thr (or of a tie
+ * across the cut) can differ from exact arithmetic. */
+size_t vsa_block_mask_workspace_size(vsa_shape s);
+vsa_status vsa_block_mask(const double *qp, const double *kp, vsa_shape s,
+                          vsa_mask_params p, int64_t *row_ptr, int32_t *col_idx,
+                          int64_t col_capacity, int32_t *kept_count,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/* 5. Block-sparse attention forward (NABLA, Methodology item 2, "expansion":
+ * the block mask decides which 64 x 64 tiles are computed; Sparse VideoGen2
+ * section 2C: dense loads of contiguous query blocks, sparse loads of K/V).
+ * For each query token of query block r of head (b,h), softmax attention over
+ * the keys of blocks col_idx[row_ptr[g] .. row_ptr[g+1]), g = (b*heads+h)*Nb + r:
+ *   O = sum_j softmax_j(scale * q . k_j) v_j,  LSE = ln sum_j exp(scale * q . k_j).
+ * qf, kf, vf : device bf16 [B,heads,N,d], flattened order.
+ * row_ptr, col_idx : as produced by vsa_block_mask (any valid CSR: columns
+ *             strictly ascending and < Nb within each row).  An empty row
+ *             gives O = 0 and LSE = -inf.
+ * scale     : logit scale; <= 0 selects 1/sqrt(d).
+ * o         : device bf16 [B,heads,N,d];  lse : device fp32 [B,heads,N].
+ * workspace : device scratch of at least vsa_sparse_attn_workspace_size(s)
+ *             bytes, 256-byte aligned (work list of the persistent scheduler). */
+size_t vsa_sparse_attn_workspace_size(vsa_shape s);
+vsa_status vsa_sparse_attn_fwd(const void *qf, const void *kf, const void *vf,
+                               const int64_t *row_ptr, const int32_t *col_idx,
+                               vsa_shape s, float scale, void *o, float *lse,
+                               void *workspace, size_t workspace_bytes,
+                               void *stream);
+
+/* Message for the last non-OK status returned to the calling thread. */
+const char *vsa_last_error(void);
+
+/* Synchronises `stream`, then reports and clears the device error word of the
+ * current device: VSA_OK, or VSA_ERR_DEVICE_TIMEOUT if a kernel gave up a
+ * bounded wait since the last call, or VSA_ERR_CUDA if the stream failed. */
+vsa_status vsa_device_status(void *stream);
+
+/* Library version, "major.minor.patch". */
+const char *vsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VSA_H */

@@ -209,6 +209,8 @@ static int ranked_cmp(const void *a, const void *b)
 void oracle_select_row(const double *a, int n, double thr, uint8_t *keep,
                        double *diag)
 {
+    if (n <= 0)
+        return;
     ranked *r = (ranked *)malloc(sizeof(ranked) * (size_t)n);
     for (int c = 0; c < n; ++c) {
         r[c].p = a[c];

@@ -1,0 +1,76 @@
+"""The C ABI library loads, exports every symbol include/vsa.h declares, and
+rejects bad arguments on the host before any CUDA call (runs without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from content_adaptive_block_fractal_b200 import _lib, Shape, MaskParams
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "vsa.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(vsa_\w+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert declared_functions() == sorted(_lib.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = _lib.load()
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    assert L.vsa_version().decode().count(".") == 2
+
+
+def _call_flatten(shape, x=1 << 12, y=1 << 20):
+    L = _lib.load()
+    return L.vsa_fractal_flatten(ctypes.c_void_p(x), ctypes.c_void_p(y), shape, None)
+
+
+@pytest.mark.parametrize("shape,status", [
+    (Shape(1, 2, 4, 16, 16, 96), 2),     # d not 64/128
+    (Shape(1, 2, 4, 16, 16, 64, P=4), 2),  # P*P != 64
+    (Shape(1, 2, 4, 12, 16, 64), 2),     # H not a multiple of P
+    (Shape(-1, 2, 4, 16, 16, 64), 1),    # negative size
+])
+def test_shape_validation(shape, status):
+    assert _call_flatten(shape.c()) == status
+    assert len(_lib.load().vsa_last_error()) > 0
+
+
+def test_null_and_misaligned_pointers_rejected():
+    s = Shape(1, 2, 4, 16, 16, 64).c()
+    assert _call_flatten(s, x=0) == 1
+    assert _call_flatten(s, x=(1 << 12) + 8) == 2
+    assert _call_flatten(s, x=1 << 12, y=(1 << 12) + 64) == 1   # overlapping buffers
+
+
+def test_mask_parameter_validation():
+    L = _lib.load()
+    s = Shape(1, 2, 4, 16, 16, 64)
+    P = ctypes.c_void_p
+    def call(params, cap=2 * 16 * 16, ws=1 << 30):
+        return L.vsa_block_mask(P(1 << 12), P(1 << 16), s.c(), params.c(), P(1 << 20), P(1 << 24),
+                                cap, None, P(1 << 28), ws, None)
+    assert call(MaskParams(1.0)) == 1
+    assert call(MaskParams(-0.1)) == 1
+    assert call(MaskParams(0.2, True, (1, -1, 1))) == 1
+    assert call(MaskParams(0.2), cap=2 * 16 * 16 - 1) == 3          # CSR capacity
+    assert call(MaskParams(0.2), ws=16) == 3                        # workspace
+    assert _lib.load().vsa_block_mask_workspace_size(Shape(1, 1, 1, 8, 8, 96).c()) == 0
+
+
+def test_attention_workspace_validation():
+    L = _lib.load()
+    s = Shape(1, 2, 4, 16, 16, 64)
+    P = ctypes.c_void_p
+    st = L.vsa_sparse_attn_fwd(P(1 << 12), P(1 << 16), P(1 << 20), P(1 << 24), P(1 << 26), s.c(),
+                               0.0, P(1 << 28), P(1 << 29), P(1 << 30), 8, None)
+    assert st == 3
+    assert L.vsa_sparse_attn_workspace_size(s.c()) > 0
