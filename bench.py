@@ -114,7 +114,7 @@ class ClockSampler:
         power = np.array([float(r[3]) for r in rows if r[3].strip() not in ("", "[N/A]")] or [0.0])
         loaded = sm[power >= np.percentile(power, 50)] if power.size == sm.size else sm
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i]})
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
         return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": mx, "reasons": reasons,
                 "samples": len(rows)}
 
@@ -342,7 +342,7 @@ def main():
                 import oracle
                 wl = __import__("content_adaptive_block_fractal_b200.workloads",
                                 fromlist=["get"]).get(args.workload)
-                ms, work_s, sample = oracle_sample(wl, [0, 1, 2, 3], 96)
+                ms, work_s, sample = oracle_sample(wl, [0, 1, 2, 3, 4, 5], 480)
                 result["cpu_baseline"] = {"value": ms, "unit": UNIT, "cores": oracle.num_threads(),
                                           "kind": "oracle", "sample": sample,
                                           "cpu_seconds_measured": work_s}
