@@ -77,6 +77,8 @@ bool empty(const vsa_shape &s) { return 1LL * s.B * s.heads * s.T * s.H * s.W ==
 }  // namespace
 
 namespace vsa {
+void set_last_error(const char *msg) { g_last_error = msg; }
+
 int num_sms() {
   static int cache[kMaxDevices] = {};
   int dev = 0;

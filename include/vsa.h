@@ -130,6 +130,24 @@ vsa_status vsa_sparse_attn_fwd(const void *qf, const void *kf, const void *vf,
                                void *workspace, size_t workspace_bytes,
                                void *stream);
 
+/* Block-sparse attention forward without a caller-provided workspace.
+ * The paper has no counterpart to this call; it exists for callers that cannot
+ * allocate device memory -- plugins whose host framework passes them only
+ * inputs and outputs, processes that reserve all device memory at start-up,
+ * and latency-critical paths where cudaMalloc/cudaFree would synchronise the
+ * device.  Same arguments and results as vsa_sparse_attn_fwd, minus the
+ * workspace: the scheduler's scratch lives in a fixed 8 MiB array inside the
+ * library (held by every GPU that loads it until the process exits), which
+ * fits about two million 128-row query tiles; larger shapes return
+ * VSA_ERR_CAPACITY.  All calls share that array and it keeps the last call's
+ * contents (each call re-plans and resets it first), so calls that overlap on
+ * the GPU race.  The first call on a device looks up the array's address;
+ * make it before any stream capture.  Allocates nothing. */
+vsa_status vsa_sparse_attn_fwd_noalloc(const void *qf, const void *kf, const void *vf,
+                                       const int64_t *row_ptr, const int32_t *col_idx,
+                                       vsa_shape s, float scale, void *o, float *lse,
+                                       void *stream);
+
 /* Message for the last non-OK status returned to the calling thread. */
 const char *vsa_last_error(void);
 
