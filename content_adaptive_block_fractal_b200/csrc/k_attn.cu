@@ -6,21 +6,25 @@
 // Blackwell mapping.  A work item is a 128-row query tile made of two 64-token
 // query blocks of one (batch, head): the same patch in frames 2t and 2t+1,
 // whose kept lists overlap most (time pairing).  The item walks the merged,
-// ascending union of both lists two key blocks (128 keys) per step:
-//   S  = Q K^T   tcgen05.mma M=128, N=64*nb, K=d   (SMEM x SMEM -> TMEM fp32)
-//   P  = online softmax of S, per row only over the blocks kept by that row's
-//        query block, written to SMEM as bf16
-//   O += P V     tcgen05.mma M=128, N=d, K=64*nb   (SMEM x SMEM -> TMEM fp32)
+// ascending union of both lists two key blocks (128 keys) per step n:
+//   S_n = Q K_n^T  tcgen05.mma M=128, N=64*nb, K=d  (SMEM x SMEM -> TMEM S[n%2])
+//   P_n = online softmax of S_n, per row only over the blocks its own query
+//         block keeps, stored to TMEM P[n%2] as packed bf16
+//   O  += P_n V_n  tcgen05.mma M=128, N=d, K=64*nb  (TMEM x SMEM -> TMEM O)
+// The MMA warp issues S_{n+1} before PV_n, so the tensor core computes the
+// next scores while the softmax warps work on the current ones.
 // Warp roles (192 threads, one CTA per SM, persistent):
-//   warp 0      producer: takes items from an atomic counter over an LPT work
-//               list, merges the two CSR lists, issues TMA loads of Q and of
-//               the K/V blocks into a 2-stage ring (128B-swizzled boxes);
-//   warp 1      allocates TMEM; one lane issues all MMAs and commits;
+//   warp 0      producer: takes items from an atomic counter over a
+//               longest-first work list, merges the two CSR lists, issues TMA
+//               loads of Q and of the K and V blocks into 3-deep rings
+//               (128B-swizzled boxes) and publishes one step record per step;
+//   warp 1      allocates 512 TMEM columns; one lane issues all MMAs/commits;
 //   warps 2..5  one thread per query row: softmax, lazy O rescale (only when
 //               the running max grows by more than 2^8), epilogue O / l -> bf16
 //               and LSE.
-// Every mbarrier wait is bounded; a wait that gives up records an error code
-// and the CTA winds down instead of hanging.
+// TMEM columns: S0 [0,128), S1 [128,256), O [256,256+d), P0 [384,448),
+// P1 [448,512).  Every mbarrier wait is bounded; a wait that gives up records
+// an error code and the CTA winds down instead of hanging.
 #include "vsa_device.cuh"
 #include "vsa_internal.h"
 
@@ -31,10 +35,12 @@ namespace vsa {
 namespace {
 
 constexpr int kThreads = 192;
-constexpr int kStages = 2;
-constexpr int kListWin = 512;          // CSR entries staged per list in SMEM
-constexpr uint32_t kTmemCols = 256;    // O: [0, 128), S: [128, 256)
-constexpr uint32_t kTmemS = 128;
+constexpr int kKStages = 3;
+constexpr int kVStages = 3;
+constexpr int kMetaRing = 4;
+constexpr int kListWin = 64;           // CSR entries staged per list in SMEM
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
 
 struct StepMeta {
   int32_t blk0, blk1;  // key blocks of this step (blk1 = -1 when nb == 1)
@@ -47,16 +53,16 @@ struct StepMeta {
 template <int D>
 struct Smem {
   static constexpr int kQBytes = 128 * D * 2;             // two query blocks
-  static constexpr int kKVHalf = 2 * 64 * D * 2;          // K (or V) of two key blocks
-  static constexpr int kStageBytes = 2 * kKVHalf;         // K + V
-  static constexpr int kPBytes = 128 * 128 * 2;           // P tile, 128 keys
+  static constexpr int kKVBytes = 2 * 64 * D * 2;         // K (or V) of two key blocks
   static constexpr int kQOff = 0;
-  static constexpr int kKVOff = kQOff + kQBytes;
-  static constexpr int kPOff = kKVOff + kStages * kStageBytes;
-  static constexpr int kMetaOff = kPOff + kPBytes;
-  static constexpr int kListOff = kMetaOff + kStages * static_cast<int>(sizeof(StepMeta));
-  static constexpr int kBarOff = kListOff + 2 * kListWin * 4;
-  static constexpr int kNumBars = 2 * kStages + 6;
+  static constexpr int kKOff = kQOff + kQBytes;
+  static constexpr int kVOff = kKOff + kKStages * kKVBytes;
+  static constexpr int kMetaOff = kVOff + kVStages * kKVBytes;
+  static constexpr int kListOff = kMetaOff + kMetaRing * static_cast<int>(sizeof(StepMeta));
+  static constexpr int kBarOff = (kListOff + 2 * kListWin * 4 + 7) & ~7;
+  // k_full[3] k_empty[3] v_full[3] v_empty[3] meta_full[4] q_full q_empty
+  // s_full[2] p_full[2] pv_done o_full o_empty
+  static constexpr int kNumBars = 4 * 3 + kMetaRing + 2 + 2 + 2 + 3;
   static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kTmemSlotOff + 16;
   static constexpr int kAlloc = kBytes + 1024;            // room to align to 1 KiB
@@ -67,7 +73,7 @@ struct AttnArgs {
   const int32_t *col_idx;
   __nv_bfloat16 *o;
   float *lse;
-  const int32_t *order;   // LPT-ordered work items
+  const int32_t *order;   // longest-first work items
   int *counter;           // next position in `order`
   unsigned *err;
   int64_t items;          // total work items
@@ -102,27 +108,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   int32_t *list0 = reinterpret_cast<int32_t *>(smem + L::kListOff);
   int32_t *list1 = list0 + kListWin;
   const uint32_t bar = sbase + L::kBarOff;
-  auto kv_full = [&](int s) { return bar + 8u * s; };
-  auto kv_empty = [&](int s) { return bar + 8u * (kStages + s); };
-  const uint32_t q_full = bar + 8u * (2 * kStages + 0);
-  const uint32_t q_empty = bar + 8u * (2 * kStages + 1);
-  const uint32_t s_full = bar + 8u * (2 * kStages + 2);
-  const uint32_t p_full = bar + 8u * (2 * kStages + 3);
-  const uint32_t o_full = bar + 8u * (2 * kStages + 4);
-  const uint32_t o_empty = bar + 8u * (2 * kStages + 5);
+  auto k_full = [&](int s) { return bar + 8u * s; };
+  auto k_empty = [&](int s) { return bar + 8u * (3 + s); };
+  auto v_full = [&](int s) { return bar + 8u * (6 + s); };
+  auto v_empty = [&](int s) { return bar + 8u * (9 + s); };
+  auto meta_full = [&](int s) { return bar + 8u * (12 + s); };
+  const uint32_t q_full = bar + 8u * (12 + kMetaRing);
+  const uint32_t q_empty = q_full + 8;
+  auto s_full = [&](int s) { return q_full + 16u + 8u * s; };
+  auto p_full = [&](int s) { return q_full + 32u + 8u * s; };
+  const uint32_t pv_done = q_full + 48;
+  const uint32_t o_full = q_full + 56;
+  const uint32_t o_empty = q_full + 64;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemSlotOff);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(kv_full(s), 1);
-      mbar_init(kv_empty(s), 1);
+    for (int s = 0; s < 3; ++s) {
+      mbar_init(k_full(s), 1);
+      mbar_init(k_empty(s), 1);
+      mbar_init(v_full(s), 1);
+      mbar_init(v_empty(s), 1);
     }
+    for (int s = 0; s < kMetaRing; ++s) mbar_init(meta_full(s), 1);
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(s_full(s), 1);
+      mbar_init(p_full(s), 128);
+    }
+    mbar_init(pv_done, 1);
     mbar_init(o_full, 1);
     mbar_init(o_empty, 128);
     fence_mbar_init();
@@ -143,34 +159,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tk);
       tma_prefetch_desc(&tv);
     }
-    int stage = 0;
-    uint32_t kv_phase = 0;   // bit s: parity to wait on kv_empty[s]
+    int n = 0;               // global step counter
     uint32_t q_phase = 0;
     bool ok = true;
     int nitems = 0;
-    // Waits until stage `stage` is free, publishes the step and loads it.
+    // Waits until the K/V stages of step n are free, publishes the step
+    // record and loads its key/value blocks.
     auto emit = [&](const StepMeta &m) -> bool {
-      if (!mbar_wait(kv_empty(stage), ((kv_phase >> stage) & 1u) ^ 1u, a.err, kErrWaitMma))
-        return false;
-      kv_phase ^= 1u << stage;
+      const int s3 = n % 3;
+      const uint32_t par = ((n / 3) & 1) ^ 1;
+      if (!mbar_wait(k_empty(s3), par, a.err, kErrWaitMma)) return false;
+      if (!mbar_wait(v_empty(s3), par, a.err, kErrWaitMma)) return false;
       if (lane == 0) {
-        meta[stage] = m;
+        meta[n % kMetaRing] = m;
+        mbar_arrive(meta_full(n % kMetaRing));
         const int nb = m.nb > 0 ? m.nb : 0;
-        mbar_arrive_expect_tx(kv_full(stage), static_cast<uint32_t>(nb * 2 * 64 * D * 2));
-        const uint32_t kbase = sbase + L::kKVOff + stage * L::kStageBytes;
-        const uint32_t vbase = kbase + L::kKVHalf;
+        const uint32_t bytes = static_cast<uint32_t>(nb * 64 * D * 2);
+        mbar_arrive_expect_tx(k_full(s3), bytes);
+        mbar_arrive_expect_tx(v_full(s3), bytes);
+        const uint32_t kbase = sbase + L::kKOff + s3 * L::kKVBytes;
+        const uint32_t vbase = sbase + L::kVOff + s3 * L::kKVBytes;
         for (int j = 0; j < nb; ++j) {
           const int row = static_cast<int>(static_cast<int64_t>(m.bh) * a.N) +
                           (j ? m.blk1 : m.blk0) * 64;
           for (int dh = 0; dh < D / 64; ++dh) {
             const uint32_t off = dh * (2 * 64 * 128) + j * (64 * 128);
-            tma_load_2d(kbase + off, &tk, kv_full(stage), dh * 64, row);
-            tma_load_2d(vbase + off, &tv, kv_full(stage), dh * 64, row);
+            tma_load_2d(kbase + off, &tk, k_full(s3), dh * 64, row);
+          }
+        }
+        for (int j = 0; j < nb; ++j) {
+          const int row = static_cast<int>(static_cast<int64_t>(m.bh) * a.N) +
+                          (j ? m.blk1 : m.blk0) * 64;
+          for (int dh = 0; dh < D / 64; ++dh) {
+            const uint32_t off = dh * (2 * 64 * 128) + j * (64 * 128);
+            tma_load_2d(vbase + off, &tv, v_full(s3), dh * 64, row);
           }
         }
       }
       __syncwarp();
-      stage = (stage + 1) % kStages;
+      ++n;
       return true;
     };
     while (ok) {
@@ -272,64 +299,90 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    int stage = 0;
-    uint32_t kv_phase = 0, q_phase = 0, p_phase = 0, oe_phase = 0;
+    uint32_t q_phase = 0, oe_phase = 0;
     bool first_item = true;
+    bool ok = true;
     constexpr uint32_t kIdescO = idesc_bf16(128, D, false, true);
-    while (true) {
-      if (!mbar_wait(kv_full(stage), (kv_phase >> stage) & 1u, a.err, kErrWaitTma)) break;
-      kv_phase ^= 1u << stage;
-      const StepMeta m = meta[stage];
-      if (m.nb < 0) break;
-      const bool first = m.first_last & 1, last = m.first_last & 2;
-      if (first) {
-        if (!mbar_wait(q_full, q_phase, a.err, kErrWaitTma)) break;
+    const uint32_t qb = sbase + L::kQOff;
+    // Waits for step n's key blocks and returns its record.
+    auto fetch = [&](int n, StepMeta &m) -> bool {
+      if (!mbar_wait(k_full(n % 3), (n / 3) & 1, a.err, kErrWaitTma)) return false;
+      m = meta[n % kMetaRing];
+      return true;
+    };
+    // S_n = Q K_n^T into S[n%2]; releases the K stage and, after an item's
+    // last step, the Q tile.
+    auto issue_s = [&](int n, const StepMeta &m) -> bool {
+      if (m.first_last & 1) {
+        if (!mbar_wait(q_full, q_phase, a.err, kErrWaitTma)) return false;
         q_phase ^= 1u;
       }
       tc_fence_after();
-      const uint32_t qb = sbase + L::kQOff;
-      const uint32_t kb = sbase + L::kKVOff + stage * L::kStageBytes;
-      const uint32_t vb = kb + L::kKVHalf;
-      const uint32_t pb = sbase + L::kPOff;
       if (lane == 0 && m.nb > 0) {
+        const uint32_t kb = sbase + L::kKOff + (n % 3) * L::kKVBytes;
         const uint32_t idesc_s = idesc_bf16(128, 64 * m.nb, false, false);
+        const uint32_t dcol = tmem + ((n & 1) ? kColS1 : kColS0);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint64_t ad = smem_desc(qb + (k >> 2) * (128 * 128) + (k & 3) * 32, 16, 1024);
           const uint64_t bd = smem_desc(kb + (k >> 2) * (2 * 64 * 128) + (k & 3) * 32, 16, 1024);
-          mma_bf16_ss(tmem + kTmemS, ad, bd, idesc_s, k > 0);
+          mma_bf16_ss(dcol, ad, bd, idesc_s, k > 0);
         }
       }
       __syncwarp();
       if (lane == 0) {
-        mma_commit(s_full);
-        if (last) mma_commit(q_empty);
+        mma_commit(s_full(n & 1));
+        mma_commit(k_empty(n % 3));
+        if (m.first_last & 2) mma_commit(q_empty);
       }
       __syncwarp();
-      if (!mbar_wait(p_full, p_phase, a.err, kErrWaitSoftmax)) break;
-      p_phase ^= 1u;
-      if (first) {
+      return true;
+    };
+    // O (+)= P_n V_n; releases the V stage.
+    auto issue_pv = [&](int n, const StepMeta &m) -> bool {
+      if (!mbar_wait(p_full(n & 1), (n >> 1) & 1, a.err, kErrWaitSoftmax)) return false;
+      if (m.first_last & 1) {
         if (!first_item) {
-          if (!mbar_wait(o_empty, oe_phase, a.err, kErrWaitSoftmax)) break;
+          if (!mbar_wait(o_empty, oe_phase, a.err, kErrWaitSoftmax)) return false;
           oe_phase ^= 1u;
         }
         first_item = false;
       }
+      if (!mbar_wait(v_full(n % 3), (n / 3) & 1, a.err, kErrWaitTma)) return false;
       tc_fence_after();
       if (lane == 0 && m.nb > 0) {
+        const uint32_t vb = sbase + L::kVOff + (n % 3) * L::kKVBytes;
+        const uint32_t pcol = tmem + ((n & 1) ? kColP1 : kColP0);
         for (int k = 0; k < 4 * m.nb; ++k) {
-          const uint64_t ad = smem_desc(pb + (k >> 2) * (128 * 128) + (k & 3) * 32, 16, 1024);
           const uint64_t bd = smem_desc(vb + k * 2048, 2 * 64 * 128, 1024);
-          mma_bf16_ss(tmem, ad, bd, kIdescO, !(first && k == 0));
+          mma_bf16_ts(tmem + kColO, pcol + k * 8, bd, kIdescO, !((m.first_last & 1) && k == 0));
         }
       }
       __syncwarp();
       if (lane == 0) {
-        mma_commit(kv_empty(stage));
-        if (last) mma_commit(o_full);
+        mma_commit(v_empty(n % 3));
+        mma_commit(pv_done);
+        if (m.first_last & 2) mma_commit(o_full);
       }
       __syncwarp();
-      stage = (stage + 1) % kStages;
+      return true;
+    };
+    StepMeta cur, nxt;
+    int n = 0;
+    if (fetch(0, cur) && cur.nb >= 0 && issue_s(0, cur)) {
+      while (ok) {
+        if (!(ok = fetch(n + 1, nxt))) break;
+        const bool more = nxt.nb >= 0;
+        const bool next_first = more && (nxt.first_last & 1);
+        // the next step's scores go first unless it opens a new item (its Q
+        // tile may still be loading; finish this item first)
+        if (more && !next_first && !(ok = issue_s(n + 1, nxt))) break;
+        if (!(ok = issue_pv(n, cur))) break;
+        if (next_first && !(ok = issue_s(n + 1, nxt))) break;
+        if (!more) break;
+        ++n;
+        cur = nxt;
+      }
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
@@ -337,47 +390,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = quarter * 32 + lane;       // query row within the tile
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const uint32_t sel = row >= 64 ? 1u : 0u;
-    unsigned char *prow = smem + L::kPOff + (row >> 3) * 1024 + (row & 7) * 128;
-    int stage = 0;
-    uint32_t kv_phase = 0, s_phase = 0, o_phase = 0;
+    uint32_t o_phase = 0;
     float m_run = -INFINITY, l_run = 0.0f;
-    while (true) {
-      if (!mbar_wait(kv_full(stage), (kv_phase >> stage) & 1u, a.err, kErrWaitTma)) break;
-      kv_phase ^= 1u << stage;
-      const StepMeta m = meta[stage];
+    for (int n = 0;; ++n) {
+      if (!mbar_wait(meta_full(n % kMetaRing), (n / kMetaRing) & 1, a.err, kErrWaitTma)) break;
+      const StepMeta m = meta[n % kMetaRing];
       if (m.nb < 0) break;
       const bool first = m.first_last & 1, last = m.first_last & 2;
       if (first) {
         m_run = -INFINITY;
         l_run = 0.0f;
       }
-      if (!mbar_wait(s_full, s_phase, a.err, kErrWaitMma)) break;
-      s_phase ^= 1u;
+      if (!mbar_wait(s_full(n & 1), (n >> 1) & 1, a.err, kErrWaitMma)) break;
       tc_fence_after();
-      float x[128];
+      // warps hold rows of one query block, so v0 / v1 are warp-uniform
       const bool v0 = (m.flags >> sel) & 1u;
-      const bool v1 = (m.flags >> (2 + sel)) & 1u;
+      const bool v1 = m.nb > 1 && ((m.flags >> (2 + sel)) & 1u);
+      float x[128];
       float mx = -INFINITY;
       if (m.nb > 0) {
-        tmem_ld32(lane_addr + kTmemS + 0, &x[0]);
-        tmem_ld32(lane_addr + kTmemS + 32, &x[32]);
-        if (m.nb > 1) {
-          tmem_ld32(lane_addr + kTmemS + 64, &x[64]);
-          tmem_ld32(lane_addr + kTmemS + 96, &x[96]);
-        }
-        tmem_wait_ld();
+        const uint32_t scol = lane_addr + ((n & 1) ? kColS1 : kColS0);
+        tmem_ld64x2(scol, scol + 64, x);
+        if (v0) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          x[j] = v0 ? x[j] * a.c : -INFINITY;
-          mx = fmaxf(mx, x[j]);
+          for (int j = 0; j < 64; ++j) mx = fmaxf(mx, x[j]);
         }
-        if (m.nb > 1) {
+        if (v1) {
 #pragma unroll
-          for (int j = 64; j < 128; ++j) {
-            x[j] = v1 ? x[j] * a.c : -INFINITY;
-            mx = fmaxf(mx, x[j]);
-          }
+          for (int j = 64; j < 128; ++j) mx = fmaxf(mx, x[j]);
         }
+        mx *= a.c;
       }
       // lazy rescale: move the reference max only when it grows by > 8 (2^8)
       float alpha = 1.0f;
@@ -385,48 +427,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (mx > m_run + 8.0f) {
         if (m_run != -INFINITY) {
           alpha = ex2(m_run - mx);
-          resc = !first;
+          resc = true;
         }
         l_run *= alpha;
         m_run = mx;
       }
       const float mref = m_run == -INFINITY ? 0.0f : m_run;
       float rs = 0.0f;
+      if (m.nb > 0) {
+        uint32_t pk[64];
+        if (v0) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (h < m.nb) {
-          unsigned char *dst = prow + h * (128 * 128);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float p0 = ex2(x[h * 64 + j * 8 + 2 * e] - mref);
-              const float p1 = ex2(x[h * 64 + j * 8 + 2 * e + 1] - mref);
-              rs += p0 + p1;
-              w[e] = pack_bf16x2(p0, p1);
-            }
-            *reinterpret_cast<uint4 *>(dst + ((j ^ (row & 7)) << 4)) =
-                make_uint4(w[0], w[1], w[2], w[3]);
+          for (int j = 0; j < 32; ++j) {
+            const float p0 = ex2(fmaf(x[2 * j], a.c, -mref));
+            const float p1 = ex2(fmaf(x[2 * j + 1], a.c, -mref));
+            rs += p0 + p1;
+            pk[j] = pack_bf16x2(p0, p1);
           }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) pk[j] = 0u;
         }
+        if (v1) {
+#pragma unroll
+          for (int j = 32; j < 64; ++j) {
+            const float p0 = ex2(fmaf(x[2 * j], a.c, -mref));
+            const float p1 = ex2(fmaf(x[2 * j + 1], a.c, -mref));
+            rs += p0 + p1;
+            pk[j] = pack_bf16x2(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int j = 32; j < 64; ++j) pk[j] = 0u;
+        }
+        const uint32_t pcol = lane_addr + ((n & 1) ? kColP1 : kColP0);
+        tmem_st32u(pcol, pk);
+        if (m.nb > 1) tmem_st32u(pcol + 32, pk + 32);
       }
       l_run += rs;
       if (__any_sync(0xFFFFFFFFu, resc)) {
+        // O must hold PV_{n-1} before it is rescaled
+        if (!mbar_wait(pv_done, (n - 1) & 1, a.err, kErrWaitMma)) break;
+        tc_fence_after();
 #pragma unroll 1
         for (int cc = 0; cc < D; cc += 32) {
           float ov[32];
-          tmem_ld32(lane_addr + cc, ov);
-          tmem_wait_ld();
+          tmem_ld32(lane_addr + kColO + cc, ov);
 #pragma unroll
           for (int j = 0; j < 32; ++j) ov[j] *= alpha;
-          tmem_st32(lane_addr + cc, ov);
+          tmem_st32(lane_addr + kColO + cc, ov);
         }
-        tmem_wait_st();
       }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(p_full(n & 1));
       if (last) {
         if (!mbar_wait(o_full, o_phase, a.err, kErrWaitMma)) break;
         o_phase ^= 1u;
@@ -441,8 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int cc = 0; cc < D; cc += 32) {
           float ov[32];
-          tmem_ld32(lane_addr + cc, ov);
-          tmem_wait_ld();
+          tmem_ld32(lane_addr + kColO + cc, ov);
           if (store) {
             if (!has_keys) {
 #pragma unroll
@@ -464,7 +517,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(o_empty);
       }
-      stage = (stage + 1) % kStages;
     }
   }
 

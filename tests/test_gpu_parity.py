@@ -184,7 +184,8 @@ def test_attention_with_oracle_mask(name):
 
 @pytest.mark.parametrize("T,H,W,d,density", [(3, 16, 24, 128, 0.3), (3, 16, 24, 64, 0.5),
                                              (5, 8, 16, 128, 0.05), (1, 8, 8, 64, 1.0),
-                                             (2, 32, 32, 128, 0.6)])
+                                             (2, 32, 32, 128, 0.6), (2, 32, 64, 128, 1.0),
+                                             (4, 24, 40, 64, 0.15)])
 def test_attention_random_mask(T, H, W, d, density):
     """Seeded random CSR (neither side's mask), with empty and single-block rows."""
     wl = small_shape(T=T, H=H, W=W, d=d)
@@ -200,6 +201,10 @@ def test_attention_random_mask(T, H, W, d, density):
         keep[1] = False
         keep[2] = False
         keep[2, Nb - 1] = True
+    HW = wl.Hb * wl.Wb
+    if T >= 2 and Nb > 3:
+        keep[3] = False                  # both query blocks of a time pair empty
+        keep[3 + HW] = False
     rp, ci = oracle.mask_to_csr(keep)
     o_ref, lse_ref = oracle.sparse_attention(qf, kf, vf, rp, ci)
     o, lse = vsa.sparse_attn_fwd(dev(qf), dev(kf), dev(vf), dev(rp), dev(ci), vsa.Shape.of(wl))
