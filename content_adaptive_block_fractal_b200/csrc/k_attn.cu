@@ -7,40 +7,48 @@
 // query blocks of one (batch, head): the same patch in frames 2t and 2t+1,
 // whose kept lists overlap most (time pairing).  The item walks the merged,
 // ascending union of both lists two key blocks (128 keys) per step n:
-//   S_n = Q K_n^T  tcgen05.mma M=128, N=64*nb, K=d  (SMEM x SMEM -> TMEM S[n%2])
+//   S_n = Q K_n^T  tcgen05.mma M=128, N=64*nb, K=d  (SMEM x SMEM -> TMEM S[n%3])
 //   P_n = online softmax of S_n, per row only over the blocks its own query
-//         block keeps, stored to TMEM P[n%2] as packed bf16
+//         block keeps, written as packed bf16 over the first 64 columns of
+//         the same TMEM buffer
 //   O  += P_n V_n  tcgen05.mma M=128, N=d, K=64*nb  (TMEM x SMEM -> TMEM O)
-// The MMA warp issues S_{n+1} before PV_n, so the tensor core computes the
-// next scores while the softmax warps work on the current ones.
-// Warp roles (192 threads, one CTA per SM, persistent):
+// Three S buffers let the MMA warp keep the scores up to two steps ahead of
+// the softmax: the tensor core runs S_{n+2} while P_n is being formed; S_{n+3}
+// reuses step n's buffer only after PV_n has completed.
+// Warp roles (352 threads, one CTA per SM, persistent):
 //   warp 0      producer: takes items from an atomic counter over a
-//               longest-first work list, merges the two CSR lists, issues TMA
-//               loads of Q and of the K and V blocks into 3-deep rings
-//               (128B-swizzled boxes) and publishes one step record per step;
-//   warp 1      allocates 512 TMEM columns; one lane issues all MMAs/commits;
-//   warps 2..5  one thread per query row: softmax, lazy O rescale (only when
-//               the running max grows by more than 2^8), epilogue O / l -> bf16
-//               and LSE.
-// TMEM columns: S0 [0,128), S1 [128,256), O [256,256+d), P0 [384,448),
-// P1 [448,512).  Every mbarrier wait is bounded; a wait that gives up records
-// an error code and the CTA winds down instead of hanging.
+//               longest-first work list, merges the two CSR lists, publishes
+//               one step record per step (8-deep ring) and issues TMA loads
+//               (128B-swizzled boxes): Q per item, K of step m and V of step
+//               m-2, each into a 3-deep ring;
+//   warp 1      allocates 512 TMEM columns; one lane issues the S MMAs;
+//   warp 10     one lane issues the PV MMAs.  tcgen05.mma issue is paced by
+//               the tensor core, so two issuers let one's waits overlap the
+//               other's MMAs (commits track each thread's own MMAs);
+//   warps 2..9  two softmax warpgroups taking alternate steps (even steps:
+//               warps 2..5, odd steps: warps 6..9), one thread per query row:
+//               softmax, lazy O rescale (only when the running max grows by
+//               more than 2^8), epilogue O / l -> bf16 and LSE.  Only the
+//               running max and row sum pass between the two groups.
+// TMEM columns: S0 [0,128), S1 [128,256), S2 [256,384), O [384,384+d).
+// Every mbarrier wait is bounded; a wait that gives up records an error code
+// and the CTA winds down instead of hanging.
 #include "vsa_device.cuh"
 #include "vsa_internal.h"
 
 #include <cmath>
+#include <cstdio>
 #include <mutex>
 
 namespace vsa {
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kKStages = 3;
-constexpr int kVStages = 3;
-constexpr int kMetaRing = 4;
-constexpr int kListWin = 64;           // CSR entries staged per list in SMEM
+constexpr int kThreads = 352;
+constexpr int kRing = 3;               // K stages, V stages, S buffers
+constexpr int kMetaRing = 8;
+constexpr int kListWin = 32;           // CSR entries staged per list in SMEM
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
+constexpr uint32_t kColO = 384;
 
 struct StepMeta {
   int32_t blk0, blk1;  // key blocks of this step (blk1 = -1 when nb == 1)
@@ -48,6 +56,7 @@ struct StepMeta {
   uint32_t flags;      // bit0/1: blk0 kept by query block 0/1; bit2/3: blk1
   int32_t bh, r0, r1;  // head slice and query blocks (r1 = -1 if absent)
   int32_t first_last;  // bit0: first step of the item, bit1: last step
+  int32_t seq;         // item sequence number within this CTA
 };
 
 template <int D>
@@ -56,16 +65,19 @@ struct Smem {
   static constexpr int kKVBytes = 2 * 64 * D * 2;         // K (or V) of two key blocks
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kQBytes;
-  static constexpr int kVOff = kKOff + kKStages * kKVBytes;
-  static constexpr int kMetaOff = kVOff + kVStages * kKVBytes;
+  static constexpr int kVOff = kKOff + kRing * kKVBytes;
+  static constexpr int kMetaOff = kVOff + kRing * kKVBytes;
   static constexpr int kListOff = kMetaOff + kMetaRing * static_cast<int>(sizeof(StepMeta));
-  static constexpr int kBarOff = (kListOff + 2 * kListWin * 4 + 7) & ~7;
-  // k_full[3] k_empty[3] v_full[3] v_empty[3] meta_full[4] q_full q_empty
-  // s_full[2] p_full[2] pv_done o_full o_empty
-  static constexpr int kNumBars = 4 * 3 + kMetaRing + 2 + 2 + 2 + 3;
+  static constexpr int kXchgOff = kListOff + 2 * kListWin * 4;   // m_sh[2][128], l_sh[2][128]
+  static constexpr int kBarOff = (kXchgOff + 4 * 128 * 4 + 7) & ~7;
+  // k_full[3] v_full[3] s_full[3] pv_buf[3] meta_full[8] meta_empty[8]
+  // q_full q_empty p_full[4] o_full o_empty m_full[2] l_full[2]
+  // (s_full also frees K stages and pv_buf V stages: same completions)
+  static constexpr int kNumBars = 4 * kRing + 2 * kMetaRing + 2 + 4 + 2 + 4;
   static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kTmemSlotOff + 16;
-  static constexpr int kAlloc = kBytes + 1024;            // room to align to 1 KiB
+  static constexpr int kAlloc = kBytes;                   // base is 1 KiB aligned
+  static_assert(kAlloc <= 232448, "shared memory layout exceeds 227 KiB");
 };
 
 struct AttnArgs {
@@ -95,50 +107,62 @@ __device__ __forceinline__ void decode_item(int item, const AttnArgs &a, int &bh
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __maxnreg__(168)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tq,
                        const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const AttnArgs a) {
   using L = Smem<D>;
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char *smem = reinterpret_cast<unsigned char *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // The 128B-swizzled operand tiles need a 1 KiB aligned base; if the
+  // dynamic allocation is not aligned, every thread leaves before touching
+  // barriers, TMEM or TMA (uniform exit, recorded in the error word).
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(a.err, kErrSmemAlign);
+    return;
+  }
+  unsigned char *smem = smem_raw;
   const uint32_t sbase = smem_u32(smem);
   StepMeta *meta = reinterpret_cast<StepMeta *>(smem + L::kMetaOff);
   int32_t *list0 = reinterpret_cast<int32_t *>(smem + L::kListOff);
   int32_t *list1 = list0 + kListWin;
+  float *m_sh = reinterpret_cast<float *>(smem + L::kXchgOff);   // [2][128]
+  float *l_sh = m_sh + 256;                                        // [2][128]
   const uint32_t bar = sbase + L::kBarOff;
   auto k_full = [&](int s) { return bar + 8u * s; };
-  auto k_empty = [&](int s) { return bar + 8u * (3 + s); };
-  auto v_full = [&](int s) { return bar + 8u * (6 + s); };
-  auto v_empty = [&](int s) { return bar + 8u * (9 + s); };
-  auto meta_full = [&](int s) { return bar + 8u * (12 + s); };
-  const uint32_t q_full = bar + 8u * (12 + kMetaRing);
+  auto v_full = [&](int s) { return bar + 8u * (kRing + s); };
+  auto s_full = [&](int s) { return bar + 8u * (2 * kRing + s); };
+  auto pv_buf = [&](int s) { return bar + 8u * (3 * kRing + s); };
+  auto meta_full = [&](int s) { return bar + 8u * (4 * kRing + s); };
+  auto meta_empty = [&](int s) { return bar + 8u * (4 * kRing + kMetaRing + s); };
+  const uint32_t q_full = bar + 8u * (4 * kRing + 2 * kMetaRing);
   const uint32_t q_empty = q_full + 8;
-  auto s_full = [&](int s) { return q_full + 16u + 8u * s; };
-  auto p_full = [&](int s) { return q_full + 32u + 8u * s; };
-  const uint32_t pv_done = q_full + 48;
-  const uint32_t o_full = q_full + 56;
-  const uint32_t o_empty = q_full + 64;
+  auto p_full = [&](int s) { return q_full + 16u + 8u * s; };   // 4 slots
+  const uint32_t o_full = q_full + 48;
+  const uint32_t o_empty = q_full + 56;
+  auto m_full = [&](int s) { return q_full + 64u + 8u * s; };
+  auto l_full = [&](int s) { return q_full + 80u + 8u * s; };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemSlotOff);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 3; ++s) {
+    for (int s = 0; s < kRing; ++s) {
       mbar_init(k_full(s), 1);
-      mbar_init(k_empty(s), 1);
       mbar_init(v_full(s), 1);
-      mbar_init(v_empty(s), 1);
+      mbar_init(s_full(s), 1);
+      mbar_init(pv_buf(s), 1);
     }
-    for (int s = 0; s < kMetaRing; ++s) mbar_init(meta_full(s), 1);
+    for (int s = 0; s < kMetaRing; ++s) {
+      mbar_init(meta_full(s), 1);
+      mbar_init(meta_empty(s), 128);
+    }
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
+    for (int s = 0; s < 4; ++s) mbar_init(p_full(s), 128);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(s_full(s), 1);
-      mbar_init(p_full(s), 128);
+      mbar_init(m_full(s), 128);
+      mbar_init(l_full(s), 128);
     }
-    mbar_init(pv_done, 1);
     mbar_init(o_full, 1);
     mbar_init(o_empty, 128);
     fence_mbar_init();
@@ -159,45 +183,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tk);
       tma_prefetch_desc(&tv);
     }
-    int n = 0;               // global step counter
+    int m = 0;               // next step whose record and K blocks go out
+    int vnext = 0;           // next step whose V blocks go out
     uint32_t q_phase = 0;
     bool ok = true;
     int nitems = 0;
-    // Waits until the K/V stages of step n are free, publishes the step
-    // record and loads its key/value blocks.
-    auto emit = [&](const StepMeta &m) -> bool {
-      const int s3 = n % 3;
-      const uint32_t par = ((n / 3) & 1) ^ 1;
-      if (!mbar_wait(k_empty(s3), par, a.err, kErrWaitMma)) return false;
-      if (!mbar_wait(v_empty(s3), par, a.err, kErrWaitMma)) return false;
-      if (lane == 0) {
-        meta[n % kMetaRing] = m;
-        mbar_arrive(meta_full(n % kMetaRing));
-        const int nb = m.nb > 0 ? m.nb : 0;
-        const uint32_t bytes = static_cast<uint32_t>(nb * 64 * D * 2);
-        mbar_arrive_expect_tx(k_full(s3), bytes);
-        mbar_arrive_expect_tx(v_full(s3), bytes);
-        const uint32_t kbase = sbase + L::kKOff + s3 * L::kKVBytes;
-        const uint32_t vbase = sbase + L::kVOff + s3 * L::kKVBytes;
-        for (int j = 0; j < nb; ++j) {
-          const int row = static_cast<int>(static_cast<int64_t>(m.bh) * a.N) +
-                          (j ? m.blk1 : m.blk0) * 64;
-          for (int dh = 0; dh < D / 64; ++dh) {
-            const uint32_t off = dh * (2 * 64 * 128) + j * (64 * 128);
-            tma_load_2d(kbase + off, &tk, k_full(s3), dh * 64, row);
-          }
-        }
-        for (int j = 0; j < nb; ++j) {
-          const int row = static_cast<int>(static_cast<int64_t>(m.bh) * a.N) +
-                          (j ? m.blk1 : m.blk0) * 64;
-          for (int dh = 0; dh < D / 64; ++dh) {
-            const uint32_t off = dh * (2 * 64 * 128) + j * (64 * 128);
-            tma_load_2d(vbase + off, &tv, v_full(s3), dh * 64, row);
-          }
+    // TMA of the (one or two) key blocks of step record r into a 3-stage ring.
+    auto load_blocks = [&](const CUtensorMap *map, uint32_t base, uint32_t bar_full,
+                           const StepMeta &r) {
+      const int nb = r.nb > 0 ? r.nb : 0;
+      mbar_arrive_expect_tx(bar_full, static_cast<uint32_t>(nb * 64 * D * 2));
+      const int head_row = static_cast<int>(static_cast<int64_t>(r.bh) * a.N);
+      if (nb > 0) {
+#pragma unroll
+        for (int dh = 0; dh < D / 64; ++dh)
+          tma_load_2d(base + dh * 16384, map, bar_full, dh * 64, head_row + r.blk0 * 64);
+        if (nb > 1) {
+#pragma unroll
+          for (int dh = 0; dh < D / 64; ++dh)
+            tma_load_2d(base + dh * 16384 + 8192, map, bar_full, dh * 64, head_row + r.blk1 * 64);
         }
       }
+    };
+    // V blocks of step vnext (two steps behind the K blocks).
+    auto emit_v = [&]() -> bool {
+      const int s3 = vnext % kRing;
+      // the stage's previous user PV_{vnext-3} has completed (its pv_buf)
+      if (vnext >= kRing &&
+          !mbar_wait(pv_buf(s3), ((vnext - kRing) / kRing) & 1, a.err, kErrWaitMma))
+        return false;
+      if (lane == 0)
+        load_blocks(&tv, sbase + L::kVOff + s3 * L::kKVBytes, v_full(s3), meta[vnext % kMetaRing]);
       __syncwarp();
-      ++n;
+      ++vnext;
+      return true;
+    };
+    // Publishes step record r as step m and loads its K blocks; the V blocks
+    // of step m-2 follow.
+    auto emit = [&](const StepMeta &r) -> bool {
+      const int s3 = m % kRing, sm = m % kMetaRing;
+      if (!mbar_wait(meta_empty(sm), ((m / kMetaRing) & 1) ^ 1, a.err, kErrWaitSoftmax)) return false;
+      // the stage's previous user S_{m-3} has completed (its s_full)
+      if (m >= kRing && !mbar_wait(s_full(s3), ((m - kRing) / kRing) & 1, a.err, kErrWaitMma))
+        return false;
+      if (lane == 0) {
+        meta[sm] = r;
+        mbar_arrive(meta_full(sm));
+        load_blocks(&tk, sbase + L::kKOff + s3 * L::kKVBytes, k_full(s3), r);
+      }
+      __syncwarp();
+      ++m;
+      while (vnext <= m - 3)
+        if (!emit_v()) return false;
       return true;
     };
     while (ok) {
@@ -205,9 +242,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) item = atomicAdd(a.counter, 1);
       item = __shfl_sync(0xFFFFFFFFu, item, 0);
       if (item >= a.items) {
-        StepMeta m{};
-        m.nb = -1;
-        emit(m);
+        // one end record per softmax group (they take alternate steps), then
+        // the V blocks still owed
+        StepMeta r{};
+        r.nb = -1;
+        const int last_real = m;
+        if (emit(r) && emit(r))
+          while (vnext < last_real && emit_v()) {
+          }
         break;
       }
       item = a.order[item];
@@ -240,6 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int64_t i0 = 0, i1 = 0, w0 = -kListWin, w1 = -kListWin;
       StepMeta pend{};
       pend.bh = bh; pend.r0 = r0; pend.r1 = r1;
+      pend.seq = nitems - 1;
       pend.nb = 0; pend.first_last = 1;
       bool have_pending = false;
       StepMeta cur = pend;
@@ -248,13 +291,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (i0 < n0 && i0 >= w0 + kListWin) {
           w0 = i0;
           __syncwarp();
-          for (int j = lane; j < kListWin && w0 + j < n0; j += 32) list0[j] = a.col_idx[b0 + w0 + j];
+          if (lane < kListWin && w0 + lane < n0) list0[lane] = a.col_idx[b0 + w0 + lane];
           __syncwarp();
         }
         if (i1 < n1 && i1 >= w1 + kListWin) {
           w1 = i1;
           __syncwarp();
-          for (int j = lane; j < kListWin && w1 + j < n1; j += 32) list1[j] = a.col_idx[b1 + w1 + j];
+          if (lane < kListWin && w1 + lane < n1) list1[lane] = a.col_idx[b1 + w1 + lane];
           __syncwarp();
         }
         const int c0 = i0 < n0 ? list0[i0 - w0] : 0x7FFFFFFF;
@@ -298,176 +341,193 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(ok = emit(pend))) break;
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    uint32_t q_phase = 0, oe_phase = 0;
-    bool first_item = true;
-    bool ok = true;
-    constexpr uint32_t kIdescO = idesc_bf16(128, D, false, true);
-    const uint32_t qb = sbase + L::kQOff;
-    // Waits for step n's key blocks and returns its record.
-    auto fetch = [&](int n, StepMeta &m) -> bool {
-      if (!mbar_wait(k_full(n % 3), (n / 3) & 1, a.err, kErrWaitTma)) return false;
-      m = meta[n % kMetaRing];
-      return true;
-    };
-    // S_n = Q K_n^T into S[n%2]; releases the K stage and, after an item's
-    // last step, the Q tile.
-    auto issue_s = [&](int n, const StepMeta &m) -> bool {
-      if (m.first_last & 1) {
-        if (!mbar_wait(q_full, q_phase, a.err, kErrWaitTma)) return false;
+    // ------------------------------------------------------------ S issuer
+    uint32_t q_phase = 0;
+    constexpr uint32_t kIdescS1 = idesc_bf16(128, 64, false, false);
+    constexpr uint32_t kIdescS2 = idesc_bf16(128, 128, false, false);
+    constexpr uint32_t kStageUnits = L::kKVBytes >> 4;   // one stage in 16-byte units
+    // Descriptors are built once; per MMA only the 14-bit start-address field
+    // (16-byte units, low word) moves.
+    const uint64_t q_desc = smem_desc(sbase + L::kQOff, 16, 1024);
+    const uint64_t k_desc0 = smem_desc(sbase + L::kKOff, 16, 1024);
+    for (int n = 0;; ++n) {
+      const int b = n % kRing;
+      if (!mbar_wait(k_full(b), (n / kRing) & 1, a.err, kErrWaitTma)) break;
+      const StepMeta r = meta[n % kMetaRing];
+      if (r.nb < 0) break;
+      // S_n overwrites the buffer whose first columns held P_{n-3}: PV_{n-3}
+      // must have finished reading it (consecutive MMAs overlap in the pipe).
+      // At most PV_{n-3} can have completed into this buffer yet, so the
+      // parity names it exactly.
+      if (n >= kRing && !mbar_wait(pv_buf(b), ((n - kRing) / kRing) & 1, a.err, kErrWaitMma)) break;
+      if (r.first_last & 1) {
+        if (!mbar_wait(q_full, q_phase, a.err, kErrWaitTma)) break;
         q_phase ^= 1u;
       }
       tc_fence_after();
-      if (lane == 0 && m.nb > 0) {
-        const uint32_t kb = sbase + L::kKOff + (n % 3) * L::kKVBytes;
-        const uint32_t idesc_s = idesc_bf16(128, 64 * m.nb, false, false);
-        const uint32_t dcol = tmem + ((n & 1) ? kColS1 : kColS0);
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint64_t ad = smem_desc(qb + (k >> 2) * (128 * 128) + (k & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc(kb + (k >> 2) * (2 * 64 * 128) + (k & 3) * 32, 16, 1024);
-          mma_bf16_ss(dcol, ad, bd, idesc_s, k > 0);
-        }
-      }
-      __syncwarp();
       if (lane == 0) {
-        mma_commit(s_full(n & 1));
-        mma_commit(k_empty(n % 3));
-        if (m.first_last & 2) mma_commit(q_empty);
+        if (r.nb > 0) {
+          const uint64_t kd = k_desc0 + static_cast<uint32_t>(b) * kStageUnits;
+          const uint32_t idesc_s = r.nb > 1 ? kIdescS2 : kIdescS1;
+          const uint32_t dcol = tmem + static_cast<uint32_t>(b) * 128u;
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            // k-th 16-column slice: 32 B inside the 128 B swizzle row, d-halves 16 KiB apart
+            const uint32_t off = (k >> 2) * 1024 + (k & 3) * 2;
+            mma_bf16_ss(dcol, q_desc + off, kd + off, idesc_s, k > 0);
+          }
+        }
+        mma_commit(s_full(b));          // also frees K stage b
+        if (r.first_last & 2) mma_commit(q_empty);
       }
       __syncwarp();
-      return true;
-    };
-    // O (+)= P_n V_n; releases the V stage.
-    auto issue_pv = [&](int n, const StepMeta &m) -> bool {
-      if (!mbar_wait(p_full(n & 1), (n >> 1) & 1, a.err, kErrWaitSoftmax)) return false;
-      if (m.first_last & 1) {
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ PV issuer
+    uint32_t oe_phase = 0;
+    bool first_item = true;
+    constexpr uint32_t kIdescO = idesc_bf16(128, D, false, true);
+    constexpr uint32_t kStageUnits = L::kKVBytes >> 4;
+    const uint64_t v_desc0 = smem_desc(sbase + L::kVOff, 2 * 64 * 128, 1024);
+    for (int n = 0;; ++n) {
+      const int b = n % kRing;
+      // the step record tells an end record apart (no P will come); slot n%8
+      // is rewritten only for step n+8, after S_{n+5}, which waits for PV_{n+2}
+      if (!mbar_wait(meta_full(n % kMetaRing), (n / kMetaRing) & 1, a.err, kErrWaitTma)) break;
+      const StepMeta r = meta[n % kMetaRing];
+      if (r.nb < 0) break;
+      // 4 slots: step n+4 needs S_{n+4}, issued only after PV_{n+1}, so this
+      // barrier is never two phases ahead of the wait
+      if (!mbar_wait(p_full(n & 3), (n >> 2) & 1, a.err, kErrWaitSoftmax)) break;
+      if (r.first_last & 1) {
         if (!first_item) {
-          if (!mbar_wait(o_empty, oe_phase, a.err, kErrWaitSoftmax)) return false;
+          if (!mbar_wait(o_empty, oe_phase, a.err, kErrWaitSoftmax)) break;
           oe_phase ^= 1u;
         }
         first_item = false;
       }
-      if (!mbar_wait(v_full(n % 3), (n / 3) & 1, a.err, kErrWaitTma)) return false;
+      if (!mbar_wait(v_full(b), (n / kRing) & 1, a.err, kErrWaitTma)) break;
       tc_fence_after();
-      if (lane == 0 && m.nb > 0) {
-        const uint32_t vb = sbase + L::kVOff + (n % 3) * L::kKVBytes;
-        const uint32_t pcol = tmem + ((n & 1) ? kColP1 : kColP0);
-        for (int k = 0; k < 4 * m.nb; ++k) {
-          const uint64_t bd = smem_desc(vb + k * 2048, 2 * 64 * 128, 1024);
-          mma_bf16_ts(tmem + kColO, pcol + k * 8, bd, kIdescO, !((m.first_last & 1) && k == 0));
-        }
-      }
-      __syncwarp();
       if (lane == 0) {
-        mma_commit(v_empty(n % 3));
-        mma_commit(pv_done);
-        if (m.first_last & 2) mma_commit(o_full);
+        if (r.nb > 0) {
+          const uint64_t vd = v_desc0 + static_cast<uint32_t>(b) * kStageUnits;
+          const uint32_t pcol = tmem + static_cast<uint32_t>(b) * 128u;   // P_n in S[n%3]
+          const bool acc0 = !(r.first_last & 1);
+          // 16 keys per MMA: 8 TMEM columns of P, 2 KiB of V
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_bf16_ts(tmem + kColO, pcol + k * 8, vd + k * 128, kIdescO, acc0 || k > 0);
+          if (r.nb > 1) {
+#pragma unroll
+            for (int k = 4; k < 8; ++k)
+              mma_bf16_ts(tmem + kColO, pcol + k * 8, vd + k * 128, kIdescO, true);
+          }
+        }
+        mma_commit(pv_buf(b));          // also frees V stage b
+        if (r.first_last & 2) mma_commit(o_full);
       }
       __syncwarp();
-      return true;
-    };
-    StepMeta cur, nxt;
-    int n = 0;
-    if (fetch(0, cur) && cur.nb >= 0 && issue_s(0, cur)) {
-      while (ok) {
-        if (!(ok = fetch(n + 1, nxt))) break;
-        const bool more = nxt.nb >= 0;
-        const bool next_first = more && (nxt.first_last & 1);
-        // the next step's scores go first unless it opens a new item (its Q
-        // tile may still be loading; finish this item first)
-        if (more && !next_first && !(ok = issue_s(n + 1, nxt))) break;
-        if (!(ok = issue_pv(n, cur))) break;
-        if (next_first && !(ok = issue_s(n + 1, nxt))) break;
-        if (!more) break;
-        ++n;
-        cur = nxt;
-      }
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
+    const int grp = (warp - 2) >> 2;          // 0: even steps, 1: odd steps
     const int quarter = warp & 3;              // TMEM lane quarter of this warp
     const int row = quarter * 32 + lane;       // query row within the tile
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const uint32_t sel = row >= 64 ? 1u : 0u;
-    uint32_t o_phase = 0;
-    float m_run = -INFINITY, l_run = 0.0f;
-    for (int n = 0;; ++n) {
-      if (!mbar_wait(meta_full(n % kMetaRing), (n / kMetaRing) & 1, a.err, kErrWaitTma)) break;
-      const StepMeta m = meta[n % kMetaRing];
+    for (int n = grp;; n += 2) {
+      const int sm = n % kMetaRing;
+      if (!mbar_wait(meta_full(sm), (n / kMetaRing) & 1, a.err, kErrWaitTma)) break;
+      const StepMeta m = meta[sm];
+      mbar_arrive(meta_empty(sm));
       if (m.nb < 0) break;
       const bool first = m.first_last & 1, last = m.first_last & 2;
-      if (first) {
-        m_run = -INFINITY;
-        l_run = 0.0f;
-      }
-      if (!mbar_wait(s_full(n & 1), (n >> 1) & 1, a.err, kErrWaitMma)) break;
+      const int sb = n % kRing;
+      const uint32_t s_addr = lane_addr + static_cast<uint32_t>(sb) * 128u;
+      if (!mbar_wait(s_full(sb), (n / kRing) & 1, a.err, kErrWaitMma)) break;
       tc_fence_after();
       // warps hold rows of one query block, so v0 / v1 are warp-uniform
       const bool v0 = (m.flags >> sel) & 1u;
       const bool v1 = m.nb > 1 && ((m.flags >> (2 + sel)) & 1u);
-      float x[128];
       float mx = -INFINITY;
-      if (m.nb > 0) {
-        const uint32_t scol = lane_addr + ((n & 1) ? kColS1 : kColS0);
-        tmem_ld64x2(scol, scol + 64, x);
-        if (v0) {
+      {
+        // pass 1: row max over the valid halves, 64 scores live at a time
+        float m8[8];
 #pragma unroll
-          for (int j = 0; j < 64; ++j) mx = fmaxf(mx, x[j]);
-        }
-        if (v1) {
+        for (int i = 0; i < 8; ++i) m8[i] = -INFINITY;
 #pragma unroll
-          for (int j = 64; j < 128; ++j) mx = fmaxf(mx, x[j]);
+        for (int h = 0; h < 2; ++h) {
+          if (h ? v1 : v0) {
+            float x[64];
+            tmem_ld64(s_addr + 64 * h, x);
+#pragma unroll
+            for (int j = 0; j < 64; ++j) m8[j & 7] = fmaxf(m8[j & 7], x[j]);
+          }
         }
+        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         mx *= a.c;
       }
+      // running max of the previous step (the other group); every step waits
+      // for it so that the hand-off barriers stay in lock step
+      float m_prev = -INFINITY;
+      if (n > 0) {
+        if (!mbar_wait(m_full((n - 1) & 1), ((n - 1) >> 1) & 1, a.err, kErrWaitSoftmax)) break;
+        if (!first) m_prev = m_sh[((n - 1) & 1) * 128 + row];
+      }
       // lazy rescale: move the reference max only when it grows by > 8 (2^8)
-      float alpha = 1.0f;
+      float m_run = m_prev, alpha = 1.0f;
       bool resc = false;
-      if (mx > m_run + 8.0f) {
-        if (m_run != -INFINITY) {
-          alpha = ex2(m_run - mx);
+      if (mx > m_prev + 8.0f) {
+        if (m_prev != -INFINITY) {
+          alpha = ex2(m_prev - mx);
           resc = true;
         }
-        l_run *= alpha;
         m_run = mx;
       }
+      m_sh[(n & 1) * 128 + row] = m_run;
+      mbar_arrive(m_full(n & 1));
       const float mref = m_run == -INFINITY ? 0.0f : m_run;
-      float rs = 0.0f;
-      if (m.nb > 0) {
-        uint32_t pk[64];
-        if (v0) {
+      float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // partial row sums
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float p0 = ex2(fmaf(x[2 * j], a.c, -mref));
-            const float p1 = ex2(fmaf(x[2 * j + 1], a.c, -mref));
-            rs += p0 + p1;
-            pk[j] = pack_bf16x2(p0, p1);
+      for (int h = 0; h < 2; ++h) {
+        if (h < m.nb) {
+          // pass 2, one 64-key half at a time; P of half h overwrites S
+          // columns [32h, 32h+32), which hold scores already read
+          const bool valid = h ? v1 : v0;
+          uint32_t pk[32];
+          if (valid) {
+            float x[64];
+            tmem_ld64(s_addr + 64 * h, x);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float p0 = ex2(fmaf(x[2 * j], a.c, -mref));
+              const float p1 = ex2(fmaf(x[2 * j + 1], a.c, -mref));
+              r8[j & 7] += p0 + p1;
+              pk[j] = pack_bf16x2(p0, p1);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) pk[j] = 0u;
           }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) pk[j] = 0u;
+          tmem_st32u(s_addr + 32 * h, pk);
         }
-        if (v1) {
-#pragma unroll
-          for (int j = 32; j < 64; ++j) {
-            const float p0 = ex2(fmaf(x[2 * j], a.c, -mref));
-            const float p1 = ex2(fmaf(x[2 * j + 1], a.c, -mref));
-            rs += p0 + p1;
-            pk[j] = pack_bf16x2(p0, p1);
-          }
-        } else {
-#pragma unroll
-          for (int j = 32; j < 64; ++j) pk[j] = 0u;
-        }
-        const uint32_t pcol = lane_addr + ((n & 1) ? kColP1 : kColP0);
-        tmem_st32u(pcol, pk);
-        if (m.nb > 1) tmem_st32u(pcol + 32, pk + 32);
       }
-      l_run += rs;
+      const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
+      // running sum: the previous step's value (other group), rescaled
+      float l_prev = 0.0f;
+      if (n > 0) {
+        if (!mbar_wait(l_full((n - 1) & 1), ((n - 1) >> 1) & 1, a.err, kErrWaitSoftmax)) break;
+        if (!first) l_prev = l_sh[((n - 1) & 1) * 128 + row];
+      }
+      const float l_run = l_prev * alpha + rs;
+      l_sh[(n & 1) * 128 + row] = l_run;
+      mbar_arrive(l_full(n & 1));
       if (__any_sync(0xFFFFFFFFu, resc)) {
-        // O must hold PV_{n-1} before it is rescaled
-        if (!mbar_wait(pv_done, (n - 1) & 1, a.err, kErrWaitMma)) break;
+        // O must hold PV_{n-1} before it is rescaled.  S_n was issued only
+        // after PV_{n-3} completed, so buffer (n-1)%3 has finished every PV
+        // before PV_{n-1} and the parity names PV_{n-1} exactly.
+        if (!mbar_wait(pv_buf((n - 1) % kRing), ((n - 1) / kRing) & 1, a.err, kErrWaitMma)) break;
         tc_fence_after();
 #pragma unroll 1
         for (int cc = 0; cc < D; cc += 32) {
@@ -480,10 +540,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full(n & 1));
+      mbar_arrive(p_full(n & 3));
       if (last) {
-        if (!mbar_wait(o_full, o_phase, a.err, kErrWaitMma)) break;
-        o_phase ^= 1u;
+        if (!mbar_wait(o_full, static_cast<uint32_t>(m.seq) & 1u, a.err, kErrWaitMma)) break;
         tc_fence_after();
         const int rblk = sel ? m.r1 : m.r0;
         const bool store = rblk >= 0;
@@ -677,20 +736,30 @@ cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
   a.lse_scale = 0.6931471805599453f;
   int grid = num_sms();
   if (L.items < grid) grid = static_cast<int>(L.items);
-  if (g.d == 128) {
-    const int smem = Smem<128>::kAlloc;
-    if ((e = cudaFuncSetAttribute(sparse_attn_kernel<128>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
-      return e;
+  const void *fn = g.d == 128 ? reinterpret_cast<const void *>(sparse_attn_kernel<128>)
+                              : reinterpret_cast<const void *>(sparse_attn_kernel<64>);
+  const int smem = g.d == 128 ? Smem<128>::kAlloc : Smem<64>::kAlloc;
+  if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+      cudaSuccess)
+    return e;
+  if (g.d == 128)
     sparse_attn_kernel<128><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
-  } else {
-    const int smem = Smem<64>::kAlloc;
-    if ((e = cudaFuncSetAttribute(sparse_attn_kernel<64>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
-      return e;
+  else
     sparse_attn_kernel<64><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    // report what the kernel needs next to what the launch asked for
+    static thread_local char msg[256];
+    cudaFuncAttributes fa{};
+    cudaFuncGetAttributes(&fa, fn);
+    snprintf(msg, sizeof msg,
+             "sparse attention launch: %s (threads %d, regs/thread %d, max threads/block %d, "
+             "static smem %zu, dynamic smem %d)",
+             cudaGetErrorString(e), kThreads, fa.numRegs, fa.maxThreadsPerBlock,
+             fa.sharedSizeBytes, smem);
+    *why = msg;
   }
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace vsa

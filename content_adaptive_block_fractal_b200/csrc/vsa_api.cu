@@ -213,7 +213,8 @@ vsa_status vsa_sparse_attn_fwd(const void *qf, const void *kf, const void *vf,
   e = vsa::launch_sparse_attn(qf, kf, vf, row_ptr, col_idx, g, scale, o, lse, workspace, err,
                               static_cast<cudaStream_t>(stream), &why);
   if (e != cudaSuccess)
-    return why ? fail(VSA_ERR_UNSUPPORTED, "%s", why) : cuda_fail(e, "sparse attention launch");
+    return why ? fail(e == cudaErrorInvalidValue ? VSA_ERR_UNSUPPORTED : VSA_ERR_CUDA, "%s", why)
+               : cuda_fail(e, "sparse attention launch");
   return VSA_OK;
 }
 
@@ -230,7 +231,7 @@ vsa_status vsa_device_status(void *stream) {
   if ((e = cudaMemcpy(err, &zero, sizeof zero, cudaMemcpyHostToDevice)) != cudaSuccess)
     return cuda_fail(e, "clear device error word");
   return fail(VSA_ERR_DEVICE_TIMEOUT,
-              "device error word 0x%x (1: TMA wait, 2: MMA wait, 4: softmax wait, 8: bad block index)",
+              "device error word 0x%x (1: TMA wait, 2: MMA wait, 4: softmax wait, 8: bad block index, 16: shared memory misaligned)",
               v);
 }
 
