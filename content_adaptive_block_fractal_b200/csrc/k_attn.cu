@@ -15,12 +15,14 @@
 // Three S buffers let the MMA warp keep the scores up to two steps ahead of
 // the softmax: the tensor core runs S_{n+2} while P_n is being formed; S_{n+3}
 // reuses step n's buffer only after PV_n has completed.
-// Warp roles (352 threads, one CTA per SM, persistent):
+// Warp roles (384 threads, one CTA per SM, persistent):
 //   warp 0      producer: takes items from an atomic counter over a
 //               longest-first work list, merges the two CSR lists, publishes
-//               one step record per step (8-deep ring) and issues TMA loads
-//               (128B-swizzled boxes): Q per item, K of step m and V of step
-//               m-2, each into a 3-deep ring;
+//               one step record per step (8-deep ring) and issues the TMA
+//               loads (128B-swizzled boxes) of Q per item and of K per step
+//               into a 3-deep ring;
+//   warp 11     V producer: follows the step records and loads V per step
+//               into its own 3-deep ring;
 //   warp 1      allocates 512 TMEM columns; one lane issues the S MMAs;
 //   warp 10     one lane issues the PV MMAs.  tcgen05.mma issue is paced by
 //               the tensor core, so two issuers let one's waits overlap the
@@ -43,7 +45,7 @@
 namespace vsa {
 namespace {
 
-constexpr int kThreads = 352;
+constexpr int kThreads = 384;
 constexpr int kRing = 3;               // K stages, V stages, S buffers
 constexpr int kMetaRing = 8;
 constexpr int kListWin = 32;           // CSR entries staged per list in SMEM
@@ -62,7 +64,8 @@ struct StepMeta {
 template <int D>
 struct Smem {
   static constexpr int kQBytes = 128 * D * 2;             // two query blocks
-  static constexpr int kKVBytes = 2 * 64 * D * 2;         // K (or V) of two key blocks
+  static constexpr int kBlockBytes = 64 * D * 2;          // one key block: [d-half][64 rows][128 B]
+  static constexpr int kKVBytes = 2 * kBlockBytes;         // K (or V) of two key blocks
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kQBytes;
   static constexpr int kVOff = kKOff + kRing * kKVBytes;
@@ -184,42 +187,11 @@ __global__ void __maxnreg__(168)
       tma_prefetch_desc(&tv);
     }
     int m = 0;               // next step whose record and K blocks go out
-    int vnext = 0;           // next step whose V blocks go out
     uint32_t q_phase = 0;
     bool ok = true;
     int nitems = 0;
-    // TMA of the (one or two) key blocks of step record r into a 3-stage ring.
-    auto load_blocks = [&](const CUtensorMap *map, uint32_t base, uint32_t bar_full,
-                           const StepMeta &r) {
-      const int nb = r.nb > 0 ? r.nb : 0;
-      mbar_arrive_expect_tx(bar_full, static_cast<uint32_t>(nb * 64 * D * 2));
-      const int head_row = static_cast<int>(static_cast<int64_t>(r.bh) * a.N);
-      if (nb > 0) {
-#pragma unroll
-        for (int dh = 0; dh < D / 64; ++dh)
-          tma_load_2d(base + dh * 16384, map, bar_full, dh * 64, head_row + r.blk0 * 64);
-        if (nb > 1) {
-#pragma unroll
-          for (int dh = 0; dh < D / 64; ++dh)
-            tma_load_2d(base + dh * 16384 + 8192, map, bar_full, dh * 64, head_row + r.blk1 * 64);
-        }
-      }
-    };
-    // V blocks of step vnext (two steps behind the K blocks).
-    auto emit_v = [&]() -> bool {
-      const int s3 = vnext % kRing;
-      // the stage's previous user PV_{vnext-3} has completed (its pv_buf)
-      if (vnext >= kRing &&
-          !mbar_wait(pv_buf(s3), ((vnext - kRing) / kRing) & 1, a.err, kErrWaitMma))
-        return false;
-      if (lane == 0)
-        load_blocks(&tv, sbase + L::kVOff + s3 * L::kKVBytes, v_full(s3), meta[vnext % kMetaRing]);
-      __syncwarp();
-      ++vnext;
-      return true;
-    };
-    // Publishes step record r as step m and loads its K blocks; the V blocks
-    // of step m-2 follow.
+    // Publishes step record r as step m and loads its K blocks (one 3-D box
+    // per block: 64 rows x all d-halves, block-major in the stage).
     auto emit = [&](const StepMeta &r) -> bool {
       const int s3 = m % kRing, sm = m % kMetaRing;
       if (!mbar_wait(meta_empty(sm), ((m / kMetaRing) & 1) ^ 1, a.err, kErrWaitSoftmax)) return false;
@@ -229,12 +201,16 @@ __global__ void __maxnreg__(168)
       if (lane == 0) {
         meta[sm] = r;
         mbar_arrive(meta_full(sm));
-        load_blocks(&tk, sbase + L::kKOff + s3 * L::kKVBytes, k_full(s3), r);
+        const int nb = r.nb > 0 ? r.nb : 0;
+        const uint32_t kf = k_full(s3);
+        mbar_arrive_expect_tx(kf, static_cast<uint32_t>(nb * L::kBlockBytes));
+        const uint32_t kbase = sbase + L::kKOff + s3 * L::kKVBytes;
+        const int head_row = static_cast<int>(static_cast<int64_t>(r.bh) * a.N);
+        if (nb > 0) tma_load_3d(kbase, &tk, kf, 0, head_row + r.blk0 * 64, 0);
+        if (nb > 1) tma_load_3d(kbase + L::kBlockBytes, &tk, kf, 0, head_row + r.blk1 * 64, 0);
       }
       __syncwarp();
       ++m;
-      while (vnext <= m - 3)
-        if (!emit_v()) return false;
       return true;
     };
     while (ok) {
@@ -246,10 +222,7 @@ __global__ void __maxnreg__(168)
         // the V blocks still owed
         StepMeta r{};
         r.nb = -1;
-        const int last_real = m;
-        if (emit(r) && emit(r))
-          while (vnext < last_real && emit_v()) {
-          }
+        if (emit(r)) emit(r);
         break;
       }
       item = a.order[item];
@@ -344,7 +317,6 @@ __global__ void __maxnreg__(168)
     // ------------------------------------------------------------ S issuer
     uint32_t q_phase = 0;
     constexpr uint32_t kIdescS1 = idesc_bf16(128, 64, false, false);
-    constexpr uint32_t kIdescS2 = idesc_bf16(128, 128, false, false);
     constexpr uint32_t kStageUnits = L::kKVBytes >> 4;   // one stage in 16-byte units
     // Descriptors are built once; per MMA only the 14-bit start-address field
     // (16-byte units, low word) moves.
@@ -366,15 +338,20 @@ __global__ void __maxnreg__(168)
       }
       tc_fence_after();
       if (lane == 0) {
-        if (r.nb > 0) {
-          const uint64_t kd = k_desc0 + static_cast<uint32_t>(b) * kStageUnits;
-          const uint32_t idesc_s = r.nb > 1 ? kIdescS2 : kIdescS1;
-          const uint32_t dcol = tmem + static_cast<uint32_t>(b) * 128u;
+        // one N=64 MMA chain per key block: S columns [64j, 64j+64)
+        const uint64_t kd = k_desc0 + static_cast<uint32_t>(b) * kStageUnits;
+        const uint32_t dcol = tmem + static_cast<uint32_t>(b) * 128u;
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            // k-th 16-column slice: 32 B inside the 128 B swizzle row, d-halves 16 KiB apart
-            const uint32_t off = (k >> 2) * 1024 + (k & 3) * 2;
-            mma_bf16_ss(dcol, q_desc + off, kd + off, idesc_s, k > 0);
+        for (int j = 0; j < 2; ++j) {
+          if (j < r.nb) {
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+              // k-th 16-column slice: 32 B inside the 128 B swizzle row; Q
+              // d-halves 16 KiB apart, K d-halves 8 KiB apart inside a block
+              const uint32_t qoff = (k >> 2) * 1024 + (k & 3) * 2;
+              const uint32_t koff = j * (L::kBlockBytes >> 4) + (k >> 2) * 512 + (k & 3) * 2;
+              mma_bf16_ss(dcol + 64 * j, q_desc + qoff, kd + koff, kIdescS1, k > 0);
+            }
           }
         }
         mma_commit(s_full(b));          // also frees K stage b
@@ -388,7 +365,9 @@ __global__ void __maxnreg__(168)
     bool first_item = true;
     constexpr uint32_t kIdescO = idesc_bf16(128, D, false, true);
     constexpr uint32_t kStageUnits = L::kKVBytes >> 4;
-    const uint64_t v_desc0 = smem_desc(sbase + L::kVOff, 2 * 64 * 128, 1024);
+    // V is an MN-major operand: 8-key groups 1 KiB apart (SBO), d-halves of a
+    // block 8 KiB apart (LBO), blocks kBlockBytes apart
+    const uint64_t v_desc0 = smem_desc(sbase + L::kVOff, 64 * 128, 1024);
     for (int n = 0;; ++n) {
       const int b = n % kRing;
       // the step record tells an end record apart (no P will come); slot n%8
@@ -418,13 +397,37 @@ __global__ void __maxnreg__(168)
           for (int k = 0; k < 4; ++k)
             mma_bf16_ts(tmem + kColO, pcol + k * 8, vd + k * 128, kIdescO, acc0 || k > 0);
           if (r.nb > 1) {
+            const uint64_t vd1 = vd + (L::kBlockBytes >> 4);
 #pragma unroll
-            for (int k = 4; k < 8; ++k)
-              mma_bf16_ts(tmem + kColO, pcol + k * 8, vd + k * 128, kIdescO, true);
+            for (int k = 0; k < 4; ++k)
+              mma_bf16_ts(tmem + kColO, pcol + 32 + k * 8, vd1 + k * 128, kIdescO, true);
           }
         }
         mma_commit(pv_buf(b));          // also frees V stage b
         if (r.first_last & 2) mma_commit(o_full);
+      }
+      __syncwarp();
+    }
+  } else if (warp == 11) {
+    // ------------------------------------------------------------ V producer
+    if (lane == 0) tma_prefetch_desc(&tv);
+    for (int n = 0;; ++n) {
+      const int b = n % kRing;
+      // slot n%8 is rewritten only for step n+8, after S_{n+5}, which waits
+      // for PV_{n+2}, which needs this warp's V_{n+2}
+      if (!mbar_wait(meta_full(n % kMetaRing), (n / kMetaRing) & 1, a.err, kErrWaitTma)) break;
+      const StepMeta r = meta[n % kMetaRing];
+      if (r.nb < 0) break;
+      // the stage's previous user PV_{n-3} has completed (its pv_buf)
+      if (n >= kRing && !mbar_wait(pv_buf(b), ((n - kRing) / kRing) & 1, a.err, kErrWaitMma)) break;
+      if (lane == 0) {
+        const int nb = r.nb > 0 ? r.nb : 0;
+        const uint32_t vf = v_full(b);
+        mbar_arrive_expect_tx(vf, static_cast<uint32_t>(nb * L::kBlockBytes));
+        const uint32_t vbase = sbase + L::kVOff + b * L::kKVBytes;
+        const int head_row = static_cast<int>(static_cast<int64_t>(r.bh) * a.N);
+        if (nb > 0) tma_load_3d(vbase, &tv, vf, 0, head_row + r.blk0 * 64, 0);
+        if (nb > 1) tma_load_3d(vbase + L::kBlockBytes, &tv, vf, 0, head_row + r.blk1 * 64, 0);
       }
       __syncwarp();
     }
@@ -660,6 +663,21 @@ EncodeFn encode_fn() {
   return fn;
 }
 
+// [rows, d] bf16 viewed as (64 elements, rows, d/64 halves): one box is a
+// whole 64-row block, its d-halves stacked (block-major SMEM layout).
+bool make_map3(CUtensorMap *m, const void *base, int64_t rows, int d) {
+  EncodeFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(d / 64)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, 128};
+  const cuuint32_t box[3] = {64, 64, static_cast<cuuint32_t>(d / 64)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 bool make_map(CUtensorMap *m, const void *base, int64_t rows, int d) {
   EncodeFn enc = encode_fn();
   if (!enc) return false;
@@ -706,8 +724,8 @@ cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
   }
   CUtensorMap mq, mk, mv;
   const int64_t rows = g.BH * g.N;
-  if (!make_map(&mq, qf, rows, g.d) || !make_map(&mk, kf, rows, g.d) ||
-      !make_map(&mv, vf, rows, g.d)) {
+  if (!make_map(&mq, qf, rows, g.d) || !make_map3(&mk, kf, rows, g.d) ||
+      !make_map3(&mv, vf, rows, g.d)) {
     *why = "sparse attention: cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
   }
