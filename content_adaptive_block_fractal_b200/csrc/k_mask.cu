@@ -35,6 +35,8 @@ constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kPad = 4;       // fp64 padding per smem row (conflict-free fragments)
 constexpr int kCand = 256;    // per-warp candidate list capacity
+constexpr int kBins = 64;     // 1/8-octave probability bins (8 octaves below the max)
+constexpr int kMaxWords = 256;  // kept-bit words per row held in SMEM (Nb <= 8192)
 constexpr int kMaxGrid = 160; // slabs in the workspace
 
 struct MaskArgs {
@@ -101,10 +103,99 @@ __device__ __forceinline__ bool sta_keep(int r, int c, const MaskArgs &a) {
   return abs(tr - tc) <= a.rt && abs(yr - yc) <= a.rh && abs(xr - xc) <= a.rw;
 }
 
+// key = bits of a probability in [0, 1]; bin 0 holds (7/8, 1], each bin is
+// 1/8 octave; kBins (the tail) collects everything more than 8 octaves down.
+__device__ __forceinline__ int prob_bin(uint32_t key) {
+  const uint32_t d = key < 0x3F800000u ? 0x3F800000u - key : 0u;
+  const uint32_t b = d >> 20;
+  return b < static_cast<uint32_t>(kBins) ? static_cast<int>(b) : kBins;
+}
+
+// The cut by bisection on the fp32 bit pattern, mass tests in fp64.  Sets
+// vkey (cut value) and need_ties, or keep_all when the sums never reach the
+// target.  General path; used when the histogram path cannot decide.
+__device__ void cut_by_bisection(int Nb, const float *ebuf, uint32_t kmax, double target,
+                                 uint32_t *cand_key, int32_t *cand_idx, uint32_t &vkey,
+                                 int &need_ties, bool &keep_all) {
+  const int lane = threadIdx.x & 31;
+  // Invariant: the cut key lies in [lo, hi); mass(key >= hi) = base < target.
+  uint32_t lo = 0, hi = kmax + 1;
+  double base = 0.0;
+  int ncand = -1;  // -1: scan the whole row
+  for (int it = 0; hi - lo > 1; ++it) {
+    const uint32_t mid = lo + ((hi - lo) >> 1);
+    double up = 0.0;
+    if (ncand < 0) {
+      for (int c = lane; c < Nb; c += 32) {
+        const float e = ebuf[c];
+        const uint32_t k = __float_as_uint(e);
+        if (k >= mid && k < hi) up += static_cast<double>(e);
+      }
+    } else {
+      for (int i = lane; i < ncand; i += 32) {
+        const uint32_t k = cand_key[i];
+        if (k >= mid && k < hi) up += static_cast<double>(__uint_as_float(k));
+      }
+    }
+    up = warp_sum(up);
+    if (base + up >= target) {
+      lo = mid;
+    } else {
+      base += up;
+      hi = mid;
+    }
+    if (ncand < 0 && it >= 5) {
+      int cnt = 0;
+      for (int c = lane; c < Nb; c += 32) {
+        const uint32_t k = __float_as_uint(ebuf[c]);
+        cnt += (k >= lo && k < hi);
+      }
+      cnt = warp_sum_i(cnt);
+      if (cnt <= kCand) {
+        int pos = 0;
+        for (int c0 = 0; c0 < Nb; c0 += 32) {
+          const int c = c0 + lane;
+          const uint32_t k = c < Nb ? __float_as_uint(ebuf[c]) : 0u;
+          const bool in = c < Nb && k >= lo && k < hi;
+          const uint32_t m = __ballot_sync(0xFFFFFFFFu, in);
+          if (in) {
+            const int p = pos + __popc(m & ((1u << lane) - 1u));
+            cand_key[p] = k;
+            cand_idx[p] = c;
+          }
+          pos += __popc(m);
+        }
+        ncand = pos;
+        __syncwarp();
+      }
+    }
+  }
+  vkey = lo;
+  if (vkey == 0u) {
+    keep_all = true;  // the sums never reach 1 - thr: keep every block
+  } else {
+    const double v = static_cast<double>(__uint_as_float(vkey));
+    int j = static_cast<int>(ceil((target - base) / v));
+    if (j < 1) j = 1;
+    while (j > 1 && base + (j - 1) * v >= target) --j;
+    while (base + j * v < target && j < Nb) ++j;
+    need_ties = j;
+  }
+}
+
 // Phase B for one row: selection and kept bits.  ebuf: this warp's Nb floats.
+//   1. probabilities relative to the row max into ebuf, their fp64 sum, and a
+//      histogram of counts / fp32 masses over 1/8-octave bins;
+//   2. the bin b where the cumulative mass reaches 1 - thr; an exact fp64 pass
+//      confirms base = mass above b < target <= base + mass of b and collects
+//      the bin's entries;
+//   3. with at most 32 entries: a warp bitonic sort on (probability desc,
+//      index asc) and an fp64 prefix scan mark the kept ones.  Otherwise (or
+//      if the fp32 histogram misled step 2) the bisection path decides.
 __device__ void select_row(const MaskArgs &a, int64_t grow, int r, const float *slab_row,
                            const double *tmax_row, float *ebuf, uint32_t *cand_key,
-                           int32_t *cand_idx, double *tscale) {
+                           int32_t *cand_idx, double *tscale, int *hcnt, float *hmass,
+                           uint32_t *wbits) {
   const int lane = threadIdx.x & 31;
   const int Nb = a.Nb;
   // row maximum over the tile maxima, per-tile rescale factors in fp64
@@ -112,108 +203,189 @@ __device__ void select_row(const MaskArgs &a, int64_t grow, int r, const float *
   for (int t = lane; t < a.ntiles; t += 32) M = fmax(M, tmax_row[t]);
   M = warp_max(M);
   for (int t = lane; t < a.ntiles; t += 32) tscale[t] = exp2(tmax_row[t] - M);
+  for (int b = lane; b < kBins; b += 32) {
+    hcnt[b] = 0;
+    hmass[b] = 0.0f;
+  }
   __syncwarp();
+  const bool need_cut = a.thr > 0.0f;
   double z = 0.0;
   uint32_t kmax = 0;
-  for (int c = lane; c < Nb; c += 32) {
-    const float e = static_cast<float>(static_cast<double>(slab_row[c]) * tscale[c / kCT]);
-    ebuf[c] = e;
-    z += static_cast<double>(e);
-    kmax = max(kmax, __float_as_uint(e));
+  // the slab row sits in L2: 16-byte loads, four in flight per lane, before
+  // any use (the row is padded to a multiple of 4 floats)
+  constexpr int kU = 4;
+  for (int c0 = 4 * lane; c0 < Nb; c0 += 128 * kU) {
+    float4 v[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+      if (c0 + 128 * u < Nb) v[u] = *reinterpret_cast<const float4 *>(slab_row + c0 + 128 * u);
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const float x4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = c0 + 128 * u + j;
+        if (c < Nb) {
+          const float e = static_cast<float>(static_cast<double>(x4[j]) * tscale[c / kCT]);
+          ebuf[c] = e;
+          z += static_cast<double>(e);
+          const uint32_t k = __float_as_uint(e);
+          kmax = max(kmax, k);
+          if (need_cut) {
+            const int b = prob_bin(k);
+            if (b < kBins) {         // the tail needs no histogram
+              atomicAdd(&hcnt[b], 1);
+              atomicAdd(&hmass[b], e);
+            }
+          }
+        }
+      }
+    }
   }
   z = warp_sum(z);
 #pragma unroll
   for (int o = 16; o; o >>= 1) kmax = max(kmax, __shfl_xor_sync(0xFFFFFFFFu, kmax, o));
   __syncwarp();
 
-  bool keep_all = !(a.thr > 0.0f);
+  bool keep_all = !need_cut;
   uint32_t vkey = 0;
   int need_ties = 0;
+  int cut_bin = -1;       // >= 0: kept = bin < cut_bin, or marked in ebuf (sign bit)
   if (!keep_all) {
     const double target = (1.0 - static_cast<double>(a.thr)) * z;
-    // Invariant: the cut key lies in [lo, hi); mass(key >= hi) = base < target.
-    uint32_t lo = 0, hi = kmax + 1;
-    double base = 0.0;
-    int ncand = -1;  // -1: scan the whole row
-    for (int it = 0; hi - lo > 1; ++it) {
-      const uint32_t mid = lo + ((hi - lo) >> 1);
-      double up = 0.0;
-      if (ncand < 0) {
-        for (int c = lane; c < Nb; c += 32) {
-          const float e = ebuf[c];
-          const uint32_t k = __float_as_uint(e);
-          if (k >= mid && k < hi) up += static_cast<double>(e);
-        }
-      } else {
-        for (int i = lane; i < ncand; i += 32) {
-          const uint32_t k = cand_key[i];
-          if (k >= mid && k < hi) up += static_cast<double>(__uint_as_float(k));
-        }
-      }
-      up = warp_sum(up);
-      if (base + up >= target) {
-        lo = mid;
-      } else {
-        base += up;
-        hi = mid;
-      }
-      if (ncand < 0 && it >= 5) {
-        int cnt = 0;
-        for (int c = lane; c < Nb; c += 32) {
-          const uint32_t k = __float_as_uint(ebuf[c]);
-          cnt += (k >= lo && k < hi);
-        }
-        cnt = warp_sum_i(cnt);
-        if (cnt <= kCand) {
-          int pos = 0;
-          for (int c0 = 0; c0 < Nb; c0 += 32) {
-            const int c = c0 + lane;
-            const uint32_t k = c < Nb ? __float_as_uint(ebuf[c]) : 0u;
-            const bool in = c < Nb && k >= lo && k < hi;
-            const uint32_t m = __ballot_sync(0xFFFFFFFFu, in);
-            if (in) {
-              const int p = pos + __popc(m & ((1u << lane) - 1u));
-              cand_key[p] = k;
-              cand_idx[p] = c;
-            }
-            pos += __popc(m);
+    // 2. cumulative bin masses (8 bins per lane, then a warp scan)
+    double loc = 0.0;
+#pragma unroll
+    for (int i = 0; i < kBins / 32; ++i) loc += static_cast<double>(hmass[lane * (kBins / 32) + i]);
+    double incl = loc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    double run = incl - loc;
+    int found = kBins;
+#pragma unroll
+    for (int i = 0; i < kBins / 32; ++i) {
+      const int b = lane * (kBins / 32) + i;
+      run += static_cast<double>(hmass[b]);
+      if (found == kBins && run >= target) found = b;
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) found = min(found, __shfl_xor_sync(0xFFFFFFFFu, found, o));
+    bool decided = false;
+    if (found < kBins && hcnt[found] <= 32) {
+      // exact mass above the bin and the bin's entries
+      double base = 0.0;
+      int pos = 0;
+      for (int c0 = 0; c0 < Nb; c0 += 32) {
+        const int c = c0 + lane;
+        const float e = c < Nb ? ebuf[c] : 0.0f;
+        const int b = c < Nb ? prob_bin(__float_as_uint(e)) : kBins;
+        if (b < found) base += static_cast<double>(e);
+        const bool in = b == found;
+        const uint32_t m = __ballot_sync(0xFFFFFFFFu, in);
+        if (in) {
+          const int p = pos + __popc(m & ((1u << lane) - 1u));
+          if (p < 32) {
+            cand_key[p] = __float_as_uint(e);
+            cand_idx[p] = c;
           }
-          ncand = pos;
-          __syncwarp();
         }
+        pos += __popc(m);
+      }
+      base = warp_sum(base);
+      __syncwarp();
+      if (pos <= 32 && base < target) {
+        // one entry per lane; sort by (probability desc, index asc)
+        uint64_t key = ~0ull;
+        if (lane < pos)
+          key = (static_cast<uint64_t>(0xFFFFFFFFu - cand_key[lane]) << 32) |
+                static_cast<uint32_t>(cand_idx[lane]);
+#pragma unroll
+        for (int size = 2; size <= 32; size <<= 1)
+#pragma unroll
+          for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            const uint64_t other = __shfl_xor_sync(0xFFFFFFFFu, key, stride);
+            const bool up = (lane & size) == 0;
+            const bool lower = (lane & stride) == 0;
+            const uint64_t lo_v = key < other ? key : other;
+            const uint64_t hi_v = key < other ? other : key;
+            key = (lower == up) ? lo_v : hi_v;
+          }
+        const bool valid = key != ~0ull;
+        const double p = valid ? static_cast<double>(__uint_as_float(0xFFFFFFFFu - static_cast<uint32_t>(key >> 32)))
+                               : 0.0;
+        double inc = p;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const double y = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+          if (lane >= o) inc += y;
+        }
+        const double total = __shfl_sync(0xFFFFFFFFu, inc, 31);
+        if (base + total >= target) {
+          // kept while the mass before the entry is still below the target
+          if (valid && base + (inc - p) < target) {
+            const int c = static_cast<int>(key & 0xFFFFFFFFu);
+            ebuf[c] = __uint_as_float(__float_as_uint(ebuf[c]) | 0x80000000u);
+          }
+          cut_bin = found;
+          decided = true;
+        }
+        __syncwarp();
       }
     }
-    vkey = lo;
-    if (vkey == 0u) {
-      keep_all = true;  // the sums never reach 1 - thr: keep every block
-    } else {
-      const double v = static_cast<double>(__uint_as_float(vkey));
-      int j = static_cast<int>(ceil((target - base) / v));
-      if (j < 1) j = 1;
-      while (j > 1 && base + (j - 1) * v >= target) --j;
-      while (base + j * v < target && j < Nb) ++j;
-      need_ties = j;
-    }
+    if (!decided)
+      cut_by_bisection(Nb, ebuf, kmax, target, cand_key, cand_idx, vkey, need_ties, keep_all);
   }
 
-  // kept bits: above the cut, the first need_ties equal keys in index order,
-  // or the STA window
-  int ties_seen = 0, count = 0;
-  uint32_t *out = a.bits + grow * a.words;
+  // kept bits: above the cut (or marked), ties by index on the bisection path
+  int ties_seen = 0;
   for (int w = 0; w < a.words; ++w) {
     const int c = w * 32 + lane;
     const bool valid = c < Nb;
     const uint32_t k = valid ? __float_as_uint(ebuf[c]) : 0u;
-    bool kept = valid && (keep_all || k > vkey);
-    const bool tie = valid && !keep_all && k == vkey;
-    const uint32_t tm = __ballot_sync(0xFFFFFFFFu, tie);
-    if (tie && ties_seen + __popc(tm & ((1u << lane) - 1u)) < need_ties) kept = true;
-    ties_seen += __popc(tm);
-    if (valid && a.use_sta && sta_keep(r, c, a)) kept = true;
+    bool kept;
+    if (keep_all) {
+      kept = valid;
+    } else if (cut_bin >= 0) {
+      kept = valid && ((k >> 31) || prob_bin(k) < cut_bin);
+    } else {
+      kept = valid && k > vkey;
+      const bool tie = valid && k == vkey;
+      const uint32_t tm = __ballot_sync(0xFFFFFFFFu, tie);
+      if (tie && ties_seen + __popc(tm & ((1u << lane) - 1u)) < need_ties) kept = true;
+      ties_seen += __popc(tm);
+    }
     const uint32_t word = __ballot_sync(0xFFFFFFFFu, kept);
-    if (lane == 0) out[w] = word;
+    if (lane == 0) wbits[w] = word;
+  }
+  __syncwarp();
+  if (a.use_sta) {
+    // the window: at most (2rt+1)(2rh+1)(2rw+1) blocks around the row's own
+    const int hw = a.Hb * a.Wb;
+    const int tr = r / hw, yr = (r / a.Wb) % a.Hb, xr = r % a.Wb;
+    const int nt = 2 * a.rt + 1, ny = 2 * a.rh + 1, nx = 2 * a.rw + 1;
+    const int T = Nb / hw;
+    for (int i = lane; i < nt * ny * nx; i += 32) {
+      const int t = tr - a.rt + i / (ny * nx);
+      const int y = yr - a.rh + (i / nx) % ny;
+      const int x = xr - a.rw + i % nx;
+      if (t >= 0 && t < T && y >= 0 && y < a.Hb && x >= 0 && x < a.Wb) {
+        const int c = (t * a.Hb + y) * a.Wb + x;
+        atomicOr(&wbits[c >> 5], 1u << (c & 31));
+      }
+    }
+    __syncwarp();
+  }
+  uint32_t *out = a.bits + grow * a.words;
+  int count = 0;
+  for (int w = lane; w < a.words; w += 32) {
+    const uint32_t word = wbits[w];
+    out[w] = word;
     count += __popc(word);
   }
+  count = warp_sum_i(count);
   if (lane == 0) a.counts[grow] = count;
   __syncwarp();
 }
@@ -320,17 +492,21 @@ __global__ void __launch_bounds__(kThreads, 1) mask_select_kernel(const MaskArgs
 
     // ---- phase B: one warp per row
     unsigned char *wbase = smem_raw + warp * (static_cast<size_t>(a.Nb) * 4 + kCand * 8 +
-                                              static_cast<size_t>(a.ntiles) * 8 + 16);
+                                              static_cast<size_t>(a.ntiles) * 8 + 16 + kBins * 8 +
+                                              kMaxWords * 4);
     float *ebuf = reinterpret_cast<float *>(wbase);
     uint32_t *cand_key = reinterpret_cast<uint32_t *>(ebuf + a.Nb);
     int32_t *cand_idx = reinterpret_cast<int32_t *>(cand_key + kCand);
     double *tscale = reinterpret_cast<double *>(
         (reinterpret_cast<uintptr_t>(cand_idx + kCand) + 15) & ~static_cast<uintptr_t>(15));
+    int *hcnt = reinterpret_cast<int *>(tscale + a.ntiles);
+    float *hmass = reinterpret_cast<float *>(hcnt + kBins);
+    uint32_t *wbits = reinterpret_cast<uint32_t *>(hmass + kBins);
     for (int row = warp; row < kRT; row += kWarps) {
       const int r = r0 + row;
       if (r >= a.Nb) break;
       select_row(a, bh * a.Nb + r, r, slab + row * a.ld_slab, tmax + row * a.ntiles, ebuf,
-                 cand_key, cand_idx, tscale);
+                 cand_key, cand_idx, tscale, hcnt, hmass, wbits);
     }
     __syncthreads();  // smem and slab are reused by the next item
   }
@@ -419,8 +595,10 @@ MaskLayout mask_layout(const Geometry &g, int grid) {
   L.total = off;
   const size_t phase_a = static_cast<size_t>(kRT + kCT) * (g.d + kPad) * 8;
   const size_t phase_b =
-      static_cast<size_t>(kWarps) * (static_cast<size_t>(g.Nb) * 4 + kCand * 8 + L.ntiles * 8 + 16);
+      static_cast<size_t>(kWarps) *
+      (static_cast<size_t>(g.Nb) * 4 + kCand * 8 + L.ntiles * 8 + 16 + kBins * 8 + kMaxWords * 4);
   L.smem = phase_a > phase_b ? phase_a : phase_b;
+  if (L.words > kMaxWords) L.smem = ~static_cast<size_t>(0) >> 1;  // reported as unsupported
   return L;
 }
 
