@@ -2,18 +2,19 @@
 // reduced attention over pooled blocks and the per-row CDF threshold; item 3:
 // union with the sliding-tile window; Sparse VideoGen2 section 2B: top-p).
 //
-// Three kernels:
-//   mask_select_kernel  persistent; one work item = 64 query blocks of one
-//                       (batch, head).  Phase A forms the 64 x Nb pooled
-//                       scores with fp64 tensor-core MMAs (m8n8k4) in column
-//                       tiles of 128, keeps each tile's row maxima in fp64 and
-//                       writes 2^(t - tile max) as fp32 to a CTA-private slab
-//                       that stays in L2.  Phase B, one warp per row, rescales
-//                       the slab to the row maximum, finds the CDF cut by
-//                       bisection on the fp32 bit pattern (mass tests in fp64,
-//                       candidates compacted once the range is narrow), breaks
-//                       ties by index, ORs in the STA window and writes a
-//                       kept-bit row and its count.
+// Four kernels:
+//   mask_scores_kernel  persistent; one work item = 64 query blocks of one
+//                       (batch, head).  Forms the 64 x Nb pooled scores with
+//                       fp64 tensor-core MMAs (m8n8k4) in column tiles of 128,
+//                       writes each tile's row maxima in fp64 and
+//                       2^(t - tile max) as fp32 to the workspace slab.
+//   mask_select_kernel  one warp per row: rescales the slab row to the row
+//                       maximum, finds the CDF cut (histogram of the top 8
+//                       octaves + exact fp64 check + warp sort of the cut
+//                       bin, or bisection on the fp32 bit pattern with fp64
+//                       mass tests), breaks ties by index, ORs in the STA
+//                       window and writes a kept-bit row and its count.  Small
+//                       SMEM per warp, so many rows are in flight per SM.
 //   scan_counts_kernel  exclusive scan of the counts into row_ptr (int64).
 //   expand_bits_kernel  kept bits -> ascending col_idx lists.
 //
@@ -37,7 +38,7 @@ constexpr int kPad = 4;       // fp64 padding per smem row (conflict-free fragme
 constexpr int kCand = 256;    // per-warp candidate list capacity
 constexpr int kBins = 64;     // 1/8-octave probability bins (8 octaves below the max)
 constexpr int kMaxWords = 256;  // kept-bit words per row held in SMEM (Nb <= 8192)
-constexpr int kMaxGrid = 160; // slabs in the workspace
+constexpr int kMaxGrid = 160; // persistent score CTAs
 
 struct MaskArgs {
   const double *qp, *kp;
@@ -46,8 +47,8 @@ struct MaskArgs {
   float thr;
   int use_sta, rt, rh, rw;
   double c;          // scale * log2(e)
-  float *slab;       // [grid][kRT][ld_slab]
-  double *tmax;      // [grid][kRT][ntiles]
+  float *slab;       // [BH*Nb][ld_slab]
+  double *tmax;      // [BH*Nb][ntiles]
   int ld_slab, ntiles;
   uint32_t *bits;    // [BH*Nb][words]
   int words;
@@ -390,7 +391,7 @@ __device__ void select_row(const MaskArgs &a, int64_t grow, int r, const float *
   __syncwarp();
 }
 
-__global__ void __launch_bounds__(kThreads, 1) mask_select_kernel(const MaskArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) mask_scores_kernel(const MaskArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   double *sQ = reinterpret_cast<double *>(smem_raw);
   const int ld = a.d + kPad;
@@ -401,13 +402,15 @@ __global__ void __launch_bounds__(kThreads, 1) mask_select_kernel(const MaskArgs
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tq = lane & 3;
   const int wm = warp >> 2, wn = warp & 3;
-  float *slab = a.slab + static_cast<int64_t>(blockIdx.x) * kRT * a.ld_slab;
-  double *tmax = a.tmax + static_cast<int64_t>(blockIdx.x) * kRT * a.ntiles;
   const int vec_per_row = a.d / 2;  // 16-byte chunks per fp64 row
 
   for (int64_t item = blockIdx.x; item < a.items; item += gridDim.x) {
     const int64_t bh = item / a.tiles_per_head;
     const int r0 = static_cast<int>(item % a.tiles_per_head) * kRT;
+    // rows of this item in the slab / tile-max arrays (rows past Nb belong
+    // to the next head or lie past the end: never written)
+    float *slab = a.slab + (bh * a.Nb + r0) * a.ld_slab;
+    double *tmax = a.tmax + (bh * a.Nb + r0) * a.ntiles;
     const double *qsrc = a.qp + (bh * a.Nb + r0) * a.d;
     const double *ksrc = a.kp + bh * a.Nb * a.d;
 
@@ -467,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_select_kernel(const MaskArgs
       if (tid < kRT) {
         const double m = fmax(fmax(sRed[tid][0], sRed[tid][1]), fmax(sRed[tid][2], sRed[tid][3]));
         sTileMax[tid] = m;
-        tmax[tid * a.ntiles + ct] = m;
+        if (r0 + tid < a.Nb) tmax[tid * a.ntiles + ct] = m;
       }
       __syncthreads();
 #pragma unroll
@@ -477,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1) mask_select_kernel(const MaskArgs
 #pragma unroll
         for (int ni = 0; ni < 4; ++ni) {
           const int col = c0 + wn * 32 + ni * 8 + 2 * tq;
-          if (col < a.Nb) {
+          if (col < a.Nb && r0 + row < a.Nb) {
             float2 e;
             e.x = exp2_split(acc[mi][ni][0] - m);
             e.y = exp2_split(acc[mi][ni][1] - m);
@@ -487,28 +490,29 @@ __global__ void __launch_bounds__(kThreads, 1) mask_select_kernel(const MaskArgs
       }
       __syncthreads();  // sK is overwritten by the next tile
     }
-    __threadfence_block();
-    __syncthreads();
+  }
+}
 
-    // ---- phase B: one warp per row
-    unsigned char *wbase = smem_raw + warp * (static_cast<size_t>(a.Nb) * 4 + kCand * 8 +
-                                              static_cast<size_t>(a.ntiles) * 8 + 16 + kBins * 8 +
-                                              kMaxWords * 4);
-    float *ebuf = reinterpret_cast<float *>(wbase);
-    uint32_t *cand_key = reinterpret_cast<uint32_t *>(ebuf + a.Nb);
-    int32_t *cand_idx = reinterpret_cast<int32_t *>(cand_key + kCand);
-    double *tscale = reinterpret_cast<double *>(
-        (reinterpret_cast<uintptr_t>(cand_idx + kCand) + 15) & ~static_cast<uintptr_t>(15));
-    int *hcnt = reinterpret_cast<int *>(tscale + a.ntiles);
-    float *hmass = reinterpret_cast<float *>(hcnt + kBins);
-    uint32_t *wbits = reinterpret_cast<uint32_t *>(hmass + kBins);
-    for (int row = warp; row < kRT; row += kWarps) {
-      const int r = r0 + row;
-      if (r >= a.Nb) break;
-      select_row(a, bh * a.Nb + r, r, slab + row * a.ld_slab, tmax + row * a.ntiles, ebuf,
-                 cand_key, cand_idx, tscale, hcnt, hmass, wbits);
-    }
-    __syncthreads();  // smem and slab are reused by the next item
+// One warp per row of the mask: selection and kept bits.
+__global__ void __launch_bounds__(kThreads) mask_select_kernel(const MaskArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int warp = threadIdx.x >> 5;
+  unsigned char *wbase = smem_raw + warp * (static_cast<size_t>(a.Nb) * 4 + kCand * 8 +
+                                            static_cast<size_t>(a.ntiles) * 8 + 16 + kBins * 8 +
+                                            kMaxWords * 4);
+  float *ebuf = reinterpret_cast<float *>(wbase);
+  uint32_t *cand_key = reinterpret_cast<uint32_t *>(ebuf + a.Nb);
+  int32_t *cand_idx = reinterpret_cast<int32_t *>(cand_key + kCand);
+  double *tscale = reinterpret_cast<double *>(
+      (reinterpret_cast<uintptr_t>(cand_idx + kCand) + 15) & ~static_cast<uintptr_t>(15));
+  int *hcnt = reinterpret_cast<int *>(tscale + a.ntiles);
+  float *hmass = reinterpret_cast<float *>(hcnt + kBins);
+  uint32_t *wbits = reinterpret_cast<uint32_t *>(hmass + kBins);
+  const int64_t rows = a.BH * a.Nb;
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * kWarps + warp; g < rows;
+       g += static_cast<int64_t>(gridDim.x) * kWarps) {
+    select_row(a, g, static_cast<int>(g % a.Nb), a.slab + g * a.ld_slab, a.tmax + g * a.ntiles,
+               ebuf, cand_key, cand_idx, tscale, hcnt, hmass, wbits);
   }
 }
 
@@ -572,7 +576,7 @@ __global__ void __launch_bounds__(256) expand_bits_kernel(const uint32_t *__rest
 struct MaskLayout {
   int ld_slab, ntiles, words, grid;
   size_t slab_off, tmax_off, bits_off, counts_off, total;
-  size_t smem;
+  size_t smem, smem_a, smem_b;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -585,19 +589,19 @@ MaskLayout mask_layout(const Geometry &g, int grid) {
   L.grid = grid;
   size_t off = 0;
   L.slab_off = off;
-  off = align256(off + static_cast<size_t>(kMaxGrid) * kRT * L.ld_slab * 4);
+  off = align256(off + static_cast<size_t>(g.BH * g.Nb) * L.ld_slab * 4);
   L.tmax_off = off;
-  off = align256(off + static_cast<size_t>(kMaxGrid) * kRT * L.ntiles * 8);
+  off = align256(off + static_cast<size_t>(g.BH * g.Nb) * L.ntiles * 8);
   L.bits_off = off;
   off = align256(off + static_cast<size_t>(g.BH * g.Nb) * L.words * 4);
   L.counts_off = off;
   off = align256(off + static_cast<size_t>(g.BH * g.Nb) * 4);
   L.total = off;
-  const size_t phase_a = static_cast<size_t>(kRT + kCT) * (g.d + kPad) * 8;
-  const size_t phase_b =
-      static_cast<size_t>(kWarps) *
-      (static_cast<size_t>(g.Nb) * 4 + kCand * 8 + L.ntiles * 8 + 16 + kBins * 8 + kMaxWords * 4);
-  L.smem = phase_a > phase_b ? phase_a : phase_b;
+  L.smem_a = static_cast<size_t>(kRT + kCT) * (g.d + kPad) * 8;
+  L.smem_b = static_cast<size_t>(kWarps) *
+             (static_cast<size_t>(g.Nb) * 4 + kCand * 8 + L.ntiles * 8 + 16 + kBins * 8 +
+              kMaxWords * 4);
+  L.smem = L.smem_a > L.smem_b ? L.smem_a : L.smem_b;
   if (L.words > kMaxWords) L.smem = ~static_cast<size_t>(0) >> 1;  // reported as unsupported
   return L;
 }
@@ -635,11 +639,18 @@ cudaError_t launch_block_mask(const double *qp, const double *kp, const Geometry
   a.words = L.words;
   a.counts = kept_count ? kept_count : reinterpret_cast<int32_t *>(w + L.counts_off);
   a.items = items; a.tiles_per_head = tiles_per_head;
-  cudaError_t e = cudaFuncSetAttribute(mask_select_kernel,
+  cudaError_t e = cudaFuncSetAttribute(mask_scores_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(L.smem));
+                                       static_cast<int>(L.smem_a));
   if (e != cudaSuccess) return e;
-  mask_select_kernel<<<grid, kThreads, L.smem, st>>>(a);
+  mask_scores_kernel<<<grid, kThreads, L.smem_a, st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(mask_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(L.smem_b))) != cudaSuccess)
+    return e;
+  const int64_t sel_blocks = (rows + kWarps - 1) / kWarps;
+  const int sel_grid = static_cast<int>(sel_blocks < 64LL * num_sms() ? sel_blocks : 64LL * num_sms());
+  mask_select_kernel<<<sel_grid, kThreads, L.smem_b, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   scan_counts_kernel<<<1, 1024, 0, st>>>(a.counts, rows, row_ptr);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
