@@ -8,6 +8,7 @@
 // whose kept lists overlap most (time pairing).  The item walks the merged,
 // ascending union of both lists two key blocks (128 keys) per step n:
 //   S_n = Q K_n^T  tcgen05.mma M=128, N=64*nb, K=d  (SMEM x SMEM -> TMEM S[n%3])
+// (N = 128 whenever the step has two blocks: N = 64 MMAs run at ~2/3 rate)
 //   P_n = online softmax of S_n, per row only over the blocks its own query
 //         block keeps, written as packed bf16 over the first 64 columns of
 //         the same TMEM buffer
@@ -19,8 +20,12 @@
 //   warp 0      producer: takes items from an atomic counter over a
 //               longest-first work list, merges the two CSR lists, publishes
 //               one step record per step (8-deep ring) and issues the TMA
-//               loads (128B-swizzled boxes) of Q per item and of K per step
-//               into a 3-deep ring;
+//               loads of Q per item and of K per step into a 3-deep ring.
+//               Every 64-row block is one 4-D box (64 elements x 8 rows x
+//               d/64 halves x 8 row groups), stored 128B-swizzled as
+//               [row group][d-half][8 rows][128 B]: the rows of two blocks
+//               then sit at one uniform group stride of 16*d bytes (the SBO)
+//               and the d-halves 1 KiB apart;
 //   warp 11     V producer: follows the step records and loads V per step
 //               into its own 3-deep ring;
 //   warp 1      allocates 512 TMEM columns; one lane issues the S MMAs;
@@ -64,7 +69,8 @@ struct StepMeta {
 template <int D>
 struct Smem {
   static constexpr int kQBytes = 128 * D * 2;             // two query blocks
-  static constexpr int kBlockBytes = 64 * D * 2;          // one key block: [d-half][64 rows][128 B]
+  static constexpr int kBlockBytes = 64 * D * 2;          // one 64-row block
+  static constexpr int kGroupBytes = 8 * D * 2;            // 8 rows, all d-halves
   static constexpr int kKVBytes = 2 * kBlockBytes;         // K (or V) of two key blocks
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kQBytes;
@@ -205,9 +211,9 @@ __global__ void __maxnreg__(168)
         const uint32_t kf = k_full(s3);
         mbar_arrive_expect_tx(kf, static_cast<uint32_t>(nb * L::kBlockBytes));
         const uint32_t kbase = sbase + L::kKOff + s3 * L::kKVBytes;
-        const int head_row = static_cast<int>(static_cast<int64_t>(r.bh) * a.N);
-        if (nb > 0) tma_load_3d(kbase, &tk, kf, 0, head_row + r.blk0 * 64, 0);
-        if (nb > 1) tma_load_3d(kbase + L::kBlockBytes, &tk, kf, 0, head_row + r.blk1 * 64, 0);
+        const int head_grp = static_cast<int>(static_cast<int64_t>(r.bh) * a.N / 8);
+        if (nb > 0) tma_load_4d(kbase, &tk, kf, 0, 0, 0, head_grp + r.blk0 * 8);
+        if (nb > 1) tma_load_4d(kbase + L::kBlockBytes, &tk, kf, 0, 0, 0, head_grp + r.blk1 * 8);
       }
       __syncwarp();
       ++m;
@@ -237,12 +243,10 @@ __global__ void __maxnreg__(168)
       if (lane == 0) {
         const int nq = r1 >= 0 ? 2 : 1;
         mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(nq * 64 * D * 2));
-        for (int j = 0; j < nq; ++j) {
-          const int row = static_cast<int>(static_cast<int64_t>(bh) * a.N) + (j ? r1 : r0) * 64;
-          for (int dh = 0; dh < D / 64; ++dh)
-            tma_load_2d(sbase + L::kQOff + dh * (128 * 128) + j * (64 * 128), &tq, q_full,
-                        dh * 64, row);
-        }
+        const int head_grp = static_cast<int>(static_cast<int64_t>(bh) * a.N / 8);
+        for (int j = 0; j < nq; ++j)
+          tma_load_4d(sbase + L::kQOff + j * L::kBlockBytes, &tq, q_full, 0, 0, 0,
+                      head_grp + (j ? r1 : r0) * 8);
       }
       // merge the two ascending lists, two union entries per step
       const int64_t g0 = static_cast<int64_t>(bh) * a.Nb + r0;
@@ -317,11 +321,12 @@ __global__ void __maxnreg__(168)
     // ------------------------------------------------------------ S issuer
     uint32_t q_phase = 0;
     constexpr uint32_t kIdescS1 = idesc_bf16(128, 64, false, false);
+    constexpr uint32_t kIdescS2 = idesc_bf16(128, 128, false, false);
     constexpr uint32_t kStageUnits = L::kKVBytes >> 4;   // one stage in 16-byte units
     // Descriptors are built once; per MMA only the 14-bit start-address field
     // (16-byte units, low word) moves.
-    const uint64_t q_desc = smem_desc(sbase + L::kQOff, 16, 1024);
-    const uint64_t k_desc0 = smem_desc(sbase + L::kKOff, 16, 1024);
+    const uint64_t q_desc = smem_desc(sbase + L::kQOff, 16, L::kGroupBytes);
+    const uint64_t k_desc0 = smem_desc(sbase + L::kKOff, 16, L::kGroupBytes);
     for (int n = 0;; ++n) {
       const int b = n % kRing;
       if (!mbar_wait(k_full(b), (n / kRing) & 1, a.err, kErrWaitTma)) break;
@@ -338,20 +343,16 @@ __global__ void __maxnreg__(168)
       }
       tc_fence_after();
       if (lane == 0) {
-        // one N=64 MMA chain per key block: S columns [64j, 64j+64)
-        const uint64_t kd = k_desc0 + static_cast<uint32_t>(b) * kStageUnits;
-        const uint32_t dcol = tmem + static_cast<uint32_t>(b) * 128u;
+        if (r.nb > 0) {
+          // one chain, N = 64*nb: both blocks' rows at the uniform group stride
+          const uint64_t kd = k_desc0 + static_cast<uint32_t>(b) * kStageUnits;
+          const uint32_t dcol = tmem + static_cast<uint32_t>(b) * 128u;
+          const uint32_t idesc_s = r.nb > 1 ? kIdescS2 : kIdescS1;
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          if (j < r.nb) {
-#pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-              // k-th 16-column slice: 32 B inside the 128 B swizzle row; Q
-              // d-halves 16 KiB apart, K d-halves 8 KiB apart inside a block
-              const uint32_t qoff = (k >> 2) * 1024 + (k & 3) * 2;
-              const uint32_t koff = j * (L::kBlockBytes >> 4) + (k >> 2) * 512 + (k & 3) * 2;
-              mma_bf16_ss(dcol + 64 * j, q_desc + qoff, kd + koff, kIdescS1, k > 0);
-            }
+          for (int k = 0; k < D / 16; ++k) {
+            // k-th 16-column slice: 32 B inside the 128 B swizzle row, d-halves 1 KiB apart
+            const uint32_t off = (k >> 2) * 64 + (k & 3) * 2;
+            mma_bf16_ss(dcol, q_desc + off, kd + off, idesc_s, k > 0);
           }
         }
         mma_commit(s_full(b));          // also frees K stage b
@@ -365,9 +366,10 @@ __global__ void __maxnreg__(168)
     bool first_item = true;
     constexpr uint32_t kIdescO = idesc_bf16(128, D, false, true);
     constexpr uint32_t kStageUnits = L::kKVBytes >> 4;
-    // V is an MN-major operand: 8-key groups 1 KiB apart (SBO), d-halves of a
-    // block 8 KiB apart (LBO), blocks kBlockBytes apart
-    const uint64_t v_desc0 = smem_desc(sbase + L::kVOff, 64 * 128, 1024);
+    // V is an MN-major operand: 8-key groups kGroupBytes apart (SBO, across
+    // both blocks), d-halves 1 KiB apart (LBO)
+    const uint64_t v_desc0 = smem_desc(sbase + L::kVOff, 1024, L::kGroupBytes);
+    constexpr uint32_t kKStep = (2 * L::kGroupBytes) >> 4;   // 16 keys
     for (int n = 0;; ++n) {
       const int b = n % kRing;
       // the step record tells an end record apart (no P will come); slot n%8
@@ -395,12 +397,11 @@ __global__ void __maxnreg__(168)
           // 16 keys per MMA: 8 TMEM columns of P, 2 KiB of V
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_bf16_ts(tmem + kColO, pcol + k * 8, vd + k * 128, kIdescO, acc0 || k > 0);
+            mma_bf16_ts(tmem + kColO, pcol + k * 8, vd + k * kKStep, kIdescO, acc0 || k > 0);
           if (r.nb > 1) {
-            const uint64_t vd1 = vd + (L::kBlockBytes >> 4);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              mma_bf16_ts(tmem + kColO, pcol + 32 + k * 8, vd1 + k * 128, kIdescO, true);
+            for (int k = 4; k < 8; ++k)
+              mma_bf16_ts(tmem + kColO, pcol + k * 8, vd + k * kKStep, kIdescO, true);
           }
         }
         mma_commit(pv_buf(b));          // also frees V stage b
@@ -425,9 +426,9 @@ __global__ void __maxnreg__(168)
         const uint32_t vf = v_full(b);
         mbar_arrive_expect_tx(vf, static_cast<uint32_t>(nb * L::kBlockBytes));
         const uint32_t vbase = sbase + L::kVOff + b * L::kKVBytes;
-        const int head_row = static_cast<int>(static_cast<int64_t>(r.bh) * a.N);
-        if (nb > 0) tma_load_3d(vbase, &tv, vf, 0, head_row + r.blk0 * 64, 0);
-        if (nb > 1) tma_load_3d(vbase + L::kBlockBytes, &tv, vf, 0, head_row + r.blk1 * 64, 0);
+        const int head_grp = static_cast<int>(static_cast<int64_t>(r.bh) * a.N / 8);
+        if (nb > 0) tma_load_4d(vbase, &tv, vf, 0, 0, 0, head_grp + r.blk0 * 8);
+        if (nb > 1) tma_load_4d(vbase + L::kBlockBytes, &tv, vf, 0, 0, 0, head_grp + r.blk1 * 8);
       }
       __syncwarp();
     }
@@ -663,29 +664,20 @@ EncodeFn encode_fn() {
   return fn;
 }
 
-// [rows, d] bf16 viewed as (64 elements, rows, d/64 halves): one box is a
-// whole 64-row block, its d-halves stacked (block-major SMEM layout).
-bool make_map3(CUtensorMap *m, const void *base, int64_t rows, int d) {
+// [rows, d] bf16 viewed as (64 elements, 8 rows, d/64 halves, rows/8 groups):
+// one box {64, 8, d/64, 8} is a whole 64-row block stored as
+// [row group][d-half][8 rows][128 B], i.e. 1 KiB swizzle atoms with the
+// d-halves of a row group side by side.
+bool make_map4(CUtensorMap *m, const void *base, int64_t rows, int d) {
   EncodeFn enc = encode_fn();
   if (!enc) return false;
-  const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(d / 64)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, 128};
-  const cuuint32_t box[3] = {64, 64, static_cast<cuuint32_t>(d / 64)};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
-}
-
-bool make_map(CUtensorMap *m, const void *base, int64_t rows, int d) {
-  EncodeFn enc = encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
-  const cuuint32_t box[2] = {64, 64};
-  const cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+  const cuuint64_t dims[4] = {64, 8, static_cast<cuuint64_t>(d / 64),
+                              static_cast<cuuint64_t>(rows / 8)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, 128,
+                                 static_cast<cuuint64_t>(d) * 2 * 8};
+  const cuuint32_t box[4] = {64, 8, static_cast<cuuint32_t>(d / 64), 8};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
@@ -724,8 +716,8 @@ cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
   }
   CUtensorMap mq, mk, mv;
   const int64_t rows = g.BH * g.N;
-  if (!make_map(&mq, qf, rows, g.d) || !make_map3(&mk, kf, rows, g.d) ||
-      !make_map3(&mv, vf, rows, g.d)) {
+  if (!make_map4(&mq, qf, rows, g.d) || !make_map4(&mk, kf, rows, g.d) ||
+      !make_map4(&mv, vf, rows, g.d)) {
     *why = "sparse attention: cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
   }

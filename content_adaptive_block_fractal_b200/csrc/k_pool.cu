@@ -4,10 +4,11 @@
 // One warp reduces one block of 64 consecutive flattened tokens.  A token row
 // of d bf16 is read by d/8 lanes with 16-byte loads (a warp covers 32/(d/8)
 // rows per step), so every load instruction moves 512 contiguous bytes.  Each
-// bf16 is widened to fp64 with integer ops (exact) and summed in fp64; the sum
-// of 64 bf16 values is exact in fp64 and the final /64 is exact, so the
-// output is the exact block mean.  HBM-bound: reads 2*N*d*2 bytes per
-// (batch, head), writes 2*Nb*d*8.
+// bf16 is widened to fp64 with integer ops (exact) and summed in fp64.  With
+// 8 significant bits per bf16, a sum of 64 of them fits fp64's 53 bits when
+// the nonzero magnitudes lie within 2^39 of each other, so the sum (in any
+// order) and the final /64 are exact and the output is the exact block mean.
+// HBM-bound: reads 2*N*d*2 bytes per (batch, head), writes 2*Nb*d*8.
 #include "vsa_device.cuh"
 #include "vsa_internal.h"
 

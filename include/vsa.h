@@ -82,9 +82,13 @@ vsa_status vsa_fractal_unflatten(const void *y, void *x, vsa_shape s, void *stre
 /* 2. Block mean pooling (NABLA, Methodology item 2, "downsampling").
  * qp[b,h,r,:] = (1/64) * sum_{i<64} qf[b,h,64r+i,:], same for k.
  * qf, kf : device bf16 [B,heads,N,d] in flattened order.
- * qp, kp : device fp64 [B,heads,Nb,d].  The sum of 64 bf16 values is exact in
- *          fp64 and the division by 64 is exact, so each pooled value is the
- *          exact block mean. */
+ * qp, kp : device fp64 [B,heads,Nb,d].  A bf16 carries 8 significant bits,
+ *          so the sum of 64 of them needs at most 14 + (exponent spread) bits:
+ *          it is exact in fp64 whenever the block's nonzero magnitudes lie
+ *          within a factor 2^39 of each other (data of one scale always do),
+ *          and the division by 64 is exact, so each pooled value is then the
+ *          exact block mean, independent of summation order.  Outside that
+ *          range the result is within a few fp64 roundings of it. */
 vsa_status vsa_pool_qk(const void *qf, const void *kf, double *qp, double *kp,
                        vsa_shape s, void *stream);
 
