@@ -50,12 +50,13 @@ def parse_args():
 
 
 def measured_peaks():
+    """(bf16 burst TFLOP/s, bf16 sustained TFLOP/s, HBM GB/s, source)."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
-        return p["bf16_tflops"], p["hbm_gbs"], "measured"
+        return p["bf16_tflops"], p["bf16_tflops_sustained"], p["hbm_gbs"], "measured"
     except Exception:
-        return 1590.0, 6650.0, "fallback"
+        return 1590.0, 1400.0, 6650.0, "fallback"
 
 
 def profile_traffic(kernel_src: str):
@@ -223,7 +224,10 @@ def run_gpu(args, rank, world, local_rank):
         if e2e:
             e2e["value"] = float(t[1]) / world
     value = ms / world
-    peak_tf, peak_gbs, peak_src = measured_peaks()
+    # The attention kernel runs back to back for the whole timed loop and
+    # holds the GPU at its power cap, so the sustained GEMM figure (a
+    # seconds-long cuBLAS loop under the same cap) is its denominator.
+    burst_tf, peak_tf, peak_gbs, peak_src = measured_peaks()
     attn_ms = parts[3]
     achieved_tf = kept_flop / (attn_ms * 1e-3) / 1e12
     traffic = profile_traffic(os.path.join(ROOT, "content_adaptive_block_fractal_b200", "csrc", "k_attn.cu"))
@@ -243,7 +247,8 @@ def run_gpu(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "kernel": "sparse_attn_kernel<128>",
                      "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": achieved_tf / peak_tf, "traffic": traffic,
-                     "peak_source": f"{peak_src} bf16 (burst)",
+                     "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long loop)",
+                     "frac_of_burst": achieved_tf / burst_tf,
                      "flop_per_kept_tile": flop_per_tile},
         "mask_path_gbs": (shape.B * shape.heads * shape.N * shape.d * 2 * 2
                           + 2 * rows * shape.d * 8) / ((parts[1] + parts[2]) * 1e-3) / 1e9,

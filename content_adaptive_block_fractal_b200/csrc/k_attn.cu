@@ -115,6 +115,37 @@ __device__ __forceinline__ void decode_item(int item, const AttnArgs &a, int &bh
   r1 = (2 * t2 + 1 < a.T) ? r0 + a.HW : -1;
 }
 
+// One 32-column chunk Q of the softmax's second pass: starts the load of
+// chunk Q+1 into `nxt`, exponentiates `cur` (already loaded) against the
+// reference, adds to the row sums and stores P as 16 packed bf16x2 columns
+// over S columns [16Q, 16Q+16) (scores already read), then waits for `nxt`.
+// Chunks 0-1 are key block 0 (valid when v0), chunks 2-3 key block 1.
+template <int Q>
+__device__ __forceinline__ void softmax_chunk(uint32_t (&cur)[32], uint32_t (&nxt)[32], int nq,
+                                              bool v0, bool v1, uint32_t s_addr, float2 c2,
+                                              float2 nm2, float2 (&r4)[4]) {
+  if (Q >= nq) return;
+  const bool vq = Q < 2 ? v0 : v1;
+  const bool vn = Q + 1 < nq && (Q + 1 < 2 ? v0 : v1);
+  if (vn) tmem_ld32_nowait(s_addr + 32 * (Q + 1), nxt);
+  uint32_t pk[16];
+  if (vq) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float2 t =
+          ffma2(make_float2(__uint_as_float(cur[2 * j]), __uint_as_float(cur[2 * j + 1])), c2, nm2);
+      const float2 p = make_float2(ex2(t.x), ex2(t.y));
+      r4[j & 3] = fadd2(r4[j & 3], p);
+      pk[j] = pack_bf16x2(p.x, p.y);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) pk[j] = 0u;
+  }
+  tmem_st16u(s_addr + 16 * Q, pk);
+  if (vn) tmem_wait_ld_regs(nxt);
+}
+
 template <int D>
 __global__ void __maxnreg__(168)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tq,
@@ -163,14 +194,14 @@ __global__ void __maxnreg__(168)
     }
     for (int s = 0; s < kMetaRing; ++s) {
       mbar_init(meta_full(s), 1);
-      mbar_init(meta_empty(s), 128);
+      mbar_init(meta_empty(s), 4);        // one arrival per softmax warp
     }
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     for (int s = 0; s < 4; ++s) mbar_init(p_full(s), 128);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(m_full(s), 128);
-      mbar_init(l_full(s), 128);
+      mbar_init(m_full(s), 4);            // one arrival per softmax warp
+      mbar_init(l_full(s), 4);
     }
     mbar_init(o_full, 1);
     mbar_init(o_empty, 128);
@@ -196,8 +227,8 @@ __global__ void __maxnreg__(168)
     uint32_t q_phase = 0;
     bool ok = true;
     int nitems = 0;
-    // Publishes step record r as step m and loads its K blocks (one 3-D box
-    // per block: 64 rows x all d-halves, block-major in the stage).
+    // Publishes step record r as step m and loads its K blocks (one 4-D box
+    // per block, row-group-major in the stage).
     auto emit = [&](const StepMeta &r) -> bool {
       const int s3 = m % kRing, sm = m % kMetaRing;
       if (!mbar_wait(meta_empty(sm), ((m / kMetaRing) & 1) ^ 1, a.err, kErrWaitSoftmax)) return false;
@@ -439,11 +470,18 @@ __global__ void __maxnreg__(168)
     const int row = quarter * 32 + lane;       // query row within the tile
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const uint32_t sel = row >= 64 ? 1u : 0u;
+    const float2 c2 = make_float2(a.c, a.c);
+    // This group's partial row sum over its own steps of the current item, in
+    // the scale of the reference it used last (m_own).  The two partial sums
+    // meet only at the item's last step.
+    float l_own = 0.0f, m_own = -INFINITY;
+    int seq_own = -1;
     for (int n = grp;; n += 2) {
       const int sm = n % kMetaRing;
       if (!mbar_wait(meta_full(sm), (n / kMetaRing) & 1, a.err, kErrWaitTma)) break;
       const StepMeta m = meta[sm];
-      mbar_arrive(meta_empty(sm));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(meta_empty(sm));
       if (m.nb < 0) break;
       const bool first = m.first_last & 1, last = m.first_last & 2;
       const int sb = n % kRing;
@@ -451,26 +489,23 @@ __global__ void __maxnreg__(168)
       if (!mbar_wait(s_full(sb), (n / kRing) & 1, a.err, kErrWaitMma)) break;
       tc_fence_after();
       // warps hold rows of one query block, so v0 / v1 are warp-uniform
-      const bool v0 = (m.flags >> sel) & 1u;
+      const bool v0 = m.nb > 0 && ((m.flags >> sel) & 1u);
       const bool v1 = m.nb > 1 && ((m.flags >> (2 + sel)) & 1u);
       float mx = -INFINITY;
-      {
+      if (v0 || v1) {
         // pass 1: row max over the valid halves, 64 scores live at a time
-        float m8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m8[i] = -INFINITY;
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           if (h ? v1 : v0) {
             float x[64];
             tmem_ld64(s_addr + 64 * h, x);
 #pragma unroll
-            for (int j = 0; j < 64; ++j) m8[j & 7] = fmaxf(m8[j & 7], x[j]);
+            for (int j = 0; j < 64; j += 2)
+              m4[(j >> 1) & 3] = fmax3(m4[(j >> 1) & 3], x[j], x[j + 1]);
           }
         }
-        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-        mx *= a.c;
+        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * a.c;
       }
       // running max of the previous step (the other group); every step waits
       // for it so that the hand-off barriers stay in lock step
@@ -478,6 +513,15 @@ __global__ void __maxnreg__(168)
       if (n > 0) {
         if (!mbar_wait(m_full((n - 1) & 1), ((n - 1) >> 1) & 1, a.err, kErrWaitSoftmax)) break;
         if (!first) m_prev = m_sh[((n - 1) & 1) * 128 + row];
+      }
+      // At the item's last step, take the other group's partial sum (posted
+      // at step n-1, in the scale m_prev) before this step's max is posted:
+      // the other group writes that slot again only at step n+1, after it has
+      // seen this step's max, so the slot cannot be overwritten under us.
+      float l_other = 0.0f;
+      if (last && !first) {
+        if (!mbar_wait(l_full((n - 1) & 1), ((n - 1) >> 1) & 1, a.err, kErrWaitSoftmax)) break;
+        l_other = l_sh[((n - 1) & 1) * 128 + row];
       }
       // lazy rescale: move the reference max only when it grows by > 8 (2^8)
       float m_run = m_prev, alpha = 1.0f;
@@ -490,43 +534,41 @@ __global__ void __maxnreg__(168)
         m_run = mx;
       }
       m_sh[(n & 1) * 128 + row] = m_run;
-      mbar_arrive(m_full(n & 1));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(m_full(n & 1));
       const float mref = m_run == -INFINITY ? 0.0f : m_run;
-      float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // partial row sums
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (h < m.nb) {
-          // pass 2, one 64-key half at a time; P of half h overwrites S
-          // columns [32h, 32h+32), which hold scores already read
-          const bool valid = h ? v1 : v0;
-          uint32_t pk[32];
-          if (valid) {
-            float x[64];
-            tmem_ld64(s_addr + 64 * h, x);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float p0 = ex2(fmaf(x[2 * j], a.c, -mref));
-              const float p1 = ex2(fmaf(x[2 * j + 1], a.c, -mref));
-              r8[j & 7] += p0 + p1;
-              pk[j] = pack_bf16x2(p0, p1);
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) pk[j] = 0u;
-          }
-          tmem_st32u(s_addr + 32 * h, pk);
+      const float2 nm2 = make_float2(-mref, -mref);
+      // pass 2 over 32-column chunks: chunk q+1 is loaded while chunk q is
+      // exponentiated; P of chunk q (16 packed columns) goes to S columns
+      // [16q, 16q+16), which hold scores already read
+      float2 r4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                      make_float2(0.f, 0.f)};
+      {
+        const int nq = 2 * (m.nb > 0 ? m.nb : 0);
+        uint32_t xa[32], xb[32];
+        if (nq > 0 && v0) {
+          tmem_ld32_nowait(s_addr, xa);
+          tmem_wait_ld_regs(xa);
         }
+        softmax_chunk<0>(xa, xb, nq, v0, v1, s_addr, c2, nm2, r4);
+        softmax_chunk<1>(xb, xa, nq, v0, v1, s_addr, c2, nm2, r4);
+        softmax_chunk<2>(xa, xb, nq, v0, v1, s_addr, c2, nm2, r4);
+        softmax_chunk<3>(xb, xa, nq, v0, v1, s_addr, c2, nm2, r4);
       }
-      const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
-      // running sum: the previous step's value (other group), rescaled
-      float l_prev = 0.0f;
-      if (n > 0) {
-        if (!mbar_wait(l_full((n - 1) & 1), ((n - 1) >> 1) & 1, a.err, kErrWaitSoftmax)) break;
-        if (!first) l_prev = l_sh[((n - 1) & 1) * 128 + row];
+      const float rs = ((r4[0].x + r4[0].y) + (r4[1].x + r4[1].y)) +
+                       ((r4[2].x + r4[2].y) + (r4[3].x + r4[3].y));
+      // this group's partial sum, moved to the reference m_run
+      if (m.seq != seq_own) {
+        l_own = 0.0f;
+        seq_own = m.seq;
+      } else if (l_own > 0.0f && m_run != m_own) {
+        l_own *= ex2(m_own - m_run);
       }
-      const float l_run = l_prev * alpha + rs;
-      l_sh[(n & 1) * 128 + row] = l_run;
-      mbar_arrive(l_full(n & 1));
+      l_own += rs;
+      m_own = m_run;
+      l_sh[(n & 1) * 128 + row] = l_own;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(l_full(n & 1));
       if (__any_sync(0xFFFFFFFFu, resc)) {
         // O must hold PV_{n-1} before it is rescaled.  S_n was issued only
         // after PV_{n-3} completed, so buffer (n-1)%3 has finished every PV
@@ -546,6 +588,10 @@ __global__ void __maxnreg__(168)
       tc_fence_before();
       mbar_arrive(p_full(n & 3));
       if (last) {
+        // total row sum in the final reference m_run; the other group's part
+        // is in the scale of step n-1's reference m_prev <= m_run
+        float l_run = l_own;
+        if (l_other > 0.0f) l_run += l_other * ex2(m_prev - m_run);
         if (!mbar_wait(o_full, static_cast<uint32_t>(m.seq) & 1u, a.err, kErrWaitMma)) break;
         tc_fence_after();
         const int rblk = sel ? m.r1 : m.r0;
