@@ -35,6 +35,9 @@ METRIC = "ms/attention layer and kept-tile TFLOP/s at Wan-14B 720p shape, thr=0.
 UNIT = "ms/layer"
 L2_FLUSH_BYTES = 256 << 20
 PROFILE = os.path.join(ROOT, "profiles", "sparse_attn_fwd_wan14b.md")
+# files whose contents make up the attention kernel (hashed against PROFILE)
+ATTN_SOURCES = [os.path.join(ROOT, "content_adaptive_block_fractal_b200", "csrc", f)
+                for f in ("k_attn.cu", "vsa_device.cuh")]
 
 
 def parse_args():
@@ -59,9 +62,17 @@ def measured_peaks():
         return 1590.0, 1400.0, 6650.0, "fallback"
 
 
-def profile_traffic(kernel_src: str):
+def kernel_source_hash(paths) -> str:
+    h = hashlib.sha256()
+    for p in paths:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profile_traffic(kernel_srcs):
     """DRAM bytes per attention launch from the committed ncu summary, if it was
-    taken on the current kernel source (same hash); else None."""
+    taken on the current kernel source (same hash of the kernel's files); else None."""
     try:
         text = open(PROFILE).read()
     except OSError:
@@ -70,7 +81,7 @@ def profile_traffic(kernel_src: str):
     b = re.search(r"dram_bytes_per_launch_full:\s*([0-9.eE+]+)", text)
     if not h or not b:
         return None
-    cur = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
+    cur = kernel_source_hash(kernel_srcs)
     return float(b.group(1)) if cur.startswith(h.group(1)) else None
 
 
@@ -141,15 +152,15 @@ def run_gpu(args, rank, world, local_rank):
     o_raster = torch.empty_like(qd)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=qd.device)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
-    launches_per_step = 3 + 1 + 3 + 2 + 1   # flatten x3, pool, mask x3, plan+attn, unflatten
+    # flatten+pool of Q,K; flatten of V; mask (scores, select, scan, expand);
+    # plan + attention; unflatten of O
+    launches_per_step = 1 + 1 + 4 + 2 + 1
 
     def step(record=False):
         if record: ev[0].record(stream)
-        vsa.fractal_flatten(qd, shape, out=qf)
-        vsa.fractal_flatten(kd, shape, out=kf)
-        vsa.fractal_flatten(vd, shape, out=vf)
+        vsa.flatten_pool_qk(qd, kd, shape, out=(qf, kf, layer.qp, layer.kp))
         if record: ev[1].record(stream)
-        vsa.pool_qk(qf, kf, shape, out=(layer.qp, layer.kp))
+        vsa.fractal_flatten(vd, shape, out=vf)
         if record: ev[2].record(stream)
         vsa.block_mask(layer.qp, layer.kp, shape, params, out=layer.csr, workspace=layer.ws_mask)
         if record: ev[3].record(stream)
@@ -166,6 +177,7 @@ def run_gpu(args, rank, world, local_rank):
     rows = shape.B * shape.heads * shape.Nb
     kept_frac = kept / (rows * shape.Nb)
     flop_per_tile = 4 * 64 * 64 * shape.d
+    tensor_bytes = shape.B * shape.heads * shape.N * shape.d * 2   # one bf16 [B,h,N,d]
     kept_flop = kept * flop_per_tile
 
     if world > 1:
@@ -230,7 +242,7 @@ def run_gpu(args, rank, world, local_rank):
     burst_tf, peak_tf, peak_gbs, peak_src = measured_peaks()
     attn_ms = parts[3]
     achieved_tf = kept_flop / (attn_ms * 1e-3) / 1e12
-    traffic = profile_traffic(os.path.join(ROOT, "content_adaptive_block_fractal_b200", "csrc", "k_attn.cu"))
+    traffic = profile_traffic(ATTN_SOURCES)
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False, "scaling": "weak",
@@ -242,7 +254,7 @@ def run_gpu(args, rank, world, local_rank):
         "kept_tile_tflops_layer": kept_flop / (ms * 1e-3) / 1e12,
         "kept_fraction": kept_frac,
         "kept_tiles": kept,
-        "breakdown_ms": {"flatten_qkv": parts[0], "pool": parts[1], "mask": parts[2],
+        "breakdown_ms": {"flatten_pool_qk": parts[0], "flatten_v": parts[1], "mask": parts[2],
                          "sparse_attn": parts[3], "unflatten_o": parts[4]},
         "roofline": {"bound": "tensor", "kernel": "sparse_attn_kernel<128>",
                      "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
@@ -250,8 +262,12 @@ def run_gpu(args, rank, world, local_rank):
                      "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long loop)",
                      "frac_of_burst": achieved_tf / burst_tf,
                      "flop_per_kept_tile": flop_per_tile},
-        "mask_path_gbs": (shape.B * shape.heads * shape.N * shape.d * 2 * 2
-                          + 2 * rows * shape.d * 8) / ((parts[1] + parts[2]) * 1e-3) / 1e9,
+        # HBM kernels: algorithmic bytes / time (read + write, each byte once)
+        "hbm_gbs": {"flatten_pool_qk": (4 * tensor_bytes + 2 * rows * shape.d * 8)
+                    / (parts[0] * 1e-3) / 1e9,
+                    "flatten_v": 2 * tensor_bytes / (parts[1] * 1e-3) / 1e9,
+                    "unflatten_o": 2 * tensor_bytes / (parts[4] * 1e-3) / 1e9,
+                    "peak": peak_gbs},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }

@@ -19,6 +19,7 @@ from . import _lib
 from ._lib import VsaError, vsa_mask_params, vsa_shape
 
 __all__ = ["Shape", "MaskParams", "VsaError", "fractal_flatten", "fractal_unflatten",
+           "flatten_pool_qk",
            "pool_qk", "block_mask", "block_mask_workspace_size", "sparse_attn_fwd",
            "sparse_attn_workspace_size", "attention_layer", "device_status", "version",
            "Csr"]
@@ -109,6 +110,20 @@ def pool_qk(qf: torch.Tensor, kf: torch.Tensor, shape: Shape, out=None, stream=N
     _lib.check(_lib.load().vsa_pool_qk(_ptr(qf), _ptr(kf), _ptr(qp), _ptr(kp), shape.c(),
                                        _stream(stream)))
     return qp, kp
+
+
+def flatten_pool_qk(q: torch.Tensor, k: torch.Tensor, shape: Shape, out=None, stream=None):
+    """Fractal flatten of raster Q and K plus their 64-token block means in one
+    pass -> (qf, kf, qp, kp); identical to fractal_flatten + pool_qk."""
+    if out is None:
+        sz = (shape.B, shape.heads, shape.Nb, shape.d)
+        out = (torch.empty_like(q), torch.empty_like(k),
+               torch.empty(sz, dtype=torch.float64, device=q.device),
+               torch.empty(sz, dtype=torch.float64, device=q.device))
+    qf, kf, qp, kp = out
+    _lib.check(_lib.load().vsa_flatten_pool_qk(_ptr(q), _ptr(k), _ptr(qf), _ptr(kf), _ptr(qp),
+                                               _ptr(kp), shape.c(), _stream(stream)))
+    return qf, kf, qp, kp
 
 
 def block_mask_workspace_size(shape: Shape) -> int:

@@ -68,7 +68,87 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint4 *__restrict__ q,
   }
 }
 
+// Steps 1 and 2 in one pass over Q and K.  One warp takes one 64-token block
+// (one P x P patch of one frame): it reads the block's 8 raster runs of 8
+// tokens, writes them as the block's contiguous 64 flattened tokens, and sums
+// the columns on the way, so the flattened tensors are never read back.  Lane
+// l always holds 16-byte column group l % (D/8) of its tokens, which keeps
+// its 8 fp64 accumulators on fixed columns (the same split as pool_kernel,
+// hence the same exact sums).  Units [0, blocks) are Q, [blocks, 2*blocks) K.
+template <int D>
+__global__ void __launch_bounds__(256)
+    flatten_pool_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ k,
+                        uint4 *__restrict__ qf, uint4 *__restrict__ kf, double *__restrict__ qp,
+                        double *__restrict__ kp, int64_t blocks, int64_t Nb, int H, int W) {
+  constexpr int kVecPerRow = D / 8;              // 16-byte vectors per token
+  constexpr int kVecPerRun = 8 * kVecPerRow;     // one patch row: 8 tokens
+  constexpr int kPerLane = kVecPerRun / 32;      // vectors per lane per run
+  const int lane = threadIdx.x & 31;
+  const int col = lane % kVecPerRow;
+  const int Wb = W >> 3;
+  const int64_t per_frame = static_cast<int64_t>(H >> 3) * Wb;
+  const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+       w < 2 * blocks; w += warps) {
+    const bool is_k = w >= blocks;
+    const int64_t g = is_k ? w - blocks : w;     // (bh, block) flattened
+    const int64_t bh = g / Nb, blk = g % Nb;
+    const int64_t t = blk / per_frame, rem = blk % per_frame;
+    const int py = static_cast<int>(rem / Wb), px = static_cast<int>(rem % Wb);
+    const int64_t head = bh * Nb * 64;           // first token of the head
+    const uint4 *src = (is_k ? k : q) + (head + (t * H + py * 8) * W + px * 8) * kVecPerRow;
+    uint4 *dst = (is_k ? kf : qf) + (head + blk * 64) * kVecPerRow;
+    double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll 2
+    for (int i = 0; i < 8; ++i) {                // patch row i: raster row py*8 + i
+      const uint4 *run = src + static_cast<int64_t>(i) * W * kVecPerRow;
+      uint4 v[kPerLane];
+#pragma unroll
+      for (int j = 0; j < kPerLane; ++j) v[j] = __ldcs(run + lane + 32 * j);
+#pragma unroll
+      for (int j = 0; j < kPerLane; ++j) {
+        __stcs(dst + i * kVecPerRun + lane + 32 * j, v[j]);
+        const uint32_t u[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          acc[2 * e] += bf16_to_f64(u[e] & 0xFFFFu);
+          acc[2 * e + 1] += bf16_to_f64(u[e] >> 16);
+        }
+      }
+    }
+#pragma unroll
+    for (int off = kVecPerRow; off < 32; off <<= 1)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] += __shfl_xor_sync(0xFFFFFFFFu, acc[j], off);
+    if (lane < kVecPerRow) {
+      double2 *d2 = reinterpret_cast<double2 *>((is_k ? kp : qp) + g * D + col * 8);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        d2[j] = make_double2(acc[2 * j] * 0.015625, acc[2 * j + 1] * 0.015625);
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_flatten_pool_qk(const void *q, const void *k, void *qf, void *kf, double *qp,
+                                   double *kp, const Geometry &g, cudaStream_t st) {
+  const int64_t blocks = g.BH * g.Nb;
+  if (blocks == 0) return cudaSuccess;
+  const int64_t want = (2 * blocks + 7) / 8;
+  const int grid = static_cast<int>(want < 32LL * num_sms() ? want : 32LL * num_sms());
+  const uint4 *q4 = static_cast<const uint4 *>(q);
+  const uint4 *k4 = static_cast<const uint4 *>(k);
+  uint4 *qf4 = static_cast<uint4 *>(qf);
+  uint4 *kf4 = static_cast<uint4 *>(kf);
+  if (g.d == 128)
+    flatten_pool_kernel<128><<<grid, 256, 0, st>>>(q4, k4, qf4, kf4, qp, kp, blocks, g.Nb, g.H,
+                                                   g.W);
+  else
+    flatten_pool_kernel<64><<<grid, 256, 0, st>>>(q4, k4, qf4, kf4, qp, kp, blocks, g.Nb, g.H,
+                                                  g.W);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_pool_qk(const void *qf, const void *kf, double *qp, double *kp,
                            const Geometry &g, cudaStream_t st) {

@@ -137,6 +137,39 @@ vsa_status vsa_pool_qk(const void *qf, const void *kf, double *qp, double *kp, v
   return e == cudaSuccess ? VSA_OK : cuda_fail(e, "pool launch");
 }
 
+static bool overlap(const void *a, size_t abytes, const void *b, size_t bbytes) {
+  const char *x = static_cast<const char *>(a);
+  const char *y = static_cast<const char *>(b);
+  return x < y + bbytes && y < x + abytes;
+}
+
+vsa_status vsa_flatten_pool_qk(const void *q, const void *k, void *qf, void *kf, double *qp,
+                               double *kp, vsa_shape s, void *stream) {
+  vsa_status st = check_shape(s);
+  if (st != VSA_OK) return st;
+  if (empty(s)) return VSA_OK;
+  if (!q || !k || !qf || !kf || !qp || !kp) return fail(VSA_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(qf) || !aligned16(kf) || !aligned16(qp) ||
+      !aligned16(kp))
+    return fail(VSA_ERR_UNSUPPORTED, "tensor pointers must be 16-byte aligned");
+  const vsa::Geometry g = vsa::geometry(s);
+  const size_t bytes = static_cast<size_t>(g.BH * g.N) * g.d * 2;
+  const size_t pbytes = static_cast<size_t>(g.BH * g.Nb) * g.d * 8;
+  // every output against every other buffer (the inputs may alias each other)
+  const void *outs[4] = {qf, kf, qp, kp};
+  const size_t osz[4] = {bytes, bytes, pbytes, pbytes};
+  for (int i = 0; i < 4; ++i) {
+    if (overlap(outs[i], osz[i], q, bytes) || overlap(outs[i], osz[i], k, bytes))
+      return fail(VSA_ERR_INVALID_ARG, "an output overlaps an input");
+    for (int j = i + 1; j < 4; ++j)
+      if (overlap(outs[i], osz[i], outs[j], osz[j]))
+        return fail(VSA_ERR_INVALID_ARG, "outputs overlap");
+  }
+  cudaError_t e = vsa::launch_flatten_pool_qk(q, k, qf, kf, qp, kp, g,
+                                              static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? VSA_OK : cuda_fail(e, "flatten+pool launch");
+}
+
 size_t vsa_block_mask_workspace_size(vsa_shape s) {
   if (check_shape(s) != VSA_OK) return 0;
   return vsa::block_mask_workspace_bytes(vsa::geometry(s));

@@ -34,6 +34,8 @@ cudaError_t launch_fractal_permute(const void *src, void *dst, const Geometry &g
                                    cudaStream_t st);
 cudaError_t launch_pool_qk(const void *qf, const void *kf, double *qp, double *kp,
                            const Geometry &g, cudaStream_t st);
+cudaError_t launch_flatten_pool_qk(const void *q, const void *k, void *qf, void *kf, double *qp,
+                                   double *kp, const Geometry &g, cudaStream_t st);
 
 // Block mask: workspace carve-up and launch.
 size_t block_mask_workspace_bytes(const Geometry &g);

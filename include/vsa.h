@@ -92,6 +92,18 @@ vsa_status vsa_fractal_unflatten(const void *y, void *x, vsa_shape s, void *stre
 vsa_status vsa_pool_qk(const void *qf, const void *kf, double *qp, double *kp,
                        vsa_shape s, void *stream);
 
+/* 1.+2. fused: fractal flattening of Q and K and their block means in one
+ * pass (NABLA, Methodology items 1-2), so the flattened tensors are not read
+ * back for pooling.  Results are bit-identical to
+ *   vsa_fractal_flatten(q -> qf), vsa_fractal_flatten(k -> kf),
+ *   vsa_pool_qk(qf, kf -> qp, kp).
+ * q, k   : device bf16 [B,heads,N,d] in raster order (may alias each other).
+ * qf, kf : device bf16 [B,heads,N,d], flattened order (outputs).
+ * qp, kp : device fp64 [B,heads,Nb,d] (outputs).
+ * No output may overlap an input or another output (VSA_ERR_INVALID_ARG). */
+vsa_status vsa_flatten_pool_qk(const void *q, const void *k, void *qf, void *kf, double *qp,
+                               double *kp, vsa_shape s, void *stream);
+
 /* 3.-4. Block mask (NABLA, Methodology items 2-3).
  * For every (b, h) and query block r: A[r,:] = softmax(qp_r . kp_c / sqrt(d))
  * over the Nb key blocks c, CDF selection at thr, union with the STA window

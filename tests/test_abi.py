@@ -74,3 +74,19 @@ def test_attention_workspace_validation():
                                0.0, P(1 << 28), P(1 << 29), P(1 << 30), 8, None)
     assert st == 3
     assert L.vsa_sparse_attn_workspace_size(s.c()) > 0
+
+
+def test_flatten_pool_validation():
+    L = _lib.load()
+    s = Shape(1, 2, 4, 16, 16, 64).c()          # 256 KiB per bf16 tensor
+    P = ctypes.c_void_p
+    MB = 1 << 20
+    def call(q=1 * MB, k=2 * MB, qf=3 * MB, kf=4 * MB, qp=5 * MB, kp=6 * MB):
+        return L.vsa_flatten_pool_qk(P(q), P(k), P(qf), P(kf), P(qp), P(kp), s, None)
+    assert call(q=0) == 1
+    assert call(kp=0) == 1
+    assert call(qf=3 * MB + 8) == 2                 # misaligned
+    assert call(qf=1 * MB + 4096) == 1              # output inside an input
+    assert call(kf=3 * MB + 65536) == 1             # two outputs overlap
+    assert call(qp=4 * MB + 128 * 1024) == 1        # pooled output inside kf
+    assert len(L.vsa_last_error()) > 0

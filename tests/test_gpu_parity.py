@@ -78,6 +78,31 @@ def test_pool_bit_exact(name):
     np.testing.assert_array_equal(kp.cpu().numpy(), oracle.pool(kf))
 
 
+# ---------------------------------------------------------------- a1+a2 fused
+@pytest.mark.parametrize("name,d,heads", [("tiny", None, None), ("wan1.3b-480p", None, 3),
+                                          ("tiny", 128, None)])
+def test_flatten_pool_fused_bit_exact(name, d, heads):
+    wl = workloads.get(name)
+    if d is not None:
+        wl = workloads.Workload(**{**wl.__dict__, "d": d})
+    q, k, _ = workloads.make_qkv(wl, heads=range(heads)) if heads else workloads.make_qkv(wl)
+    shape = vsa.Shape(wl.B, q.shape[1], wl.T, wl.H, wl.W, wl.d)
+    qd, kd = dev(q), dev(k)
+    qf, kf, qp, kp = vsa.flatten_pool_qk(qd, kd, shape)
+    qf_o, kf_o = (oracle.flatten(x, wl.T, wl.H, wl.W) for x in (q, k))
+    np.testing.assert_array_equal(u16(qf), qf_o)
+    np.testing.assert_array_equal(u16(kf), kf_o)
+    np.testing.assert_array_equal(qp.cpu().numpy(), oracle.pool(qf_o))
+    np.testing.assert_array_equal(kp.cpu().numpy(), oracle.pool(kf_o))
+    # the separate entry points give the same bits
+    qp2, kp2 = vsa.pool_qk(vsa.fractal_flatten(qd, shape), vsa.fractal_flatten(kd, shape), shape)
+    assert torch.equal(qp, qp2) and torch.equal(kp, kp2)
+    # Q and K may be the same tensor
+    _, _, qp3, kp3 = vsa.flatten_pool_qk(qd, qd, shape)
+    assert torch.equal(qp3, qp) and torch.equal(kp3, qp)
+    vsa.device_status()
+
+
 # ---------------------------------------------------------------- a3/a4 mask
 def compare_csr(csr, keep_o, diag_o, thr, rows=None):
     """GPU CSR vs oracle kept flags.  Returns (#ambiguous rows, #mismatches there)."""
