@@ -49,6 +49,9 @@ def parse_args():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="thr x STA sweep at the Wan-14B 720p shape: one JSON line per point "
+                         "(mask + attention; inputs generated once)")
     return ap.parse_args()
 
 
@@ -276,6 +279,71 @@ def run_gpu(args, rank, world, local_rank):
     return result, (q, k, v, wl)
 
 
+# --------------------------------------------------------------------------- sweep
+def run_sweep(args):
+    """Mask + attention at every (thr, STA) point of the Wan-14B sweep, on one
+    set of inputs (the points differ only in the mask parameters)."""
+    import torch
+    import content_adaptive_block_fractal_b200 as vsa
+    from content_adaptive_block_fractal_b200 import workloads
+
+    torch.cuda.set_device(0)
+    points = workloads.sweep_workloads()
+    wl0 = points[0]
+    shape = vsa.Shape.of(wl0)
+    q, k, v = workloads.make_qkv(wl0)
+    qd, kd, vd = (x.cuda() for x in (q, k, v))
+    layer = vsa.Layer(shape, vsa.MaskParams(wl0.thr, wl0.use_sta, wl0.sta), qd.device)
+    qf, kf = torch.empty_like(qd), torch.empty_like(kd)
+    vsa.flatten_pool_qk(qd, kd, shape, out=(qf, kf, layer.qp, layer.kp))
+    vf = vsa.fractal_flatten(vd, shape)
+    del q, k, v
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=qd.device)
+    stream = torch.cuda.current_stream()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    burst_tf, peak_tf, _, peak_src = measured_peaks()
+    flop_per_tile = 4 * 64 * 64 * shape.d
+    steps = max(args.steps, 1)
+    for wl in points:
+        params = vsa.MaskParams(wl.thr, wl.use_sta, wl.sta)
+
+        def step(record=False):
+            if record: ev[0].record(stream)
+            vsa.block_mask(layer.qp, layer.kp, shape, params, out=layer.csr,
+                           workspace=layer.ws_mask)
+            if record: ev[1].record(stream)
+            vsa.sparse_attn_fwd(qf, kf, vf, layer.csr.row_ptr, layer.csr.col_idx, shape, 0.0,
+                                out=(layer.o, layer.lse), workspace=layer.ws_attn)
+            if record: ev[2].record(stream)
+
+        for _ in range(max(args.warmup, 3)):
+            step()
+        vsa.device_status()
+        kept = int(layer.csr.row_ptr[-1].item())
+        t_mask = t_attn = 0.0
+        with ClockSampler(0) as clk:
+            for _ in range(steps):
+                flush.zero_()
+                step(record=True)
+                ev[2].synchronize()
+                t_mask += ev[0].elapsed_time(ev[1])
+                t_attn += ev[1].elapsed_time(ev[2])
+        vsa.device_status()
+        t_mask /= steps
+        t_attn /= steps
+        tf = kept * flop_per_tile / (t_attn * 1e-3) / 1e12
+        print(json.dumps({
+            "metric": "mask + sparse attention ms at Wan-14B 720p shape, sweep point",
+            "value": t_mask + t_attn, "unit": "ms", "steps": steps,
+            "config": {"workload": wl.name, "thr": wl.thr, "sta": wl.use_sta,
+                       "seed": wl.seed, "data": "synthetic"},
+            "kept_tiles": kept, "kept_fraction": kept / (shape.B * shape.heads * shape.Nb ** 2),
+            "mask_ms": t_mask, "sparse_attn_ms": t_attn, "kept_tile_tflops": tf,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": peak_tf, "frac": tf / peak_tf,
+                         "peak_source": f"{peak_src} bf16 sustained"},
+            "clocks": clk.summary()}), flush=True)
+
+
 # --------------------------------------------------------------------------- CPU oracle
 def oracle_sample(wl, heads, n_qblocks, seed=0):
     """Time the oracle on `heads` (flatten, pool, mask in full; attention on
@@ -348,6 +416,10 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             run_reference(args)
+        return
+    if args.sweep:
+        if rank == 0:
+            run_sweep(args)
         return
     if world > 1:
         import datetime
