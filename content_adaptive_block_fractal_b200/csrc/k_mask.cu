@@ -3,9 +3,10 @@
 // union with the sliding-tile window; Sparse VideoGen2 section 2B: top-p).
 //
 // Four kernels:
-//   mask_scores_kernel  persistent; one work item = 64 query blocks of one
-//                       (batch, head).  Forms the 64 x Nb pooled scores with
-//                       fp64 tensor-core MMAs (m8n8k4) in column tiles of 128,
+//   mask_scores_kernel  persistent; one work unit = 64 query blocks x 128 key
+//                       blocks of one (batch, head), units split evenly over
+//                       the CTAs.  Forms the pooled scores with fp64
+//                       tensor-core MMAs (m8n8k4), K streamed in slices,
 //                       writes each tile's row maxima in fp64 and
 //                       2^(t - tile max) as fp32 to the workspace slab.
 //   mask_select_kernel  one warp per row: rescales the slab row to the row
@@ -35,6 +36,8 @@ constexpr int kCT = 128;      // key blocks per phase-A column tile
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kPad = 4;       // fp64 padding per smem row (conflict-free fragments)
+constexpr int kKS = 32;       // columns of d per K slice in the score kernel
+constexpr int kLdK = kKS + kPad;
 constexpr int kCand = 256;    // per-warp candidate list capacity
 constexpr int kBins = 64;     // 1/8-octave probability bins (8 octaves below the max)
 constexpr int kMaxWords = 256;  // kept-bit words per row held in SMEM (Nb <= 8192)
@@ -68,8 +71,12 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool va
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem), "r"(n)
                : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ double warp_sum(double v) {
@@ -195,7 +202,7 @@ __device__ void cut_by_bisection(int Nb, const float *ebuf, uint32_t kmax, doubl
 //      if the fp32 histogram misled step 2) the bisection path decides.
 __device__ void select_row(const MaskArgs &a, int64_t grow, int r, const float *slab_row,
                            const double *tmax_row, float *ebuf, uint32_t *cand_key,
-                           int32_t *cand_idx, double *tscale, int *hcnt, float *hmass,
+                           int32_t *cand_idx, float *tscale, int *hcnt, float *hmass,
                            uint32_t *wbits) {
   const int lane = threadIdx.x & 31;
   const int Nb = a.Nb;
@@ -203,7 +210,7 @@ __device__ void select_row(const MaskArgs &a, int64_t grow, int r, const float *
   double M = -INFINITY;
   for (int t = lane; t < a.ntiles; t += 32) M = fmax(M, tmax_row[t]);
   M = warp_max(M);
-  for (int t = lane; t < a.ntiles; t += 32) tscale[t] = exp2(tmax_row[t] - M);
+  for (int t = lane; t < a.ntiles; t += 32) tscale[t] = static_cast<float>(exp2(tmax_row[t] - M));
   for (int b = lane; b < kBins; b += 32) {
     hcnt[b] = 0;
     hmass[b] = 0.0f;
@@ -223,13 +230,19 @@ __device__ void select_row(const MaskArgs &a, int64_t grow, int r, const float *
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       const float x4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      // the four entries share a 128-column tile (c0 is a multiple of 4)
+      const float ts = c0 + 128 * u < Nb ? tscale[(c0 + 128 * u) / kCT] : 0.0f;
+      float e4[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) e4[j] = c0 + 128 * u + j < Nb ? x4[j] * ts : 0.0f;
+      // row mass: fp32 sums of four, fp64 across (relative error ~1e-7)
+      z += static_cast<double>((e4[0] + e4[1]) + (e4[2] + e4[3]));
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int c = c0 + 128 * u + j;
         if (c < Nb) {
-          const float e = static_cast<float>(static_cast<double>(x4[j]) * tscale[c / kCT]);
+          const float e = e4[j];
           ebuf[c] = e;
-          z += static_cast<double>(e);
           const uint32_t k = __float_as_uint(e);
           kmax = max(kmax, k);
           if (need_cut) {
@@ -284,6 +297,9 @@ __device__ void select_row(const MaskArgs &a, int64_t grow, int r, const float *
         const float e = c < Nb ? ebuf[c] : 0.0f;
         const int b = c < Nb ? prob_bin(__float_as_uint(e)) : kBins;
         if (b < found) base += static_cast<double>(e);
+        // entries above the cut bin are kept whatever the bin's order
+        const uint32_t above = __ballot_sync(0xFFFFFFFFu, b < found);
+        if (lane == 0) wbits[c0 >> 5] = above;
         const bool in = b == found;
         const uint32_t m = __ballot_sync(0xFFFFFFFFu, in);
         if (in) {
@@ -326,9 +342,10 @@ __device__ void select_row(const MaskArgs &a, int64_t grow, int r, const float *
         const double total = __shfl_sync(0xFFFFFFFFu, inc, 31);
         if (base + total >= target) {
           // kept while the mass before the entry is still below the target
+          __syncwarp();
           if (valid && base + (inc - p) < target) {
             const int c = static_cast<int>(key & 0xFFFFFFFFu);
-            ebuf[c] = __uint_as_float(__float_as_uint(ebuf[c]) | 0x80000000u);
+            atomicOr(&wbits[c >> 5], 1u << (c & 31));
           }
           cut_bin = found;
           decided = true;
@@ -340,17 +357,16 @@ __device__ void select_row(const MaskArgs &a, int64_t grow, int r, const float *
       cut_by_bisection(Nb, ebuf, kmax, target, cand_key, cand_idx, vkey, need_ties, keep_all);
   }
 
-  // kept bits: above the cut (or marked), ties by index on the bisection path
+  // kept bits (the histogram path wrote them already): everything, or above
+  // the bisection cut with ties by index
   int ties_seen = 0;
-  for (int w = 0; w < a.words; ++w) {
+  for (int w = 0; cut_bin < 0 && w < a.words; ++w) {
     const int c = w * 32 + lane;
     const bool valid = c < Nb;
     const uint32_t k = valid ? __float_as_uint(ebuf[c]) : 0u;
     bool kept;
     if (keep_all) {
       kept = valid;
-    } else if (cut_bin >= 0) {
-      kept = valid && ((k >> 31) || prob_bin(k) < cut_bin);
     } else {
       kept = valid && k > vkey;
       const bool tie = valid && k == vkey;
@@ -391,105 +407,141 @@ __device__ void select_row(const MaskArgs &a, int64_t grow, int r, const float *
   __syncwarp();
 }
 
+// Work unit = (batch-head, 64-row tile, 128-column tile), numbered row-tile
+// major; CTA i takes the contiguous range [i*U/G, (i+1)*U/G), so the units
+// are spread evenly and a CTA meets a new row tile (and reloads Q) only a few
+// times.  K comes in slices of kKS columns of d through two cp.async buffers:
+// the next slice (the next unit's first one at a unit's end) is in flight
+// while the current one feeds the DMMAs.
 __global__ void __launch_bounds__(kThreads, 1) mask_scores_kernel(const MaskArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   double *sQ = reinterpret_cast<double *>(smem_raw);
   const int ld = a.d + kPad;
-  double *sK = sQ + kRT * ld;
+  double *sK = sQ + kRT * ld;                  // [2][kCT][kLdK]
   __shared__ double sRed[kRT][4];
   __shared__ double sTileMax[kRT];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tq = lane & 3;
   const int wm = warp >> 2, wn = warp & 3;
-  const int vec_per_row = a.d / 2;  // 16-byte chunks per fp64 row
+  const int nslices = a.d / kKS;
+  const int64_t units = a.items * a.ntiles;
+  const int64_t u_begin = units * blockIdx.x / gridDim.x;
+  const int64_t u_end = units * (blockIdx.x + 1) / gridDim.x;
+  if (u_begin >= u_end) return;
 
-  for (int64_t item = blockIdx.x; item < a.items; item += gridDim.x) {
+  // K slice s (columns [s*kKS, s*kKS + kKS) of d) of unit u into buffer b
+  auto load_slice = [&](int64_t u, int sl, int b) {
+    const int64_t item = u / a.ntiles;
+    const int c0 = static_cast<int>(u % a.ntiles) * kCT;
+    const double *ksrc = a.kp + (item / a.tiles_per_head) * a.Nb * a.d + sl * kKS;
+    double *dst = sK + b * (kCT * kLdK);
+    for (int i = tid; i < kCT * (kKS / 2); i += kThreads) {
+      const int row = i / (kKS / 2), ch = i % (kKS / 2);
+      const bool ok = c0 + row < a.Nb;
+      cp_async16(dst + row * kLdK + ch * 2,
+                 ok ? ksrc + static_cast<int64_t>(c0 + row) * a.d + ch * 2 : a.kp, ok);
+    }
+    cp_async_commit();
+  };
+
+  load_slice(u_begin, 0, 0);
+  int buf = 0;
+  int64_t q_item = -1;
+  for (int64_t u = u_begin; u < u_end; ++u) {
+    const int64_t item = u / a.ntiles;
+    const int ct = static_cast<int>(u % a.ntiles);
     const int64_t bh = item / a.tiles_per_head;
     const int r0 = static_cast<int>(item % a.tiles_per_head) * kRT;
-    // rows of this item in the slab / tile-max arrays (rows past Nb belong
-    // to the next head or lie past the end: never written)
-    float *slab = a.slab + (bh * a.Nb + r0) * a.ld_slab;
-    double *tmax = a.tmax + (bh * a.Nb + r0) * a.ntiles;
-    const double *qsrc = a.qp + (bh * a.Nb + r0) * a.d;
-    const double *ksrc = a.kp + bh * a.Nb * a.d;
-
-    // ---- phase A: scores, tile maxima, exp2 slab
-    for (int i = tid; i < kRT * vec_per_row; i += kThreads) {
-      const int row = i / vec_per_row, ch = i % vec_per_row;
-      const bool ok = r0 + row < a.Nb;
-      cp_async16(sQ + row * ld + ch * 2, ok ? qsrc + row * a.d + ch * 2 : a.qp, ok);
-    }
-    for (int ct = 0; ct < a.ntiles; ++ct) {
-      const int c0 = ct * kCT;
-      for (int i = tid; i < kCT * vec_per_row; i += kThreads) {
+    const int c0 = ct * kCT;
+    if (item != q_item) {
+      // every warp finished the previous unit (barrier at its end)
+      const double *qsrc = a.qp + (bh * a.Nb + r0) * a.d;
+      const int vec_per_row = a.d / 2;
+      for (int i = tid; i < kRT * vec_per_row; i += kThreads) {
         const int row = i / vec_per_row, ch = i % vec_per_row;
-        const bool ok = c0 + row < a.Nb;
-        cp_async16(sK + row * ld + ch * 2,
-                   ok ? ksrc + static_cast<int64_t>(c0 + row) * a.d + ch * 2 : a.kp, ok);
+        const bool ok = r0 + row < a.Nb;
+        cp_async16(sQ + row * ld + ch * 2, ok ? qsrc + row * a.d + ch * 2 : a.qp, ok);
       }
-      cp_async_wait_all();
-      __syncthreads();
+      cp_async_commit();
+      q_item = item;
+    }
 
-      double acc[4][4][2];
+    double acc[4][4][2];
 #pragma unroll
-      for (int mi = 0; mi < 4; ++mi)
+    for (int mi = 0; mi < 4; ++mi)
 #pragma unroll
-        for (int ni = 0; ni < 4; ++ni) acc[mi][ni][0] = acc[mi][ni][1] = 0.0;
-      const double *qa = sQ + (wm * 32 + g) * ld + tq;
-      const double *kb = sK + (wn * 32 + g) * ld + tq;
+      for (int ni = 0; ni < 4; ++ni) acc[mi][ni][0] = acc[mi][ni][1] = 0.0;
+    for (int sl = 0; sl < nslices; ++sl) {
+      // prefetch the next slice (the next unit's first at the last slice)
+      bool more = true;
+      if (sl + 1 < nslices) load_slice(u, sl + 1, buf ^ 1);
+      else if (u + 1 < u_end) load_slice(u + 1, 0, buf ^ 1);
+      else more = false;
+      // everything but the prefetch has landed: this slice (and Q)
+      if (more) cp_async_wait_group<1>();
+      else cp_async_wait_group<0>();
+      __syncthreads();
+      const double *qa = sQ + (wm * 32 + g) * ld + sl * kKS + tq;
+      const double *kb = sK + buf * (kCT * kLdK) + (wn * 32 + g) * kLdK + tq;
 #pragma unroll 2
-      for (int k = 0; k < a.d; k += 4) {
+      for (int k = 0; k < kKS; k += 4) {
         double af[4], bf[4];
 #pragma unroll
         for (int mi = 0; mi < 4; ++mi) af[mi] = qa[mi * 8 * ld + k];
 #pragma unroll
-        for (int ni = 0; ni < 4; ++ni) bf[ni] = kb[ni * 8 * ld + k];
+        for (int ni = 0; ni < 4; ++ni) bf[ni] = kb[ni * 8 * kLdK + k];
 #pragma unroll
         for (int mi = 0; mi < 4; ++mi)
 #pragma unroll
           for (int ni = 0; ni < 4; ++ni) dmma(acc[mi][ni], af[mi], bf[ni]);
       }
-      // scaled log2 scores; columns past Nb do not exist
+      __syncthreads();   // this buffer is refilled by the prefetch after next
+      buf ^= 1;
+    }
+
+    // scaled log2 scores; columns past Nb do not exist
+    float *slab = a.slab + (bh * a.Nb + r0) * a.ld_slab;
+    double *tmax = a.tmax + (bh * a.Nb + r0) * a.ntiles;
 #pragma unroll
-      for (int mi = 0; mi < 4; ++mi) {
-        double m = -INFINITY;
+    for (int mi = 0; mi < 4; ++mi) {
+      double m = -INFINITY;
 #pragma unroll
-        for (int ni = 0; ni < 4; ++ni)
+      for (int ni = 0; ni < 4; ++ni)
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int col = c0 + wn * 32 + ni * 8 + 2 * tq + j;
-            acc[mi][ni][j] = col < a.Nb ? acc[mi][ni][j] * a.c : -INFINITY;
-            m = fmax(m, acc[mi][ni][j]);
-          }
-        m = fmax(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-        m = fmax(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-        if (tq == 0) sRed[wm * 32 + mi * 8 + g][wn] = m;
-      }
-      __syncthreads();
-      if (tid < kRT) {
-        const double m = fmax(fmax(sRed[tid][0], sRed[tid][1]), fmax(sRed[tid][2], sRed[tid][3]));
-        sTileMax[tid] = m;
-        if (r0 + tid < a.Nb) tmax[tid * a.ntiles + ct] = m;
-      }
-      __syncthreads();
+        for (int j = 0; j < 2; ++j) {
+          const int col = c0 + wn * 32 + ni * 8 + 2 * tq + j;
+          acc[mi][ni][j] = col < a.Nb ? acc[mi][ni][j] * a.c : -INFINITY;
+          m = fmax(m, acc[mi][ni][j]);
+        }
+      m = fmax(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+      m = fmax(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+      if (tq == 0) sRed[wm * 32 + mi * 8 + g][wn] = m;
+    }
+    __syncthreads();
+    if (tid < kRT) {
+      const double m = fmax(fmax(sRed[tid][0], sRed[tid][1]), fmax(sRed[tid][2], sRed[tid][3]));
+      sTileMax[tid] = m;
+      if (r0 + tid < a.Nb) tmax[tid * a.ntiles + ct] = m;
+    }
+    __syncthreads();
 #pragma unroll
-      for (int mi = 0; mi < 4; ++mi) {
-        const int row = wm * 32 + mi * 8 + g;
-        const double m = sTileMax[row];
+    for (int mi = 0; mi < 4; ++mi) {
+      const int row = wm * 32 + mi * 8 + g;
+      const double m = sTileMax[row];
 #pragma unroll
-        for (int ni = 0; ni < 4; ++ni) {
-          const int col = c0 + wn * 32 + ni * 8 + 2 * tq;
-          if (col < a.Nb && r0 + row < a.Nb) {
-            float2 e;
-            e.x = exp2_split(acc[mi][ni][0] - m);
-            e.y = exp2_split(acc[mi][ni][1] - m);
-            *reinterpret_cast<float2 *>(slab + row * a.ld_slab + col) = e;
-          }
+      for (int ni = 0; ni < 4; ++ni) {
+        const int col = c0 + wn * 32 + ni * 8 + 2 * tq;
+        if (col < a.Nb && r0 + row < a.Nb) {
+          float2 e;
+          e.x = exp2_split(acc[mi][ni][0] - m);
+          e.y = exp2_split(acc[mi][ni][1] - m);
+          *reinterpret_cast<float2 *>(slab + row * a.ld_slab + col) = e;
         }
       }
-      __syncthreads();  // sK is overwritten by the next tile
     }
+    // sRed / sTileMax and sQ are reused by the next unit
+    __syncthreads();
   }
 }
 
@@ -503,7 +555,7 @@ __global__ void __launch_bounds__(kThreads) mask_select_kernel(const MaskArgs a)
   float *ebuf = reinterpret_cast<float *>(wbase);
   uint32_t *cand_key = reinterpret_cast<uint32_t *>(ebuf + a.Nb);
   int32_t *cand_idx = reinterpret_cast<int32_t *>(cand_key + kCand);
-  double *tscale = reinterpret_cast<double *>(
+  float *tscale = reinterpret_cast<float *>(
       (reinterpret_cast<uintptr_t>(cand_idx + kCand) + 15) & ~static_cast<uintptr_t>(15));
   int *hcnt = reinterpret_cast<int *>(tscale + a.ntiles);
   float *hmass = reinterpret_cast<float *>(hcnt + kBins);
@@ -597,7 +649,7 @@ MaskLayout mask_layout(const Geometry &g, int grid) {
   L.counts_off = off;
   off = align256(off + static_cast<size_t>(g.BH * g.Nb) * 4);
   L.total = off;
-  L.smem_a = static_cast<size_t>(kRT + kCT) * (g.d + kPad) * 8;
+  L.smem_a = (static_cast<size_t>(kRT) * (g.d + kPad) + 2 * static_cast<size_t>(kCT) * kLdK) * 8;
   L.smem_b = static_cast<size_t>(kWarps) *
              (static_cast<size_t>(g.Nb) * 4 + kCand * 8 + L.ntiles * 8 + 16 + kBins * 8 +
               kMaxWords * 4);
@@ -622,9 +674,10 @@ cudaError_t launch_block_mask(const double *qp, const double *kp, const Geometry
   }
   const int64_t tiles_per_head = (g.Nb + kRT - 1) / kRT;
   const int64_t items = g.BH * tiles_per_head;
+  const int64_t units = items * ((g.Nb + kCT - 1) / kCT);
   int grid = num_sms();
   if (grid > kMaxGrid) grid = kMaxGrid;
-  if (items < grid) grid = static_cast<int>(items);
+  if (units < grid) grid = static_cast<int>(units);
   MaskLayout L = mask_layout(g, grid);
   unsigned char *w = static_cast<unsigned char *>(ws);
   MaskArgs a;
