@@ -55,6 +55,10 @@ def lib():
         L.oracle_sta_keep.restype = _I
         L.oracle_block_mask.argtypes = [_P, _P, _I64, _I, _I, _I, _I, _D, _I, _I,
                                         _I, _I, _P, _I64, _P, _P]
+        L.oracle_select_topk_row.argtypes = [_P, _I, _I, _P, _P]
+        L.oracle_block_mask_topk.argtypes = [_P, _P, _I64, _I, _I, _I, _I, _I, _I, _I,
+                                             _I, _I, _P, _I64, _P, _P]
+        L.oracle_sta_mask.argtypes = [_I, _I, _I, _I, _I, _I, _P]
         L.oracle_sparse_attention.argtypes = [_P, _P, _P, _I64, _I64, _I, _P, _P,
                                               _D, _P, _I64, _P, _P]
     return _lib
@@ -171,6 +175,56 @@ def block_mask(qp: np.ndarray, kp: np.ndarray, Hb: int, Wb: int, thr: float,
                             int(bool(use_sta)), int(sta[0]), int(sta[1]), int(sta[2]),
                             rp, n, _ptr(keep), _ptr(diag))
     return keep, diag
+
+
+def block_mask_topk(qp: np.ndarray, kp: np.ndarray, Hb: int, Wb: int, k: int,
+                    use_sta: bool, sta=(1, 1, 1), rows=None):
+    """Static-ratio mask: kept flags (uint8, rows x Nb) and, per row, the last
+    kept and first dropped probabilities (rows x 2)."""
+    qp = np.ascontiguousarray(qp, dtype=np.float64)
+    kp = np.ascontiguousarray(kp, dtype=np.float64)
+    Nb, d = qp.shape[-2], qp.shape[-1]
+    BH = qp.size // (Nb * d)
+    if rows is None:
+        n, rp = BH * Nb, None
+    else:
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        n, rp = rows.size, _ptr(rows)
+    keep = np.zeros((n, Nb), dtype=np.uint8)
+    diag = np.zeros((n, 2))
+    lib().oracle_block_mask_topk(_ptr(qp), _ptr(kp), BH, Nb, d, Hb, Wb, int(k),
+                                 int(bool(use_sta)), int(sta[0]), int(sta[1]), int(sta[2]),
+                                 rp, n, _ptr(keep), _ptr(diag))
+    return keep, diag
+
+
+def select_topk_row(a: np.ndarray, k: int):
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    keep = np.zeros(a.size, dtype=np.uint8)
+    diag = np.zeros(2)
+    lib().oracle_select_topk_row(_ptr(a), a.size, int(k), _ptr(keep), _ptr(diag))
+    return keep, diag
+
+
+def sta_mask(T: int, Hb: int, Wb: int, sta=(1, 1, 1)) -> np.ndarray:
+    """The STA window alone: kept flags of one head's (T*Hb*Wb)^2 block grid."""
+    Nb = T * Hb * Wb
+    keep = np.zeros((Nb, Nb), dtype=np.uint8)
+    lib().oracle_sta_mask(Nb, Hb, Wb, int(sta[0]), int(sta[1]), int(sta[2]), _ptr(keep))
+    return keep
+
+
+def ambiguous_topk(diag: np.ndarray, eps: float = 1e-5, row_max=None) -> np.ndarray:
+    """Static-ratio rows whose kept set is not fixed by fp32-accurate
+    probabilities: the last kept and first dropped probabilities within a
+    relative eps of each other (a near tie across the cut), or, when the row
+    maxima are given, a cut probability below 2^-120 of the row maximum (where
+    fp32 storage of the ratio underflows)."""
+    last, nxt = diag[:, 0], diag[:, 1]
+    amb = (nxt >= 0) & (np.abs(last - nxt) <= eps * np.maximum(last, 1e-300))
+    if row_max is not None:
+        amb |= (nxt >= 0) & (last < row_max * 2.0 ** -120)
+    return amb
 
 
 def mask_to_csr(keep: np.ndarray):

@@ -283,6 +283,80 @@ void oracle_block_mask(const double *qp, const double *kp, int64_t BH, int Nb,
 }
 
 /*
+ * Static-ratio selection (DynamicRad summary, section 2, "Dual-Mode
+ * Strategy", Static-Ratio mode: every row keeps a fixed share of its
+ * blocks).  The page does not say which blocks; reading taken: the k blocks of
+ * highest reduced-attention probability, ordered exactly as in the top-p rule
+ * (probability descending, equal probabilities to the lower block index);
+ * k >= n keeps the whole row, k <= 0 keeps nothing.  diag[0] is the last kept
+ * probability, diag[1] the first dropped one (-1 where there is none).
+ */
+void oracle_select_topk_row(const double *a, int n, int k, uint8_t *keep,
+                            double *diag)
+{
+    if (n <= 0)
+        return;
+    ranked *r = (ranked *)malloc(sizeof(ranked) * (size_t)n);
+    for (int c = 0; c < n; ++c) {
+        r[c].p = a[c];
+        r[c].idx = c;
+    }
+    qsort(r, (size_t)n, sizeof(ranked), ranked_cmp);
+    memset(keep, 0, (size_t)n);
+    int kept = k < 0 ? 0 : (k < n ? k : n);
+    for (int i = 0; i < kept; ++i)
+        keep[r[i].idx] = 1;
+    if (diag) {
+        diag[0] = kept > 0 ? r[kept - 1].p : -1.0;
+        diag[1] = kept < n ? r[kept].p : -1.0;
+    }
+    free(r);
+}
+
+/* The static-ratio mask for the listed rows (all rows when rows is NULL),
+ * with the STA union as in oracle_block_mask.  diag: 2 values per row. */
+void oracle_block_mask_topk(const double *qp, const double *kp, int64_t BH,
+                            int Nb, int d, int Hb, int Wb, int k, int use_sta,
+                            int rt, int rh, int rw, const int64_t *rows,
+                            int64_t nrows, uint8_t *keep_out, double *diag_out)
+{
+    if (!rows)
+        nrows = BH * Nb;
+#pragma omp parallel
+    {
+        double *a = (double *)malloc(sizeof(double) * (size_t)Nb);
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t i = 0; i < nrows; ++i) {
+            int64_t row = rows ? rows[i] : i;
+            int64_t r = row % Nb;
+            uint8_t *keep = keep_out + i * Nb;
+            reduced_row(qp, kp, row, Nb, d, a);
+            oracle_select_topk_row(a, Nb, k, keep, diag_out ? diag_out + i * 2 : NULL);
+            if (use_sta)
+                for (int c = 0; c < Nb; ++c)
+                    if (oracle_sta_keep(r, c, Hb, Wb, rt, rh, rw))
+                        keep[c] = 1;
+        }
+        free(a);
+    }
+}
+
+/*
+ * The STA window on its own (NABLA summary, "Methodology" item 3, the
+ * sliding-tile component M_STA of M = M_nabla OR M_STA, used without the
+ * content-adaptive part): keep[r][c] = 1 exactly when key block c lies within
+ * the Chebyshev radii of query block r.  One head's Nb x Nb grid; every head
+ * has the same mask.
+ */
+void oracle_sta_mask(int Nb, int Hb, int Wb, int rt, int rh, int rw, uint8_t *keep)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < Nb; ++r)
+        for (int64_t c = 0; c < Nb; ++c)
+            keep[r * Nb + c] = (uint8_t)oracle_sta_keep(r, c, Hb, Wb, rt, rh, rw);
+}
+
+/*
  * O5. Block-sparse attention (NABLA, Methodology item 2, "expansion": the
  * block mask decides which 64 x 64 tiles are computed).  For every query token
  * of query block r, softmax attention over the keys of the kept key blocks

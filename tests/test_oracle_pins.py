@@ -298,3 +298,77 @@ def test_ambiguity_classifier():
                      [1.0, 0.85, 0.15, -1.0, 9]])      # nothing dropped
     np.testing.assert_array_equal(oracle.ambiguous_rows(diag, 0.1),
                                   [False, True, True, True, False])
+
+
+# ---------------------------------------------------------------- f2 static ratio (top-k)
+def test_topk_golden_rows():
+    for ln in _lines("topk_rows.txt"):
+        k, p, kept = (part.strip() for part in ln.split("|"))
+        keep, _ = oracle.select_topk_row(np.array([float(x) for x in p.split()]), int(k))
+        assert np.nonzero(keep)[0].tolist() == [int(x) for x in kept.split()], ln
+
+
+def test_topk_invariants_on_random_rows():
+    """Exactly min(k, n) kept; every kept probability >= every dropped one;
+    at the cut, an equal probability is kept only if every lower index with
+    that probability is kept too; k = 1 is numpy's argmax (first maximum)."""
+    rng = np.random.default_rng(5)
+    for trial in range(300):
+        n = int(rng.integers(1, 40))
+        # coarse values so that ties are common
+        p = rng.integers(0, 6, n).astype(np.float64)
+        p = p / max(p.sum(), 1.0)
+        for k in (1, 2, n // 2, n - 1, n, n + 3):
+            if k < 1:
+                continue
+            keep, diag = oracle.select_topk_row(p, k)
+            kept, dropped = p[keep == 1], p[keep == 0]
+            assert keep.sum() == min(k, n)
+            if dropped.size and kept.size:
+                assert kept.min() >= dropped.max()
+                cut = kept.min()
+                tied = np.nonzero(p == cut)[0]
+                flags = keep[tied]
+                assert np.all(np.diff(flags.astype(int)) <= 0), "a higher index won a tie"
+                assert diag[0] == cut and diag[1] == dropped.max()
+            if k == 1:
+                assert np.nonzero(keep)[0].tolist() == [int(np.argmax(p))]
+
+
+def test_topk_agrees_with_topp_prefix():
+    """Top-p keeps a prefix of the same (probability desc, index asc) order, so
+    top-k with k = the top-p count must keep the same set."""
+    wl = workloads.get("tiny")
+    q, k, _ = workloads.make_qkv(wl)
+    qf, kf = (oracle.flatten(x, wl.T, wl.H, wl.W) for x in (q, k))
+    qp, kp = oracle.pool(qf), oracle.pool(kf)
+    keep_p, _ = oracle.block_mask(qp, kp, wl.Hb, wl.Wb, 0.2, False)
+    counts = keep_p.sum(axis=1)
+    for kk in np.unique(counts):
+        rows = np.nonzero(counts == kk)[0]
+        keep_k, _ = oracle.block_mask_topk(qp, kp, wl.Hb, wl.Wb, int(kk), False, rows=rows)
+        np.testing.assert_array_equal(keep_k, keep_p[rows])
+
+
+def test_sta_mask_closed_form_and_fixture():
+    """Row counts are products of clipped window widths; the mask is symmetric;
+    radius 0 is the identity; it agrees with the hand-derived window fixture."""
+    for T, Hb, Wb, rad in [(3, 3, 3, (1, 1, 1)), (4, 2, 5, (0, 1, 2)), (2, 3, 4, (0, 0, 0)),
+                           (5, 4, 6, (2, 1, 1)), (2, 2, 2, (9, 9, 9))]:
+        m = oracle.sta_mask(T, Hb, Wb, rad)
+        Nb = T * Hb * Wb
+        r = np.arange(Nb)
+        t, y, x = r // (Hb * Wb), (r // Wb) % Hb, r % Wb
+
+        def span(c, rr, n):
+            return np.minimum(c + rr, n - 1) - np.maximum(c - rr, 0) + 1
+        want = span(t, rad[0], T) * span(y, rad[1], Hb) * span(x, rad[2], Wb)
+        np.testing.assert_array_equal(m.sum(axis=1), want)
+        np.testing.assert_array_equal(m, m.T)
+        if rad == (0, 0, 0):
+            np.testing.assert_array_equal(m, np.eye(Nb, dtype=np.uint8))
+    # the fixture lists the window of given rows on a 3x3x3 grid, radius 1
+    m = oracle.sta_mask(3, 3, 3, (1, 1, 1))
+    for ln in _lines("sta_window_T3_Hb3_Wb3_r1.txt"):
+        r, cols = (part.strip() for part in ln.split(":"))
+        assert np.nonzero(m[int(r)])[0].tolist() == [int(c) for c in cols.split()], ln
