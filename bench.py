@@ -16,6 +16,7 @@ oracle/) on a bounded sample of the same workload, extrapolated to one layer.
 from __future__ import annotations
 
 import argparse
+import functools
 import hashlib
 import json
 import math
@@ -304,13 +305,25 @@ def run_sweep(args):
     burst_tf, peak_tf, _, peak_src = measured_peaks()
     flop_per_tile = 4 * 64 * 64 * shape.d
     steps = max(args.steps, 1)
-    for wl in points:
-        params = vsa.MaskParams(wl.thr, wl.use_sta, wl.sta)
+    k10 = shape.Nb // 10
+    sta_csr = vsa.Csr(layer.csr.row_ptr, layer.csr.col_idx, layer.csr.kept_count)
+    cases = [(f"top-p thr={wl.thr}" + (" + STA" if wl.use_sta else ""), wl,
+              functools.partial(vsa.block_mask, layer.qp, layer.kp, shape,
+                                vsa.MaskParams(wl.thr, wl.use_sta, wl.sta),
+                                out=layer.csr, workspace=layer.ws_mask))
+             for wl in points]
+    for sta in (True, False):
+        cases.append((f"static-ratio k={k10} (Nb/10)" + (" + STA" if sta else ""), wl0,
+                      functools.partial(vsa.block_mask_topk, layer.qp, layer.kp, shape, k10,
+                                        vsa.MaskParams(0.0, sta, wl0.sta), out=layer.csr,
+                                        workspace=layer.ws_mask)))
+    cases.append(("STA window alone (+-1)", wl0,
+                  functools.partial(vsa.sta_mask, shape, wl0.sta, out=sta_csr)))
+    for label, wl, make_mask in cases:
 
         def step(record=False):
             if record: ev[0].record(stream)
-            vsa.block_mask(layer.qp, layer.kp, shape, params, out=layer.csr,
-                           workspace=layer.ws_mask)
+            make_mask()
             if record: ev[1].record(stream)
             vsa.sparse_attn_fwd(qf, kf, vf, layer.csr.row_ptr, layer.csr.col_idx, shape, 0.0,
                                 out=(layer.o, layer.lse), workspace=layer.ws_attn)
@@ -334,9 +347,10 @@ def run_sweep(args):
         tf = kept * flop_per_tile / (t_attn * 1e-3) / 1e12
         print(json.dumps({
             "metric": "mask + sparse attention ms at Wan-14B 720p shape, sweep point",
-            "value": t_mask + t_attn, "unit": "ms", "steps": steps,
-            "config": {"workload": wl.name, "thr": wl.thr, "sta": wl.use_sta,
-                       "seed": wl.seed, "data": "synthetic"},
+            "value": t_mask + t_attn, "unit": "ms", "steps": steps, "mask": label,
+            "config": {"workload": "wan14b-720p", "B": shape.B, "heads": shape.heads,
+                       "d": shape.d, "grid": [shape.T, shape.H, shape.W], "seed": wl.seed,
+                       "data": "synthetic"},
             "kept_tiles": kept, "kept_fraction": kept / (shape.B * shape.heads * shape.Nb ** 2),
             "mask_ms": t_mask, "sparse_attn_ms": t_attn, "kept_tile_tflops": tf,
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peak_tf, "frac": tf / peak_tf,

@@ -20,7 +20,8 @@ from ._lib import VsaError, vsa_mask_params, vsa_shape
 
 __all__ = ["Shape", "MaskParams", "VsaError", "fractal_flatten", "fractal_unflatten",
            "flatten_pool_qk",
-           "pool_qk", "block_mask", "block_mask_workspace_size", "sparse_attn_fwd",
+           "pool_qk", "block_mask", "block_mask_topk", "sta_mask", "sta_mask_nnz",
+           "block_mask_workspace_size", "sparse_attn_fwd",
            "sparse_attn_workspace_size", "attention_layer", "device_status", "version",
            "Csr"]
 
@@ -154,6 +155,51 @@ def block_mask(qp: torch.Tensor, kp: torch.Tensor, shape: Shape, params: MaskPar
         _ptr(qp), _ptr(kp), shape.c(), params.c(), _ptr(out.row_ptr), _ptr(out.col_idx),
         out.col_idx.numel(), _ptr(out.kept_count), _ptr(workspace), workspace.numel(),
         _stream(stream)))
+    return out
+
+
+def block_mask_topk(qp: torch.Tensor, kp: torch.Tensor, shape: Shape, k: int,
+                    params: MaskParams | None = None, out: Csr | None = None,
+                    workspace: torch.Tensor | None = None, stream=None) -> Csr:
+    """Static-ratio selection: each row's k most probable blocks [+ STA union
+    from params; params.thr is ignored] -> CSR kept lists."""
+    params = MaskParams(0.0, False) if params is None else params
+    rows = shape.B * shape.heads * shape.Nb
+    dev = qp.device
+    if out is None:
+        out = Csr(torch.empty(rows + 1, dtype=torch.int64, device=dev),
+                  torch.empty(max(rows * shape.Nb, 1), dtype=torch.int32, device=dev),
+                  torch.empty(max(rows, 1), dtype=torch.int32, device=dev))
+    if workspace is None:
+        workspace = _workspace(block_mask_workspace_size(shape), dev)
+    _lib.check(_lib.load().vsa_block_mask_topk(
+        _ptr(qp), _ptr(kp), shape.c(), int(k), params.c(), _ptr(out.row_ptr),
+        _ptr(out.col_idx), out.col_idx.numel(), _ptr(out.kept_count), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
+    return out
+
+
+def sta_mask_nnz(shape: Shape, radii=(1, 1, 1)) -> int:
+    """Entries of the STA-only mask: heads x product of summed clipped widths."""
+    def total(n, r):
+        return sum(min(c + r, n - 1) - max(c - r, 0) + 1 for c in range(n))
+    Hb, Wb = shape.H // shape.P, shape.W // shape.P
+    return (shape.B * shape.heads * total(shape.T, radii[0]) * total(Hb, radii[1])
+            * total(Wb, radii[2]))
+
+
+def sta_mask(shape: Shape, radii=(1, 1, 1), out: Csr | None = None, device="cuda",
+             stream=None) -> Csr:
+    """The STA window alone as the block mask (no pooling, no scores)."""
+    rows = shape.B * shape.heads * shape.Nb
+    if out is None:
+        nnz = sta_mask_nnz(shape, radii)
+        out = Csr(torch.empty(rows + 1, dtype=torch.int64, device=device),
+                  torch.empty(max(nnz, 1), dtype=torch.int32, device=device),
+                  torch.empty(max(rows, 1), dtype=torch.int32, device=device))
+    _lib.check(_lib.load().vsa_sta_mask(
+        shape.c(), int(radii[0]), int(radii[1]), int(radii[2]), _ptr(out.row_ptr),
+        _ptr(out.col_idx), out.col_idx.numel(), _ptr(out.kept_count), _stream(stream)))
     return out
 
 

@@ -19,7 +19,8 @@ STATUS_NAMES = {0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_UNSUPPORTED",
 # Every symbol include/vsa.h declares.
 EXPORTS = ("vsa_fractal_flatten", "vsa_fractal_unflatten", "vsa_pool_qk",
            "vsa_flatten_pool_qk",
-           "vsa_block_mask_workspace_size", "vsa_block_mask",
+           "vsa_block_mask_workspace_size", "vsa_block_mask", "vsa_block_mask_topk",
+           "vsa_sta_mask",
            "vsa_sparse_attn_workspace_size", "vsa_sparse_attn_fwd",
            "vsa_sparse_attn_fwd_noalloc",
            "vsa_last_error", "vsa_device_status", "vsa_version")
@@ -65,6 +66,10 @@ def load():
         "vsa_pool_qk": [P, P, P, P, vsa_shape, P],
         "vsa_flatten_pool_qk": [P, P, P, P, P, P, vsa_shape, P],
         "vsa_block_mask": [P, P, vsa_shape, vsa_mask_params, P, P, I64, P, P, S, P],
+        "vsa_block_mask_topk": [P, P, vsa_shape, ctypes.c_int32, vsa_mask_params, P, P, I64, P,
+                                P, S, P],
+        "vsa_sta_mask": [vsa_shape, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P, I64,
+                         P, P],
         "vsa_sparse_attn_fwd": [P, P, P, P, P, vsa_shape, F, P, P, P, S, P],
         "vsa_sparse_attn_fwd_noalloc": [P, P, P, P, P, vsa_shape, F, P, P, P],
         "vsa_device_status": [P],

@@ -41,6 +41,7 @@ constexpr int kLdK = kKS + kPad;
 constexpr int kCand = 256;    // per-warp candidate list capacity
 constexpr int kBins = 64;     // 1/8-octave probability bins (8 octaves below the max)
 constexpr int kMaxWords = 256;  // kept-bit words per row held in SMEM (Nb <= 8192)
+constexpr int kOctaves = 256;   // fp32 exponent bins of the static-ratio selection
 constexpr int kMaxGrid = 160; // persistent score CTAs
 
 struct MaskArgs {
@@ -57,6 +58,7 @@ struct MaskArgs {
   int words;
   int32_t *counts;   // [BH*Nb]
   int64_t items, tiles_per_head;
+  int k;             // static-ratio selection: blocks kept per row (0: top-p)
 };
 
 __device__ __forceinline__ void dmma(double (&c)[2], double a, double b) {
@@ -200,6 +202,40 @@ __device__ void cut_by_bisection(int Nb, const float *ebuf, uint32_t kmax, doubl
 //   3. with at most 32 entries: a warp bitonic sort on (probability desc,
 //      index asc) and an fp64 prefix scan mark the kept ones.  Otherwise (or
 //      if the fp32 histogram misled step 2) the bisection path decides.
+// Shared end of both selections: OR in the STA window, write the kept-bit
+// row and its count.  wbits holds the selection's bits (warp-synchronised).
+__device__ void finish_row(const MaskArgs &a, int64_t grow, int r, uint32_t *wbits) {
+  const int lane = threadIdx.x & 31;
+  const int Nb = a.Nb;
+  if (a.use_sta) {
+    // the window: at most (2rt+1)(2rh+1)(2rw+1) blocks around the row's own
+    const int hw = a.Hb * a.Wb;
+    const int tr = r / hw, yr = (r / a.Wb) % a.Hb, xr = r % a.Wb;
+    const int nt = 2 * a.rt + 1, ny = 2 * a.rh + 1, nx = 2 * a.rw + 1;
+    const int T = Nb / hw;
+    for (int i = lane; i < nt * ny * nx; i += 32) {
+      const int t = tr - a.rt + i / (ny * nx);
+      const int y = yr - a.rh + (i / nx) % ny;
+      const int x = xr - a.rw + i % nx;
+      if (t >= 0 && t < T && y >= 0 && y < a.Hb && x >= 0 && x < a.Wb) {
+        const int c = (t * a.Hb + y) * a.Wb + x;
+        atomicOr(&wbits[c >> 5], 1u << (c & 31));
+      }
+    }
+    __syncwarp();
+  }
+  uint32_t *out = a.bits + grow * a.words;
+  int count = 0;
+  for (int w = lane; w < a.words; w += 32) {
+    const uint32_t word = wbits[w];
+    out[w] = word;
+    count += __popc(word);
+  }
+  count = warp_sum_i(count);
+  if (lane == 0) a.counts[grow] = count;
+  __syncwarp();
+}
+
 __device__ void select_row(const MaskArgs &a, int64_t grow, int r, const float *slab_row,
                            const double *tmax_row, float *ebuf, uint32_t *cand_key,
                            int32_t *cand_idx, float *tscale, int *hcnt, float *hmass,
@@ -378,33 +414,7 @@ __device__ void select_row(const MaskArgs &a, int64_t grow, int r, const float *
     if (lane == 0) wbits[w] = word;
   }
   __syncwarp();
-  if (a.use_sta) {
-    // the window: at most (2rt+1)(2rh+1)(2rw+1) blocks around the row's own
-    const int hw = a.Hb * a.Wb;
-    const int tr = r / hw, yr = (r / a.Wb) % a.Hb, xr = r % a.Wb;
-    const int nt = 2 * a.rt + 1, ny = 2 * a.rh + 1, nx = 2 * a.rw + 1;
-    const int T = Nb / hw;
-    for (int i = lane; i < nt * ny * nx; i += 32) {
-      const int t = tr - a.rt + i / (ny * nx);
-      const int y = yr - a.rh + (i / nx) % ny;
-      const int x = xr - a.rw + i % nx;
-      if (t >= 0 && t < T && y >= 0 && y < a.Hb && x >= 0 && x < a.Wb) {
-        const int c = (t * a.Hb + y) * a.Wb + x;
-        atomicOr(&wbits[c >> 5], 1u << (c & 31));
-      }
-    }
-    __syncwarp();
-  }
-  uint32_t *out = a.bits + grow * a.words;
-  int count = 0;
-  for (int w = lane; w < a.words; w += 32) {
-    const uint32_t word = wbits[w];
-    out[w] = word;
-    count += __popc(word);
-  }
-  count = warp_sum_i(count);
-  if (lane == 0) a.counts[grow] = count;
-  __syncwarp();
+  finish_row(a, grow, r, wbits);
 }
 
 // Work unit = (batch-head, 64-row tile, 128-column tile), numbered row-tile
@@ -546,6 +556,149 @@ __global__ void __launch_bounds__(kThreads, 1) mask_scores_kernel(const MaskArgs
 }
 
 // One warp per row of the mask: selection and kept bits.
+// Static-ratio selection of one row (DynamicRad, "Dual-Mode Strategy",
+// Static-Ratio mode; reading: the k most probable blocks, equal probabilities
+// to the lower index, k >= Nb keeps the row).  The probabilities are positive
+// fp32 values, so their bit patterns order like the values: a histogram of
+// the exponent field finds the octave holding the k-th largest, a bisection
+// over that octave's 2^23 patterns (on its members, compacted when there are
+// at most kCand) finds the k-th largest pattern, and equal patterns at the cut
+// are taken in index order.
+__device__ void select_row_topk(const MaskArgs &a, int64_t grow, int r, const float *slab_row,
+                                const double *tmax_row, float *ebuf, uint32_t *cand_key,
+                                int32_t *cand_idx, float *tscale, int *hist, uint32_t *wbits) {
+  const int lane = threadIdx.x & 31;
+  const int Nb = a.Nb, k = a.k;
+  double M = -INFINITY;
+  for (int t = lane; t < a.ntiles; t += 32) M = fmax(M, tmax_row[t]);
+  M = warp_max(M);
+  for (int t = lane; t < a.ntiles; t += 32) tscale[t] = static_cast<float>(exp2(tmax_row[t] - M));
+  for (int b = lane; b < kOctaves; b += 32) hist[b] = 0;
+  __syncwarp();
+  const bool keep_all = k >= Nb;
+  for (int c = lane; c < Nb; c += 32) {
+    const float e = slab_row[c] * tscale[c / kCT];
+    ebuf[c] = e;
+    if (!keep_all) atomicAdd(&hist[__float_as_uint(e) >> 23], 1);
+  }
+  __syncwarp();
+
+  bool bits_done = false;
+  uint32_t vkey = 0;
+  int need_ties = 0;
+  if (!keep_all) {
+    // lane l owns exponent bins 255-8l .. 248-8l: lane order = descending values
+    int loc = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) loc += hist[kOctaves - 1 - 8 * lane - i];
+    int incl = loc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - loc, found = -1, above = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int b = kOctaves - 1 - 8 * lane - i;
+      if (found < 0 && run + hist[b] >= k) {
+        found = b;
+        above = run;
+      }
+      run += hist[b];
+    }
+    // the highest such bin (the lowest lane that found one); every entry is
+    // counted, so one exists as k < Nb
+    const uint32_t fm = __ballot_sync(0xFFFFFFFFu, found >= 0);
+    const int src = __ffs(fm) - 1;
+    found = __shfl_sync(0xFFFFFFFFu, found, src);
+    above = __shfl_sync(0xFFFFFFFFu, above, src);
+    const bool compact = hist[found] <= kCand;
+    // entries of higher octaves are kept whatever happens at the cut
+    int pos = 0;
+    for (int c0 = 0; c0 < Nb; c0 += 32) {
+      const int c = c0 + lane;
+      const int ex = c < Nb ? static_cast<int>(__float_as_uint(ebuf[c]) >> 23) : -1;
+      const uint32_t hi_word = __ballot_sync(0xFFFFFFFFu, ex > found);
+      if (lane == 0) wbits[c0 >> 5] = hi_word;
+      if (compact) {
+        const bool in = ex == found;
+        const uint32_t m = __ballot_sync(0xFFFFFFFFu, in);
+        if (in) {
+          const int p = pos + __popc(m & ((1u << lane) - 1u));
+          cand_key[p] = __float_as_uint(ebuf[c]);
+          cand_idx[p] = c;
+        }
+        pos += __popc(m);
+      }
+    }
+    __syncwarp();
+    // k-th largest pattern inside the octave: count(key >= hi) + above < k
+    // <= count(key >= lo) + above
+    uint32_t lo = static_cast<uint32_t>(found) << 23, hi = lo + (1u << 23);
+    int cnt_hi = 0;
+    while (hi - lo > 1) {
+      const uint32_t mid = lo + ((hi - lo) >> 1);
+      int cin = 0;
+      if (compact) {
+        for (int i = lane; i < pos; i += 32) cin += cand_key[i] >= mid && cand_key[i] < hi;
+      } else {
+        for (int c = lane; c < Nb; c += 32) {
+          const uint32_t key = __float_as_uint(ebuf[c]);
+          cin += key >= mid && key < hi;
+        }
+      }
+      cin = warp_sum_i(cin);
+      if (above + cnt_hi + cin >= k) {
+        lo = mid;
+      } else {
+        cnt_hi += cin;
+        hi = mid;
+      }
+    }
+    vkey = lo;
+    need_ties = k - (above + cnt_hi);   // >= 1 entries equal to vkey
+    if (compact) {
+      // members in ascending index order: patterns above vkey, then the
+      // first need_ties equal to it
+      int ties_seen = 0;
+      for (int i0 = 0; i0 < pos; i0 += 32) {
+        const int i = i0 + lane;
+        const uint32_t key = i < pos ? cand_key[i] : 0u;
+        bool kept = i < pos && key > vkey;
+        const bool tie = i < pos && key == vkey;
+        const uint32_t tm = __ballot_sync(0xFFFFFFFFu, tie);
+        if (tie && ties_seen + __popc(tm & ((1u << lane) - 1u)) < need_ties) kept = true;
+        ties_seen += __popc(tm);
+        if (kept) atomicOr(&wbits[cand_idx[i] >> 5], 1u << (cand_idx[i] & 31));
+      }
+      bits_done = true;
+    }
+  }
+  if (!bits_done) {
+    int ties_seen = 0;
+    for (int w = 0; w < a.words; ++w) {
+      const int c = w * 32 + lane;
+      const bool valid = c < Nb;
+      const uint32_t key = valid ? __float_as_uint(ebuf[c]) : 0u;
+      bool kept;
+      if (keep_all) {
+        kept = valid;
+      } else {
+        kept = valid && key > vkey;
+        const bool tie = valid && key == vkey;
+        const uint32_t tm = __ballot_sync(0xFFFFFFFFu, tie);
+        if (tie && ties_seen + __popc(tm & ((1u << lane) - 1u)) < need_ties) kept = true;
+        ties_seen += __popc(tm);
+      }
+      const uint32_t word = __ballot_sync(0xFFFFFFFFu, kept);
+      if (lane == 0) wbits[w] = word;
+    }
+  }
+  __syncwarp();
+  finish_row(a, grow, r, wbits);
+}
+
 __global__ void __launch_bounds__(kThreads) mask_select_kernel(const MaskArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int warp = threadIdx.x >> 5;
@@ -565,6 +718,30 @@ __global__ void __launch_bounds__(kThreads) mask_select_kernel(const MaskArgs a)
        g += static_cast<int64_t>(gridDim.x) * kWarps) {
     select_row(a, g, static_cast<int>(g % a.Nb), a.slab + g * a.ld_slab, a.tmax + g * a.ntiles,
                ebuf, cand_key, cand_idx, tscale, hcnt, hmass, wbits);
+  }
+}
+
+// Per-warp SMEM of the static-ratio selection (all 4-byte fields).
+__host__ __device__ inline size_t topk_warp_bytes(int Nb, int ntiles) {
+  return (static_cast<size_t>(Nb + 2 * kCand + ntiles + kOctaves + kMaxWords) * 4 + 15) &
+         ~static_cast<size_t>(15);
+}
+
+__global__ void __launch_bounds__(kThreads) mask_select_topk_kernel(const MaskArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int warp = threadIdx.x >> 5;
+  unsigned char *wbase = smem_raw + warp * topk_warp_bytes(a.Nb, a.ntiles);
+  float *ebuf = reinterpret_cast<float *>(wbase);
+  uint32_t *cand_key = reinterpret_cast<uint32_t *>(ebuf + a.Nb);
+  int32_t *cand_idx = reinterpret_cast<int32_t *>(cand_key + kCand);
+  float *tscale = reinterpret_cast<float *>(cand_idx + kCand);
+  int *hist = reinterpret_cast<int *>(tscale + a.ntiles);
+  uint32_t *wbits = reinterpret_cast<uint32_t *>(hist + kOctaves);
+  const int64_t rows = a.BH * a.Nb;
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * kWarps + warp; g < rows;
+       g += static_cast<int64_t>(gridDim.x) * kWarps) {
+    select_row_topk(a, g, static_cast<int>(g % a.Nb), a.slab + g * a.ld_slab,
+                    a.tmax + g * a.ntiles, ebuf, cand_key, cand_idx, tscale, hist, wbits);
   }
 }
 
@@ -628,7 +805,7 @@ __global__ void __launch_bounds__(256) expand_bits_kernel(const uint32_t *__rest
 struct MaskLayout {
   int ld_slab, ntiles, words, grid;
   size_t slab_off, tmax_off, bits_off, counts_off, total;
-  size_t smem, smem_a, smem_b;
+  size_t smem, smem_a, smem_b, smem_k;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -653,7 +830,9 @@ MaskLayout mask_layout(const Geometry &g, int grid) {
   L.smem_b = static_cast<size_t>(kWarps) *
              (static_cast<size_t>(g.Nb) * 4 + kCand * 8 + L.ntiles * 8 + 16 + kBins * 8 +
               kMaxWords * 4);
+  L.smem_k = static_cast<size_t>(kWarps) * topk_warp_bytes(static_cast<int>(g.Nb), L.ntiles);
   L.smem = L.smem_a > L.smem_b ? L.smem_a : L.smem_b;
+  if (L.smem_k > L.smem) L.smem = L.smem_k;
   if (L.words > kMaxWords) L.smem = ~static_cast<size_t>(0) >> 1;  // reported as unsupported
   return L;
 }
@@ -665,8 +844,9 @@ size_t block_mask_workspace_bytes(const Geometry &g) { return mask_layout(g, kMa
 size_t block_mask_smem_bytes(const Geometry &g) { return mask_layout(g, kMaxGrid).smem; }
 
 cudaError_t launch_block_mask(const double *qp, const double *kp, const Geometry &g,
-                              const vsa_mask_params &p, int64_t *row_ptr, int32_t *col_idx,
-                              int32_t *kept_count, void *ws, unsigned *err, cudaStream_t st) {
+                              const vsa_mask_params &p, int topk, int64_t *row_ptr,
+                              int32_t *col_idx, int32_t *kept_count, void *ws, unsigned *err,
+                              cudaStream_t st) {
   (void)err;
   const int64_t rows = g.BH * g.Nb;
   if (rows == 0) {
@@ -692,18 +872,27 @@ cudaError_t launch_block_mask(const double *qp, const double *kp, const Geometry
   a.words = L.words;
   a.counts = kept_count ? kept_count : reinterpret_cast<int32_t *>(w + L.counts_off);
   a.items = items; a.tiles_per_head = tiles_per_head;
+  a.k = topk;
   cudaError_t e = cudaFuncSetAttribute(mask_scores_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(L.smem_a));
   if (e != cudaSuccess) return e;
   mask_scores_kernel<<<grid, kThreads, L.smem_a, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if ((e = cudaFuncSetAttribute(mask_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(L.smem_b))) != cudaSuccess)
-    return e;
   const int64_t sel_blocks = (rows + kWarps - 1) / kWarps;
   const int sel_grid = static_cast<int>(sel_blocks < 64LL * num_sms() ? sel_blocks : 64LL * num_sms());
-  mask_select_kernel<<<sel_grid, kThreads, L.smem_b, st>>>(a);
+  if (topk > 0) {
+    if ((e = cudaFuncSetAttribute(mask_select_topk_kernel,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(L.smem_k))) != cudaSuccess)
+      return e;
+    mask_select_topk_kernel<<<sel_grid, kThreads, L.smem_k, st>>>(a);
+  } else {
+    if ((e = cudaFuncSetAttribute(mask_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(L.smem_b))) != cudaSuccess)
+      return e;
+    mask_select_kernel<<<sel_grid, kThreads, L.smem_b, st>>>(a);
+  }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   scan_counts_kernel<<<1, 1024, 0, st>>>(a.counts, rows, row_ptr);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -210,9 +210,74 @@ vsa_status vsa_block_mask(const double *qp, const double *kp, vsa_shape s, vsa_m
   cudaError_t e;
   unsigned *err = device_error_word(&e);
   if (!err) return cuda_fail(e, "device error word");
-  e = vsa::launch_block_mask(qp, kp, g, p, row_ptr, col_idx, kept_count, workspace, err,
+  e = vsa::launch_block_mask(qp, kp, g, p, 0, row_ptr, col_idx, kept_count, workspace, err,
                              static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? VSA_OK : cuda_fail(e, "block mask launch");
+}
+
+vsa_status vsa_block_mask_topk(const double *qp, const double *kp, vsa_shape s, int32_t k,
+                               vsa_mask_params p, int64_t *row_ptr, int32_t *col_idx,
+                               int64_t col_capacity, int32_t *kept_count, void *workspace,
+                               size_t workspace_bytes, void *stream) {
+  vsa_status st = check_shape(s);
+  if (st != VSA_OK) return st;
+  if (k < 1) return fail(VSA_ERR_INVALID_ARG, "k=%d: at least one block per row", k);
+  if (p.use_sta && (p.sta_t < 0 || p.sta_h < 0 || p.sta_w < 0))
+    return fail(VSA_ERR_INVALID_ARG, "negative STA radius (%d, %d, %d)", p.sta_t, p.sta_h, p.sta_w);
+  if (!row_ptr) return fail(VSA_ERR_INVALID_ARG, "null row_ptr");
+  const vsa::Geometry g = vsa::geometry(s);
+  const int64_t need = g.BH * g.Nb * g.Nb;
+  if (col_capacity < need)
+    return fail(VSA_ERR_CAPACITY, "col_capacity %lld < B*heads*Nb*Nb = %lld",
+                static_cast<long long>(col_capacity), static_cast<long long>(need));
+  if (empty(s)) {
+    cudaError_t e = cudaMemsetAsync(row_ptr, 0, sizeof(int64_t), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? VSA_OK : cuda_fail(e, "row_ptr reset");
+  }
+  if (!qp || !kp || !col_idx || !workspace)
+    return fail(VSA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(qp) || !aligned16(kp) || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      (reinterpret_cast<uintptr_t>(row_ptr) & 7u) || (reinterpret_cast<uintptr_t>(col_idx) & 3u) ||
+      (kept_count && (reinterpret_cast<uintptr_t>(kept_count) & 3u)))
+    return fail(VSA_ERR_UNSUPPORTED, "misaligned pointer (tensors 16 B, workspace 256 B)");
+  const size_t ws = vsa::block_mask_workspace_bytes(g);
+  if (workspace_bytes < ws)
+    return fail(VSA_ERR_CAPACITY, "block mask workspace %zu < %zu bytes", workspace_bytes, ws);
+  if (vsa::block_mask_smem_bytes(g) > kMaxSmem)
+    return fail(VSA_ERR_UNSUPPORTED, "Nb=%lld blocks per head exceeds the mask kernel's shared memory",
+                static_cast<long long>(g.Nb));
+  cudaError_t e;
+  unsigned *err = device_error_word(&e);
+  if (!err) return cuda_fail(e, "device error word");
+  e = vsa::launch_block_mask(qp, kp, g, p, k, row_ptr, col_idx, kept_count, workspace, err,
+                             static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? VSA_OK : cuda_fail(e, "static-ratio mask launch");
+}
+
+vsa_status vsa_sta_mask(vsa_shape s, int32_t sta_t, int32_t sta_h, int32_t sta_w,
+                        int64_t *row_ptr, int32_t *col_idx, int64_t col_capacity,
+                        int32_t *kept_count, void *stream) {
+  vsa_status st = check_shape(s);
+  if (st != VSA_OK) return st;
+  if (sta_t < 0 || sta_h < 0 || sta_w < 0)
+    return fail(VSA_ERR_INVALID_ARG, "negative STA radius (%d, %d, %d)", sta_t, sta_h, sta_w);
+  if (!row_ptr) return fail(VSA_ERR_INVALID_ARG, "null row_ptr");
+  const vsa::Geometry g = vsa::geometry(s);
+  const int64_t need = vsa::sta_mask_nnz(g, sta_t, sta_h, sta_w);
+  if (col_capacity < need)
+    return fail(VSA_ERR_CAPACITY, "col_capacity %lld < the window's %lld entries",
+                static_cast<long long>(col_capacity), static_cast<long long>(need));
+  if (empty(s)) {
+    cudaError_t e = cudaMemsetAsync(row_ptr, 0, sizeof(int64_t), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? VSA_OK : cuda_fail(e, "row_ptr reset");
+  }
+  if (!col_idx) return fail(VSA_ERR_INVALID_ARG, "null col_idx");
+  if ((reinterpret_cast<uintptr_t>(row_ptr) & 7u) || (reinterpret_cast<uintptr_t>(col_idx) & 3u) ||
+      (kept_count && (reinterpret_cast<uintptr_t>(kept_count) & 3u)))
+    return fail(VSA_ERR_UNSUPPORTED, "misaligned pointer");
+  cudaError_t e = vsa::launch_sta_mask(g, sta_t, sta_h, sta_w, row_ptr, col_idx, kept_count,
+                                       static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? VSA_OK : cuda_fail(e, "STA mask launch");
 }
 
 size_t vsa_sparse_attn_workspace_size(vsa_shape s) {

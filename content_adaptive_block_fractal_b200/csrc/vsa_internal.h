@@ -39,9 +39,16 @@ cudaError_t launch_flatten_pool_qk(const void *q, const void *k, void *qf, void 
 
 // Block mask: workspace carve-up and launch.
 size_t block_mask_workspace_bytes(const Geometry &g);
+// topk > 0 selects the static-ratio rule (k blocks per row), 0 the top-p rule.
 cudaError_t launch_block_mask(const double *qp, const double *kp, const Geometry &g,
-                              const vsa_mask_params &p, int64_t *row_ptr, int32_t *col_idx,
-                              int32_t *kept_count, void *ws, unsigned *err, cudaStream_t st);
+                              const vsa_mask_params &p, int topk, int64_t *row_ptr,
+                              int32_t *col_idx, int32_t *kept_count, void *ws, unsigned *err,
+                              cudaStream_t st);
+
+// STA window alone: closed-form CSR, no workspace.
+int64_t sta_mask_nnz(const Geometry &g, int rt, int rh, int rw);
+cudaError_t launch_sta_mask(const Geometry &g, int rt, int rh, int rw, int64_t *row_ptr,
+                            int32_t *col_idx, int32_t *kept_count, cudaStream_t st);
 
 // Sparse attention: workspace carve-up and launch.
 size_t sparse_attn_workspace_bytes(const Geometry &g);

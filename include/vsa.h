@@ -125,6 +125,36 @@ vsa_status vsa_block_mask(const double *qp, const double *kp, vsa_shape s,
                           int64_t col_capacity, int32_t *kept_count,
                           void *workspace, size_t workspace_bytes, void *stream);
 
+/* Static-ratio block mask (DynamicRad, arXiv 2604.20470 summary, section 2,
+ * "Dual-Mode Strategy", Static-Ratio mode: every row keeps a fixed share of
+ * its blocks).  The page does not say which blocks; this call keeps each
+ * row's k blocks of highest reduced-attention probability, ordered as in
+ * vsa_block_mask (probability descending, equal probabilities to the lower
+ * block index), then ORs in the STA window when p.use_sta is set (p.thr is
+ * ignored).  k >= Nb keeps every block; k < 1 is VSA_ERR_INVALID_ARG.
+ * Outputs, capacity, alignment and workspace (vsa_block_mask_workspace_size)
+ * are those of vsa_block_mask.  Probabilities are fp32-accurate, so only rows
+ * whose k-th and (k+1)-th probabilities lie within a relative 1e-5 (or below
+ * 2^-120 of the row maximum) can differ from exact arithmetic. */
+vsa_status vsa_block_mask_topk(const double *qp, const double *kp, vsa_shape s, int32_t k,
+                               vsa_mask_params p, int64_t *row_ptr, int32_t *col_idx,
+                               int64_t col_capacity, int32_t *kept_count, void *workspace,
+                               size_t workspace_bytes, void *stream);
+
+/* The STA window as the whole mask (NABLA, Methodology item 3, the sliding-
+ * tile component M_STA alone; equally a static local-window mask): query block
+ * (t, y, x) keeps the key blocks within Chebyshev radii (sta_t, sta_h, sta_w)
+ * in (frame, patch row, patch column), clipped at the grid edges, ascending;
+ * the same for every (b, h).  Needs no pooled tensors and no workspace.
+ *   row_ptr : device int64 [B*heads*Nb + 1];  kept_count : optional int32.
+ *   col_idx : device int32, col_capacity >= the window's total entry count
+ *             (B*heads * sum_t w_t * sum_y w_y * sum_x w_x, w the clipped
+ *             widths), else VSA_ERR_CAPACITY.  Negative radii are
+ *             VSA_ERR_INVALID_ARG. */
+vsa_status vsa_sta_mask(vsa_shape s, int32_t sta_t, int32_t sta_h, int32_t sta_w,
+                        int64_t *row_ptr, int32_t *col_idx, int64_t col_capacity,
+                        int32_t *kept_count, void *stream);
+
 /* 5. Block-sparse attention forward (NABLA, Methodology item 2, "expansion":
  * the block mask decides which 64 x 64 tiles are computed; Sparse VideoGen2
  * section 2C: dense loads of contiguous query blocks, sparse loads of K/V).

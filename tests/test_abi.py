@@ -6,6 +6,7 @@ import re
 
 import pytest
 
+import content_adaptive_block_fractal_b200 as vsa
 from content_adaptive_block_fractal_b200 import _lib, Shape, MaskParams
 
 HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "vsa.h")
@@ -89,4 +90,26 @@ def test_flatten_pool_validation():
     assert call(qf=1 * MB + 4096) == 1              # output inside an input
     assert call(kf=3 * MB + 65536) == 1             # two outputs overlap
     assert call(qp=4 * MB + 128 * 1024) == 1        # pooled output inside kf
+    assert len(L.vsa_last_error()) > 0
+
+
+def test_static_ratio_and_sta_validation():
+    L = _lib.load()
+    s = Shape(1, 2, 4, 16, 16, 64)              # Nb = 16 per head, 32 rows
+    P = ctypes.c_void_p
+    def topk(k, cap=2 * 16 * 16, ws=1 << 30, params=MaskParams(0.0, True)):
+        return L.vsa_block_mask_topk(P(1 << 12), P(1 << 16), s.c(), k, params.c(), P(1 << 20),
+                                     P(1 << 24), cap, None, P(1 << 28), ws, None)
+    assert topk(0) == 1                                     # k < 1
+    assert topk(-3) == 1
+    assert topk(4, params=MaskParams(0.0, True, (1, -1, 0))) == 1
+    assert topk(4, cap=2 * 16 * 16 - 1) == 3                # CSR capacity
+    assert topk(4, ws=16) == 3                              # workspace
+    def sta(r=(1, 1, 1), cap=1 << 20):
+        return L.vsa_sta_mask(s.c(), r[0], r[1], r[2], P(1 << 20), P(1 << 24), cap, None, None)
+    assert sta((-1, 0, 0)) == 1
+    need = vsa.sta_mask_nnz(s, (1, 1, 1))
+    # 2 heads x (sum of clipped widths: 4 frames -> 2+3+3+2, 2 patch rows -> 2+2, 2 cols -> 2+2)
+    assert need == 2 * 10 * 4 * 4
+    assert sta(cap=need - 1) == 3
     assert len(L.vsa_last_error()) > 0
