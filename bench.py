@@ -317,22 +317,43 @@ def run_sweep(args):
                       functools.partial(vsa.block_mask_topk, layer.qp, layer.kp, shape, k10,
                                         vsa.MaskParams(0.0, sta, wl0.sta), out=layer.csr,
                                         workspace=layer.ws_mask)))
+    cases = [c + (None,) for c in cases]
     cases.append(("STA window alone (+-1)", wl0,
-                  functools.partial(vsa.sta_mask, shape, wl0.sta, out=sta_csr)))
-    for label, wl, make_mask in cases:
+                  functools.partial(vsa.sta_mask, shape, wl0.sta, out=sta_csr), None))
+    # query subsets (HSA-style active blocks): a seeded 25% of the query blocks
+    rows_all = shape.B * shape.heads * shape.Nb
+    active = torch.as_tensor(np.sort(np.random.default_rng(7).choice(
+        rows_all, rows_all // 4, replace=False)), dtype=torch.int32, device=qd.device)
+    cases.append(("query subset 25% of blocks, every key block (full context)", points[0],
+                  functools.partial(vsa.block_mask, layer.qp, layer.kp, shape,
+                                    vsa.MaskParams(0.0, False), out=layer.csr,
+                                    workspace=layer.ws_mask), active))
+    cases.append(("query subset 25% of blocks, top-p thr=0.1 + STA", wl0,
+                  functools.partial(vsa.block_mask, layer.qp, layer.kp, shape,
+                                    vsa.MaskParams(0.1, True, wl0.sta), out=layer.csr,
+                                    workspace=layer.ws_mask), active))
+    for label, wl, make_mask, qblocks in cases:
 
         def step(record=False):
             if record: ev[0].record(stream)
             make_mask()
             if record: ev[1].record(stream)
-            vsa.sparse_attn_fwd(qf, kf, vf, layer.csr.row_ptr, layer.csr.col_idx, shape, 0.0,
-                                out=(layer.o, layer.lse), workspace=layer.ws_attn)
+            if qblocks is None:
+                vsa.sparse_attn_fwd(qf, kf, vf, layer.csr.row_ptr, layer.csr.col_idx, shape,
+                                    0.0, out=(layer.o, layer.lse), workspace=layer.ws_attn)
+            else:
+                vsa.sparse_attn_fwd_rows(qf, kf, vf, layer.csr.row_ptr, layer.csr.col_idx,
+                                         shape, qblocks, 0.0, out=(layer.o, layer.lse),
+                                         workspace=layer.ws_attn)
             if record: ev[2].record(stream)
 
         for _ in range(max(args.warmup, 3)):
             step()
         vsa.device_status()
-        kept = int(layer.csr.row_ptr[-1].item())
+        if qblocks is None:
+            kept = int(layer.csr.row_ptr[-1].item())
+        else:   # tiles of the listed query blocks only
+            kept = int(layer.csr.kept_count[qblocks.long()].sum().item())
         t_mask = t_attn = 0.0
         with ClockSampler(0) as clk:
             for _ in range(steps):
@@ -352,6 +373,7 @@ def run_sweep(args):
                        "d": shape.d, "grid": [shape.T, shape.H, shape.W], "seed": wl.seed,
                        "data": "synthetic"},
             "kept_tiles": kept, "kept_fraction": kept / (shape.B * shape.heads * shape.Nb ** 2),
+            "query_blocks": int(qblocks.numel()) if qblocks is not None else rows_all,
             "mask_ms": t_mask, "sparse_attn_ms": t_attn, "kept_tile_tflops": tf,
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peak_tf, "frac": tf / peak_tf,
                          "peak_source": f"{peak_src} bf16 sustained"},

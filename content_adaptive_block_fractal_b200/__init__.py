@@ -21,7 +21,7 @@ from ._lib import VsaError, vsa_mask_params, vsa_shape
 __all__ = ["Shape", "MaskParams", "VsaError", "fractal_flatten", "fractal_unflatten",
            "flatten_pool_qk",
            "pool_qk", "block_mask", "block_mask_topk", "sta_mask", "sta_mask_nnz",
-           "block_mask_workspace_size", "sparse_attn_fwd",
+           "block_mask_workspace_size", "sparse_attn_fwd", "sparse_attn_fwd_rows",
            "sparse_attn_workspace_size", "attention_layer", "device_status", "version",
            "Csr"]
 
@@ -215,6 +215,25 @@ def sparse_attn_fwd(qf, kf, vf, row_ptr, col_idx, shape: Shape, scale: float = 0
     _lib.check(_lib.load().vsa_sparse_attn_fwd(
         _ptr(qf), _ptr(kf), _ptr(vf), _ptr(row_ptr), _ptr(col_idx), shape.c(), float(scale),
         _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return o, lse
+
+
+def sparse_attn_fwd_rows(qf, kf, vf, row_ptr, col_idx, shape: Shape, qblocks: torch.Tensor,
+                         scale: float = 0.0, out=None, workspace=None, stream=None):
+    """Attention for the listed query blocks only (int32 global block rows,
+    strictly ascending); other rows of `out` are left as they are."""
+    if out is None:
+        out = (torch.zeros_like(qf),
+               torch.full((shape.B, shape.heads, shape.N), float("nan"), dtype=torch.float32,
+                          device=qf.device))
+    o, lse = out
+    if workspace is None:
+        workspace = _workspace(sparse_attn_workspace_size(shape), qf.device)
+    qb = qblocks.to(device=qf.device, dtype=torch.int32).contiguous()
+    _lib.check(_lib.load().vsa_sparse_attn_fwd_rows(
+        _ptr(qf), _ptr(kf), _ptr(vf), _ptr(row_ptr), _ptr(col_idx), shape.c(), float(scale),
+        _ptr(qb) if qb.numel() else ctypes_void(0), qb.numel(), _ptr(o), _ptr(lse),
+        _ptr(workspace), workspace.numel(), _stream(stream)))
     return o, lse
 
 

@@ -97,7 +97,11 @@ struct AttnArgs {
   const int32_t *order;   // longest-first work items
   int *counter;           // next position in `order`
   unsigned *err;
-  int64_t items;          // total work items
+  int64_t items;          // total work items (when n_items is null)
+  const int *n_items;     // query-subset mode: item count written by the planner;
+                          // order[] then holds the list index of each item's lead
+  const int32_t *qblocks; // query-subset mode: the listed global query-block rows
+  int64_t n_qblocks;
   int64_t N;              // tokens per head
   int Nb, T, HW;          // blocks per head, frames, patches per frame
   int pairs_per_head;
@@ -105,9 +109,20 @@ struct AttnArgs {
   float lse_scale;        // ln(2)
 };
 
-// item -> (bh, r0, r1): the same patch in frames 2t and 2t+1.
+// item -> (bh, r0, r1): the same patch in frames 2t and 2t+1.  In the
+// query-subset mode an item is the list index i of its lead block; the next
+// listed block joins it when it belongs to the same head and comes after it
+// (the planner emits only leads, in range).
 __device__ __forceinline__ void decode_item(int item, const AttnArgs &a, int &bh, int &r0,
                                             int &r1) {
+  if (a.n_items) {
+    const int32_t g0 = a.qblocks[item];
+    bh = g0 / a.Nb;
+    r0 = g0 % a.Nb;
+    const int32_t g1 = item + 1 < a.n_qblocks ? a.qblocks[item + 1] : -1;
+    r1 = (g1 > g0 && g1 / a.Nb == bh) ? g1 % a.Nb : -1;
+    return;
+  }
   bh = item / a.pairs_per_head;
   const int p = item % a.pairs_per_head;
   const int t2 = p / a.HW, sp = p % a.HW;
@@ -223,6 +238,7 @@ __global__ void __maxnreg__(168)
       tma_prefetch_desc(&tk);
       tma_prefetch_desc(&tv);
     }
+    const int64_t n_items = a.n_items ? static_cast<int64_t>(*a.n_items) : a.items;
     int m = 0;               // next step whose record and K blocks go out
     uint32_t q_phase = 0;
     bool ok = true;
@@ -254,7 +270,7 @@ __global__ void __maxnreg__(168)
       int item = 0;
       if (lane == 0) item = atomicAdd(a.counter, 1);
       item = __shfl_sync(0xFFFFFFFFu, item, 0);
-      if (item >= a.items) {
+      if (item >= n_items) {
         // one end record per softmax group (they take alternate steps), then
         // the V blocks still owed
         StepMeta r{};
@@ -284,8 +300,9 @@ __global__ void __maxnreg__(168)
       const int64_t b0 = a.row_ptr[g0], n0 = a.row_ptr[g0 + 1] - b0;
       int64_t b1 = 0, n1 = 0;
       if (r1 >= 0) {
-        b1 = a.row_ptr[g0 + a.HW];
-        n1 = a.row_ptr[g0 + a.HW + 1] - b1;
+        const int64_t g1 = static_cast<int64_t>(bh) * a.Nb + r1;
+        b1 = a.row_ptr[g1];
+        n1 = a.row_ptr[g1 + 1] - b1;
       }
       int64_t i0 = 0, i1 = 0, w0 = -kListWin, w1 = -kListWin;
       StepMeta pend{};
@@ -684,6 +701,33 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int64_t *__restrict__ 
 }
 
 // Fallback order (no per-head sort) for very large heads.
+// Query-subset planner: the listed query blocks (global rows, strictly
+// ascending) are paired in list order within each head -- the block of even
+// rank within its head leads an item, the next one joins it -- so every item
+// but a head's last fills the 128-row tile.  An entry out of range or out of
+// order is recorded in the error word and not emitted (the set then computed
+// is unspecified, every access stays in bounds).  *n_items starts at zero.
+__global__ void plan_rows_kernel(const int32_t *__restrict__ qblocks, int64_t n, int64_t rows,
+                                 int Nb, int32_t *order, int *n_items, unsigned *err) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const int32_t g = qblocks[i];
+  if (g < 0 || g >= rows || (i > 0 && qblocks[i - 1] >= g)) {
+    atomicOr(err, kErrBadIndex);
+    return;
+  }
+  // rank of the entry within its head: index minus the head's first entry
+  const int32_t head0 = (g / Nb) * Nb;
+  int64_t lo = 0, hi = n;
+  while (lo < hi) {
+    const int64_t mid = (lo + hi) >> 1;
+    if (qblocks[mid] < head0) lo = mid + 1; else hi = mid;
+  }
+  if ((i - lo) & 1) return;        // the second block of its item
+  const int pos = atomicAdd(n_items, 1);
+  order[pos] = static_cast<int32_t>(i);
+}
+
 __global__ void identity_order_kernel(int32_t *order, int64_t n, int *counter) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i == 0) *counter = 0;
@@ -740,7 +784,7 @@ AttnLayout attn_layout(const Geometry &g) {
   L.HW = g.Hb * g.Wb;
   L.pairs = ((g.T + 1) / 2) * L.HW;
   L.items = g.BH * L.pairs;
-  L.counter_off = 0;
+  L.counter_off = 0;      // scheduler counter, then the query-subset item count
   L.order_off = 256;
   L.total = L.order_off + ((static_cast<size_t>(L.items) * 4 + 255) & ~static_cast<size_t>(255));
   return L;
@@ -753,9 +797,10 @@ size_t sparse_attn_workspace_bytes(const Geometry &g) { return attn_layout(g).to
 cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
                                const int64_t *row_ptr, const int32_t *col_idx,
                                const Geometry &g, float scale, void *o, float *lse, void *ws,
-                               unsigned *err, cudaStream_t st, const char **why) {
+                               unsigned *err, cudaStream_t st, const char **why,
+                               const int32_t *qblocks, int64_t n_qblocks) {
   const AttnLayout L = attn_layout(g);
-  if (L.items == 0) return cudaSuccess;
+  if (L.items == 0 || (qblocks && n_qblocks == 0)) return cudaSuccess;
   if (L.items > 0x7FFFFFFF || g.BH * g.N > 0x7FFFFFFF) {
     *why = "sparse attention: too many tokens for 32-bit TMA row coordinates";
     return cudaErrorInvalidValue;
@@ -770,10 +815,15 @@ cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
   unsigned char *w = static_cast<unsigned char *>(ws);
   int *counter = reinterpret_cast<int *>(w + L.counter_off);
   int32_t *order = reinterpret_cast<int32_t *>(w + L.order_off);
+  int *n_items = counter + 1;
   int n2 = 1;
   while (n2 < L.pairs) n2 <<= 1;
   cudaError_t e;
-  if (n2 <= 4096) {
+  if (qblocks) {
+    if ((e = cudaMemsetAsync(counter, 0, 2 * sizeof(int), st)) != cudaSuccess) return e;
+    plan_rows_kernel<<<static_cast<int>((n_qblocks + 255) / 256), 256, 0, st>>>(
+        qblocks, n_qblocks, g.BH * g.Nb, static_cast<int>(g.Nb), order, n_items, err);
+  } else if (n2 <= 4096) {
     plan_kernel<<<static_cast<int>(g.BH), 1024, n2 * 8, st>>>(row_ptr, static_cast<int>(g.Nb),
                                                               g.T, L.HW, L.pairs, order, counter);
   } else {
@@ -787,11 +837,15 @@ cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
   a.o = static_cast<__nv_bfloat16 *>(o); a.lse = lse;
   a.order = order; a.counter = counter; a.err = err;
   a.items = L.items; a.N = g.N; a.Nb = static_cast<int>(g.Nb); a.T = g.T; a.HW = L.HW;
+  a.n_items = qblocks ? n_items : nullptr;
+  a.qblocks = qblocks;
+  a.n_qblocks = n_qblocks;
   a.pairs_per_head = L.pairs;
   a.c = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   a.lse_scale = 0.6931471805599453f;
   int grid = num_sms();
-  if (L.items < grid) grid = static_cast<int>(L.items);
+  const int64_t max_items = qblocks ? (n_qblocks < L.items ? n_qblocks : L.items) : L.items;
+  if (max_items < grid) grid = static_cast<int>(max_items);
   const void *fn = g.d == 128 ? reinterpret_cast<const void *>(sparse_attn_kernel<128>)
                               : reinterpret_cast<const void *>(sparse_attn_kernel<64>);
   const int smem = g.d == 128 ? Smem<128>::kAlloc : Smem<64>::kAlloc;

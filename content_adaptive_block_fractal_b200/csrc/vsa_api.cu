@@ -285,10 +285,44 @@ size_t vsa_sparse_attn_workspace_size(vsa_shape s) {
   return vsa::sparse_attn_workspace_bytes(vsa::geometry(s));
 }
 
+static vsa_status sparse_attn(const void *qf, const void *kf, const void *vf,
+                              const int64_t *row_ptr, const int32_t *col_idx, vsa_shape s,
+                              float scale, const int32_t *qblocks, int64_t n_qblocks, void *o,
+                              float *lse, void *workspace, size_t workspace_bytes, void *stream);
+
 vsa_status vsa_sparse_attn_fwd(const void *qf, const void *kf, const void *vf,
                                const int64_t *row_ptr, const int32_t *col_idx, vsa_shape s,
                                float scale, void *o, float *lse, void *workspace,
                                size_t workspace_bytes, void *stream) {
+  return sparse_attn(qf, kf, vf, row_ptr, col_idx, s, scale, nullptr, 0, o, lse, workspace,
+                     workspace_bytes, stream);
+}
+
+vsa_status vsa_sparse_attn_fwd_rows(const void *qf, const void *kf, const void *vf,
+                                    const int64_t *row_ptr, const int32_t *col_idx,
+                                    vsa_shape s, float scale, const int32_t *qblocks,
+                                    int64_t n_qblocks, void *o, float *lse, void *workspace,
+                                    size_t workspace_bytes, void *stream) {
+  vsa_status st = check_shape(s);
+  if (st != VSA_OK) return st;
+  if (n_qblocks < 0) return fail(VSA_ERR_INVALID_ARG, "negative query-block count");
+  const vsa::Geometry g = vsa::geometry(s);
+  if (n_qblocks > g.BH * g.Nb)
+    return fail(VSA_ERR_INVALID_ARG, "%lld query blocks listed, the shape has %lld",
+                static_cast<long long>(n_qblocks), static_cast<long long>(g.BH * g.Nb));
+  if (g.BH * g.Nb >= (1LL << 30))
+    return fail(VSA_ERR_UNSUPPORTED, "too many query blocks for the subset planner");
+  if (n_qblocks > 0 && (!qblocks || (reinterpret_cast<uintptr_t>(qblocks) & 3u)))
+    return fail(VSA_ERR_INVALID_ARG, "null or misaligned query-block list");
+  if (n_qblocks == 0) return VSA_OK;
+  return sparse_attn(qf, kf, vf, row_ptr, col_idx, s, scale, qblocks, n_qblocks, o, lse,
+                     workspace, workspace_bytes, stream);
+}
+
+static vsa_status sparse_attn(const void *qf, const void *kf, const void *vf,
+                              const int64_t *row_ptr, const int32_t *col_idx, vsa_shape s,
+                              float scale, const int32_t *qblocks, int64_t n_qblocks, void *o,
+                              float *lse, void *workspace, size_t workspace_bytes, void *stream) {
   vsa_status st = check_shape(s);
   if (st != VSA_OK) return st;
   if (empty(s)) return VSA_OK;
@@ -309,7 +343,7 @@ vsa_status vsa_sparse_attn_fwd(const void *qf, const void *kf, const void *vf,
   if (!err) return cuda_fail(e, "device error word");
   const char *why = nullptr;
   e = vsa::launch_sparse_attn(qf, kf, vf, row_ptr, col_idx, g, scale, o, lse, workspace, err,
-                              static_cast<cudaStream_t>(stream), &why);
+                              static_cast<cudaStream_t>(stream), &why, qblocks, n_qblocks);
   if (e != cudaSuccess)
     return why ? fail(e == cudaErrorInvalidValue ? VSA_ERR_UNSUPPORTED : VSA_ERR_CUDA, "%s", why)
                : cuda_fail(e, "sparse attention launch");

@@ -55,6 +55,7 @@ size_t sparse_attn_workspace_bytes(const Geometry &g);
 cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
                                const int64_t *row_ptr, const int32_t *col_idx,
                                const Geometry &g, float scale, void *o, float *lse, void *ws,
-                               unsigned *err, cudaStream_t st, const char **why);
+                               unsigned *err, cudaStream_t st, const char **why,
+                               const int32_t *qblocks = nullptr, int64_t n_qblocks = 0);
 
 }  // namespace vsa

@@ -176,6 +176,29 @@ vsa_status vsa_sparse_attn_fwd(const void *qf, const void *kf, const void *vf,
                                void *workspace, size_t workspace_bytes,
                                void *stream);
 
+/* Query-subset attention (HSA, arXiv 2605.06892 summary, section 2.2 "KV cache
+ * synchronisation": only the active tokens form queries, against the whole
+ * cached K and V, so the cost is O(|active| * N) instead of O(N^2)).  At block
+ * granularity: only the listed query blocks are computed, each exactly as
+ * vsa_sparse_attn_fwd computes it over its CSR key blocks (a CSR that keeps
+ * every block gives HSA's full-context attention); O and LSE rows of every
+ * other query block are left untouched.  A block with an active token is
+ * computed whole (all 64 of its rows).
+ * qblocks : device int32 [n_qblocks], global query-block rows
+ *           g = (b*heads + h)*Nb + r, strictly ascending.  Listed blocks share
+ *           128-row tensor-core tiles two by two in list order within a head.
+ *           An entry out of range or out of order is recorded in the device
+ *           error word (vsa_device_status reports "bad block index"); the set
+ *           of blocks then computed is unspecified, and every access stays in
+ *           bounds.
+ * Other arguments, layouts and the workspace are those of vsa_sparse_attn_fwd;
+ * n_qblocks = 0 does nothing. */
+vsa_status vsa_sparse_attn_fwd_rows(const void *qf, const void *kf, const void *vf,
+                                    const int64_t *row_ptr, const int32_t *col_idx,
+                                    vsa_shape s, float scale, const int32_t *qblocks,
+                                    int64_t n_qblocks, void *o, float *lse, void *workspace,
+                                    size_t workspace_bytes, void *stream);
+
 /* Block-sparse attention forward without a caller-provided workspace.
  * The paper has no counterpart to this call; it exists for callers that cannot
  * allocate device memory -- plugins whose host framework passes them only

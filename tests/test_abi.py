@@ -113,3 +113,18 @@ def test_static_ratio_and_sta_validation():
     assert need == 2 * 10 * 4 * 4
     assert sta(cap=need - 1) == 3
     assert len(L.vsa_last_error()) > 0
+
+
+def test_query_subset_validation():
+    L = _lib.load()
+    s = Shape(1, 2, 4, 16, 16, 64)              # 32 query blocks
+    P = ctypes.c_void_p
+    def call(qb, n):
+        return L.vsa_sparse_attn_fwd_rows(P(1 << 12), P(1 << 16), P(1 << 20), P(1 << 24),
+                                          P(1 << 26), s.c(), 0.0, qb, n, P(1 << 28), P(1 << 29),
+                                          P(1 << 30), 1 << 20, None)
+    assert call(P(1 << 12), -1) == 1
+    assert call(None, 4) == 1                   # null list
+    assert call(P((1 << 12) + 2), 4) == 1       # misaligned list
+    assert call(P(1 << 12), 33) == 1            # more entries than query blocks
+    assert call(None, 0) == 0                   # nothing to do

@@ -372,3 +372,25 @@ def test_sta_mask_closed_form_and_fixture():
     for ln in _lines("sta_window_T3_Hb3_Wb3_r1.txt"):
         r, cols = (part.strip() for part in ln.split(":"))
         assert np.nonzero(m[int(r)])[0].tolist() == [int(c) for c in cols.split()], ln
+
+
+# ---------------------------------------------------------------- f4 query subset
+def test_query_subset_rows_equal_full_rows_and_dense():
+    """Attention restricted to listed query blocks gives exactly those rows of
+    the full result; with every block kept they are rows of textbook dense
+    attention (torch SDPA in fp64)."""
+    wl = workloads.get("tiny")
+    q, k, v = workloads.make_qkv(wl)
+    qf, kf, vf = (oracle.flatten(x, wl.T, wl.H, wl.W) for x in (q, k, v))
+    rows = wl.B * wl.heads * wl.Nb
+    keep = np.ones((rows, wl.Nb), dtype=np.uint8)
+    rp, ci = oracle.mask_to_csr(keep)
+    o_all, l_all = oracle.sparse_attention(qf, kf, vf, rp, ci)
+    sub = np.array([0, 3, 5, 16, 17, 31])
+    o_sub, l_sub = oracle.sparse_attention(qf, kf, vf, rp, ci, qblocks=sub)
+    idx = (sub[:, None] * 64 + np.arange(64)[None, :]).reshape(-1)
+    np.testing.assert_array_equal(o_sub, o_all[idx])
+    np.testing.assert_array_equal(l_sub, l_all[idx])
+    qt, kt, vt = (oracle.to_bf16_tensor(x).double() for x in (qf, kf, vf))
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt)
+    np.testing.assert_allclose(o_sub, ref.reshape(-1, wl.d).numpy()[idx], rtol=0, atol=1e-12)
