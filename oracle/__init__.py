@@ -59,6 +59,12 @@ def lib():
         L.oracle_block_mask_topk.argtypes = [_P, _P, _I64, _I, _I, _I, _I, _I, _I, _I,
                                              _I, _I, _P, _I64, _P, _P]
         L.oracle_sta_mask.argtypes = [_I, _I, _I, _I, _I, _I, _P]
+        L.oracle_kmeans_assign.argtypes = [_P, _P, _I64, _I, _I, _P, _P]
+        L.oracle_kmeans_update.argtypes = [_P, _P, _I64, _I, _I, _P, _P]
+        L.oracle_cluster_order.argtypes = [_P, _I64, _I, _P, _P]
+        L.oracle_centroid_topp.argtypes = [_P, _P, _P, _I, _I, _I, _D, _P, _P]
+        L.oracle_cluster_attention.argtypes = [_P, _P, _P, _I64, _I, _P, _P, _P, _I, _D, _P,
+                                               _I64, _P, _P]
         L.oracle_sparse_attention.argtypes = [_P, _P, _P, _I64, _I64, _I, _P, _P,
                                               _D, _P, _I64, _P, _P]
     return _lib
@@ -225,6 +231,98 @@ def ambiguous_topk(diag: np.ndarray, eps: float = 1e-5, row_max=None) -> np.ndar
     if row_max is not None:
         amb |= (nxt >= 0) & (last < row_max * 2.0 ** -120)
     return amb
+
+
+# ---------------------------------------------------------------- semantic permutation
+def kmeans_init(x_u16: np.ndarray, C: int) -> np.ndarray:
+    """Initial centroids of one (batch, head): the tokens at floor(j*N/C)."""
+    x = to_f64(x_u16)
+    N = x.shape[0]
+    return x[(np.arange(C) * N) // C].astype(np.float32)
+
+
+def to_f64(x_u16: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> float64 (exact)."""
+    return (np.ascontiguousarray(x_u16, dtype=np.uint16).astype(np.uint32) << 16).view(
+        np.float32).astype(np.float64)
+
+
+def kmeans_assign(x_u16: np.ndarray, cent: np.ndarray):
+    """Labels (int32 [N]) and (best, second) distances for one (b, h)."""
+    x = np.ascontiguousarray(x_u16, dtype=np.uint16)
+    cent = np.ascontiguousarray(cent, dtype=np.float32)
+    N, d = x.shape
+    C = cent.shape[0]
+    label = np.zeros(N, dtype=np.int32)
+    diag = np.zeros((N, 2))
+    lib().oracle_kmeans_assign(_ptr(x), _ptr(cent), N, d, C, _ptr(label), _ptr(diag))
+    return label, diag
+
+
+def kmeans_update(x_u16: np.ndarray, label: np.ndarray, cent: np.ndarray):
+    """New centroids (member means; empty clusters keep theirs) and sizes."""
+    x = np.ascontiguousarray(x_u16, dtype=np.uint16)
+    out = np.array(cent, dtype=np.float32, copy=True)
+    N, d = x.shape
+    C = out.shape[0]
+    count = np.zeros(C, dtype=np.int32)
+    lib().oracle_kmeans_update(_ptr(x), _ptr(np.ascontiguousarray(label, dtype=np.int32)), N, d,
+                               C, _ptr(out), _ptr(count))
+    return out, count
+
+
+def kmeans(x_u16: np.ndarray, C: int, iters: int, init=None):
+    """Lloyd's iterations: init -> (assign, update) x iters -> final labels.
+    Returns (labels, centroids, sizes)."""
+    cent = kmeans_init(x_u16, C) if init is None else np.array(init, dtype=np.float32)
+    for _ in range(iters):
+        label, _ = kmeans_assign(x_u16, cent)
+        cent, count = kmeans_update(x_u16, label, cent)
+    label, _ = kmeans_assign(x_u16, cent)
+    _, count = kmeans_update(x_u16, label, cent)
+    return label, cent, count
+
+
+def cluster_order(label: np.ndarray, C: int):
+    """Stable sort by label: (order int64 [N], start int64 [C+1])."""
+    label = np.ascontiguousarray(label, dtype=np.int32)
+    order = np.zeros(label.size, dtype=np.int64)
+    start = np.zeros(C + 1, dtype=np.int64)
+    lib().oracle_cluster_order(_ptr(label), label.size, C, _ptr(order), _ptr(start))
+    return order, start
+
+
+def centroid_topp(cq: np.ndarray, ck: np.ndarray, nk: np.ndarray, p: float):
+    """Kept key clusters per query cluster (uint8 [Cq, Ck]) and diagnostics."""
+    cq = np.ascontiguousarray(cq, dtype=np.float32)
+    ck = np.ascontiguousarray(ck, dtype=np.float32)
+    nk = np.ascontiguousarray(nk, dtype=np.int32)
+    Cq, d = cq.shape
+    Ck = ck.shape[0]
+    keep = np.zeros((Cq, Ck), dtype=np.uint8)
+    diag = np.zeros((Cq, 5))
+    lib().oracle_centroid_topp(_ptr(cq), _ptr(ck), _ptr(nk), Cq, Ck, d, float(p), _ptr(keep),
+                               _ptr(diag))
+    return keep, diag
+
+
+def cluster_attention(q_u16, k_u16, v_u16, lq, lk, keep, qtok, scale=None):
+    """O (fp64 [len(qtok), d]) and LSE of the listed query tokens of one
+    (b, h) over the keys of their kept clusters, original token order."""
+    q, k, v = (np.ascontiguousarray(x, dtype=np.uint16) for x in (q_u16, k_u16, v_u16))
+    N, d = q.shape
+    qtok = np.ascontiguousarray(qtok, dtype=np.int64)
+    keep = np.ascontiguousarray(keep, dtype=np.uint8)
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    o = np.zeros((qtok.size, d))
+    lse = np.zeros(qtok.size)
+    lib().oracle_cluster_attention(_ptr(q), _ptr(k), _ptr(v), N, d,
+                                   _ptr(np.ascontiguousarray(lq, dtype=np.int32)),
+                                   _ptr(np.ascontiguousarray(lk, dtype=np.int32)), _ptr(keep),
+                                   keep.shape[1], float(scale), _ptr(qtok), qtok.size, _ptr(o),
+                                   _ptr(lse))
+    return o, lse
 
 
 def mask_to_csr(keep: np.ndarray):

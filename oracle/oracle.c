@@ -342,6 +342,202 @@ void oracle_block_mask_topk(const double *qp, const double *kp, int64_t BH,
 }
 
 /*
+ * Semantic-aware permutation (Sparse VideoGen2 summary, section 2A; k-means
+ * on Q and on K, independently, tokens of one cluster made contiguous) and
+ * centroid top-p (section 2B).  Readings where the page is silent: Lloyd's
+ * iterations from the tokens at positions floor(j*N/C) (or from cached
+ * centroids, section 2C), squared Euclidean distance, ties to the lower
+ * cluster, the assignment decided with the centroids rounded to bf16 (the
+ * precision the kernel's tensor-core contraction uses), an empty cluster
+ * keeping its centroid; the estimated attention of query cluster i on key
+ * cluster j proportional to |K_j| exp(c_qi . c_kj / sqrt(d)).
+ */
+
+/* bf16 rounding (round to nearest even) of a float, as the kernel's operand */
+static double bf16_round(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7F800000u) != 0x7F800000u)
+        u = (u + 0x7FFFu + ((u >> 16) & 1u)) & 0xFFFF0000u;
+    float r;
+    memcpy(&r, &u, 4);
+    return (double)r;
+}
+
+/* Assignment step for one (batch, head): x bf16 [N][d], centroids fp32
+ * [C][d].  label[t] = argmin_j ||x_t - c~_j||^2 with c~ = bf16(c), computed as
+ * ||c~_j||^2 - 2 x_t . c~_j in fp64.  diag[t] = (best, second best). */
+void oracle_kmeans_assign(const uint16_t *x, const float *cent, int64_t N, int d, int C,
+                          int32_t *label, double *diag)
+{
+    double *ct = (double *)malloc(sizeof(double) * (size_t)C * d);
+    double *cn = (double *)malloc(sizeof(double) * (size_t)C);
+    for (int j = 0; j < C; ++j) {
+        double s = 0.0;
+        for (int i = 0; i < d; ++i) {
+            double v = bf16_round(cent[(size_t)j * d + i]);
+            ct[(size_t)j * d + i] = v;
+            s += v * v;
+        }
+        cn[j] = s;
+    }
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < N; ++t) {
+        double best = INFINITY, second = INFINITY;
+        int arg = 0;
+        for (int j = 0; j < C; ++j) {
+            double dot = 0.0;
+            for (int i = 0; i < d; ++i)
+                dot += bf16_value(x[t * d + i]) * ct[(size_t)j * d + i];
+            double dist = cn[j] - 2.0 * dot;
+            if (dist < best) {
+                second = best;
+                best = dist;
+                arg = j;
+            } else if (dist < second) {
+                second = dist;
+            }
+        }
+        label[t] = arg;
+        if (diag) {
+            diag[2 * t] = best;
+            diag[2 * t + 1] = second;
+        }
+    }
+    free(ct);
+    free(cn);
+}
+
+/* Update step: the centroid of each non-empty cluster becomes the mean of
+ * its members (fp64 sum in token order, stored as fp32); an empty cluster
+ * keeps its centroid.  count[j] receives the cluster sizes. */
+void oracle_kmeans_update(const uint16_t *x, const int32_t *label, int64_t N, int d, int C,
+                          float *cent, int32_t *count)
+{
+    double *sum = (double *)calloc((size_t)C * d, sizeof(double));
+    memset(count, 0, sizeof(int32_t) * (size_t)C);
+    for (int64_t t = 0; t < N; ++t) {
+        int j = label[t];
+        ++count[j];
+        for (int i = 0; i < d; ++i)
+            sum[(size_t)j * d + i] += bf16_value(x[t * d + i]);
+    }
+    for (int j = 0; j < C; ++j)
+        if (count[j] > 0)
+            for (int i = 0; i < d; ++i)
+                cent[(size_t)j * d + i] = (float)(sum[(size_t)j * d + i] / count[j]);
+    free(sum);
+}
+
+/* The permutation: tokens in order of cluster, and in token order within a
+ * cluster (a stable sort by label).  order[p] = token at position p;
+ * start[j] = first position of cluster j (start[C] = N). */
+void oracle_cluster_order(const int32_t *label, int64_t N, int C, int64_t *order,
+                          int64_t *start)
+{
+    int64_t *cnt = (int64_t *)calloc((size_t)C + 1, sizeof(int64_t));
+    for (int64_t t = 0; t < N; ++t)
+        ++cnt[label[t] + 1];
+    for (int j = 0; j < C; ++j)
+        cnt[j + 1] += cnt[j];
+    for (int j = 0; j <= C; ++j)
+        start[j] = cnt[j];
+    for (int64_t t = 0; t < N; ++t)
+        order[cnt[label[t]]++] = t;
+    free(cnt);
+}
+
+/* Centroid top-p for one (batch, head): for query cluster i the estimated
+ * attention over key clusters a_ij = n_j exp(s_ij) / sum, s_ij = c_qi.c_kj /
+ * sqrt(d) (fp64, fp32 centroids as stored); the kept key clusters are the
+ * smallest prefix of (a desc, index asc) whose mass reaches p (the top-p rule
+ * of oracle_select_row with thr = 1 - p).  keep [Cq][Ck]; diag [Cq][5] as in
+ * oracle_select_row.  Empty key clusters have a = 0. */
+void oracle_centroid_topp(const float *cq, const float *ck, const int32_t *nk, int Cq,
+                          int Ck, int d, double p, uint8_t *keep, double *diag)
+{
+#pragma omp parallel
+    {
+        double *a = (double *)malloc(sizeof(double) * (size_t)Ck);
+#pragma omp for schedule(static)
+        for (int i = 0; i < Cq; ++i) {
+            double m = -INFINITY;
+            for (int j = 0; j < Ck; ++j) {
+                double s = 0.0;
+                for (int e = 0; e < d; ++e)
+                    s += (double)cq[(size_t)i * d + e] * (double)ck[(size_t)j * d + e];
+                a[j] = nk[j] > 0 ? s / sqrt((double)d) : -INFINITY;
+                if (a[j] > m)
+                    m = a[j];
+            }
+            double z = 0.0;
+            for (int j = 0; j < Ck; ++j) {
+                a[j] = nk[j] > 0 ? (double)nk[j] * exp(a[j] - m) : 0.0;
+                z += a[j];
+            }
+            for (int j = 0; j < Ck; ++j)
+                a[j] /= z;
+            oracle_select_row(a, Ck, 1.0 - p, keep + (size_t)i * Ck,
+                              diag ? diag + (size_t)i * 5 : NULL);
+        }
+        free(a);
+    }
+}
+
+/* Attention of the listed query tokens of one (batch, head) over the key
+ * tokens whose key cluster is kept for the query token's cluster, in the
+ * original token order (the permutation changes no result, SVG2 section 2A).
+ * q, k, v bf16 [N][d]; lq, lk labels; keep [Cq][Ck]; o [nq][d], lse [nq]. */
+void oracle_cluster_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                              int64_t N, int d, const int32_t *lq, const int32_t *lk,
+                              const uint8_t *keep, int Ck, double scale,
+                              const int64_t *qtok, int64_t nq, double *o, double *lse)
+{
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)N);
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t a = 0; a < nq; ++a) {
+            int64_t t = qtok[a];
+            const uint8_t *kr = keep + (size_t)lq[t] * Ck;
+            double m = -INFINITY;
+            for (int64_t u = 0; u < N; ++u) {
+                if (!kr[lk[u]]) {
+                    s[u] = -INFINITY;
+                    continue;
+                }
+                double dot = 0.0;
+                for (int e = 0; e < d; ++e)
+                    dot += bf16_value(q[t * d + e]) * bf16_value(k[u * d + e]);
+                s[u] = dot * scale;
+                if (s[u] > m)
+                    m = s[u];
+            }
+            double z = 0.0;
+            for (int e = 0; e < d; ++e)
+                o[a * d + e] = 0.0;
+            if (m == -INFINITY) {
+                lse[a] = -INFINITY;
+                continue;
+            }
+            for (int64_t u = 0; u < N; ++u) {
+                if (s[u] == -INFINITY)
+                    continue;
+                double w = exp(s[u] - m);
+                z += w;
+                for (int e = 0; e < d; ++e)
+                    o[a * d + e] += w * bf16_value(v[u * d + e]);
+            }
+            for (int e = 0; e < d; ++e)
+                o[a * d + e] /= z;
+            lse[a] = m + log(z);
+        }
+        free(s);
+    }
+}
+
+/*
  * The STA window on its own (NABLA summary, "Methodology" item 3, the
  * sliding-tile component M_STA of M = M_nabla OR M_STA, used without the
  * content-adaptive part): keep[r][c] = 1 exactly when key block c lies within

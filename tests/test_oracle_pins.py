@@ -394,3 +394,114 @@ def test_query_subset_rows_equal_full_rows_and_dense():
     qt, kt, vt = (oracle.to_bf16_tensor(x).double() for x in (qf, kf, vf))
     ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt)
     np.testing.assert_allclose(o_sub, ref.reshape(-1, wl.d).numpy()[idx], rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- f1 semantic-aware permutation
+def _bf16_u16(a: np.ndarray) -> np.ndarray:
+    return oracle.as_u16(torch.from_numpy(np.asarray(a, dtype=np.float32)).to(torch.bfloat16))
+
+
+def test_kmeans_recovers_planted_clusters():
+    """Three well-separated groups laid out so that the evenly spaced initial
+    tokens fall one in each: labels recover the groups and centroids are the
+    groups' means."""
+    rng = np.random.default_rng(8)
+    d, n = 16, 90
+    centers = np.zeros((3, d))
+    centers[0, 0], centers[1, 1], centers[2, 2] = 20.0, -20.0, 20.0
+    truth = np.arange(n) % 3
+    x = _bf16_u16(centers[truth] + 0.1 * rng.standard_normal((n, d)))
+    # group-major layout: the initial tokens 0, 30, 60 fall one per group
+    order = np.argsort(truth, kind="stable")            # 0..0 1..1 2..2
+    xs = x[order]
+    label, cent, count = oracle.kmeans(xs, 3, 4)
+    np.testing.assert_array_equal(label, np.repeat([0, 1, 2], n // 3))
+    np.testing.assert_array_equal(count, [n // 3] * 3)
+    xf = oracle.to_f64(xs)
+    for j in range(3):
+        np.testing.assert_allclose(cent[j], xf[label == j].mean(axis=0), rtol=1e-6, atol=1e-6)
+
+
+def test_kmeans_assign_is_argmin_of_numpy_distances():
+    """The oracle's ||c~||^2 - 2 x.c~ against numpy's full squared distance
+    with the same bf16-rounded centroids; ties would go to the lower index in
+    both (numpy argmin returns the first minimum)."""
+    rng = np.random.default_rng(9)
+    x = _bf16_u16(rng.standard_normal((200, 32)))
+    cent = rng.standard_normal((7, 32)).astype(np.float32)
+    label, diag = oracle.kmeans_assign(x, cent)
+    cb = oracle.to_f64(_bf16_u16(cent))
+    dist = ((oracle.to_f64(x)[:, None, :] - cb[None, :, :]) ** 2).sum(-1)
+    np.testing.assert_array_equal(label, np.argmin(dist, axis=1))
+    xn = (oracle.to_f64(x) ** 2).sum(-1)
+    np.testing.assert_allclose(diag[:, 0] + xn, dist.min(axis=1), rtol=1e-12, atol=1e-9)
+
+
+def test_kmeans_update_means_and_empty_cluster():
+    rng = np.random.default_rng(10)
+    x = _bf16_u16(rng.standard_normal((50, 8)))
+    label = rng.integers(0, 3, 50).astype(np.int32)          # cluster 3 is empty
+    old = rng.standard_normal((4, 8)).astype(np.float32)
+    cent, count = oracle.kmeans_update(x, label, old)
+    np.testing.assert_array_equal(count, np.bincount(label, minlength=4))
+    xf = oracle.to_f64(x)
+    for j in range(3):
+        np.testing.assert_allclose(cent[j], xf[label == j].mean(axis=0).astype(np.float32),
+                                   rtol=0, atol=2e-7)
+    np.testing.assert_array_equal(cent[3], old[3])
+
+
+def test_cluster_order_is_stable_sort():
+    rng = np.random.default_rng(12)
+    label = rng.integers(0, 9, 500).astype(np.int32)
+    order, start = oracle.cluster_order(label, 10)
+    np.testing.assert_array_equal(order, np.argsort(label, kind="stable"))
+    np.testing.assert_array_equal(start, np.concatenate([[0], np.cumsum(np.bincount(label, minlength=10))]))
+
+
+def test_centroid_topp_size_weighting():
+    """Two key clusters with the same centroid: estimated attention in the
+    ratio of their sizes (30:10, so 0.75 and 0.25 exactly); an empty cluster
+    gets none."""
+    ck = np.array([[1.0, 0.0], [1.0, 0.0], [0.0, 5.0]], dtype=np.float32)
+    cq = np.array([[0.5, 0.0]], dtype=np.float32)
+    nk = np.array([30, 10, 0], dtype=np.int32)
+    keep, diag = oracle.centroid_topp(cq, ck, nk, 0.75)       # 0.75 = 30/40 exactly
+    np.testing.assert_array_equal(keep[0], [1, 0, 0])
+    keep, _ = oracle.centroid_topp(cq, ck, nk, 0.8)
+    np.testing.assert_array_equal(keep[0], [1, 1, 0])
+    # p = 1 keeps every cluster, as thr = 0 does in the top-p rule (an empty
+    # cluster brings no keys)
+    keep, _ = oracle.centroid_topp(cq, ck, nk, 1.0)
+    np.testing.assert_array_equal(keep[0], [1, 1, 1])
+
+
+def test_cluster_attention_against_masked_sdpa_and_permutation():
+    """Token-level attention over kept clusters equals torch SDPA with the
+    boolean mask built from the labels; all clusters kept is dense attention;
+    and computing it on the permuted sequence and permuting back gives the
+    same result (SVG2 section 2A)."""
+    wl = workloads.get("tiny")
+    q, k, v = workloads.make_qkv(wl)
+    qu, ku, vu = (oracle.as_u16(x)[0, 0] for x in (q, k, v))
+    lq, cq, nq = oracle.kmeans(qu, 6, 2)
+    lk, ck, nk = oracle.kmeans(ku, 9, 2)
+    keep, _ = oracle.centroid_topp(cq, ck, nk, 0.7)
+    tok = np.arange(wl.N)
+    o, lse = oracle.cluster_attention(qu, ku, vu, lq, lk, keep, tok)
+    qt, kt, vt = (torch.from_numpy(oracle.to_f64(x)) for x in (qu, ku, vu))
+    mask = torch.from_numpy(keep[lq][:, lk].astype(bool))
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask)
+    np.testing.assert_allclose(o, ref.numpy(), rtol=0, atol=1e-12)
+    ones = np.ones_like(keep)
+    o_all, _ = oracle.cluster_attention(qu, ku, vu, lq, lk, ones, tok)
+    dense = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt)
+    np.testing.assert_allclose(o_all, dense.numpy(), rtol=0, atol=1e-12)
+    # permuted computation, permuted back
+    oq, _ = oracle.cluster_order(lq, 6)
+    ok, _ = oracle.cluster_order(lk, 9)
+    pm = torch.from_numpy(keep[lq[oq]][:, lk[ok]].astype(bool))
+    perm = torch.nn.functional.scaled_dot_product_attention(qt[oq], kt[ok], vt[ok], attn_mask=pm)
+    back = torch.empty_like(perm)
+    back[torch.from_numpy(oq)] = perm
+    np.testing.assert_allclose(back.numpy(), o, rtol=0, atol=1e-12)
