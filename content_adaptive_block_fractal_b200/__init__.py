@@ -22,6 +22,7 @@ __all__ = ["Shape", "MaskParams", "VsaError", "fractal_flatten", "fractal_unflat
            "flatten_pool_qk",
            "pool_qk", "block_mask", "block_mask_topk", "sta_mask", "sta_mask_nnz",
            "block_mask_workspace_size", "sparse_attn_fwd", "sparse_attn_fwd_rows",
+           "ClusterParams", "cluster_attention", "cluster_attn_workspace_size",
            "sparse_attn_workspace_size", "attention_layer", "device_status", "version",
            "Csr"]
 
@@ -235,6 +236,63 @@ def sparse_attn_fwd_rows(qf, kf, vf, row_ptr, col_idx, shape: Shape, qblocks: to
         _ptr(qb) if qb.numel() else ctypes_void(0), qb.numel(), _ptr(o), _ptr(lse),
         _ptr(workspace), workspace.numel(), _stream(stream)))
     return o, lse
+
+
+@dataclasses.dataclass
+class ClusterParams:
+    """Semantic-aware permutation: clusters of Q and K, Lloyd iterations, and
+    the estimated-attention mass kept per query cluster."""
+    Cq: int = 256
+    Ck: int = 512
+    iters: int = 2
+    p: float = 0.9
+
+    def c(self):
+        return _lib.vsa_cluster_params(int(self.Cq), int(self.Ck), int(self.iters),
+                                       float(self.p))
+
+
+def cluster_attn_workspace_size(shape: Shape, params: ClusterParams) -> int:
+    return int(_lib.load().vsa_cluster_attn_workspace_size(shape.c(), params.c()))
+
+
+def cluster_attention(q, k, v, shape: Shape, params: ClusterParams, scale: float = 0.0,
+                      init=None, want_state: bool = False, out=None, workspace=None,
+                      stream=None):
+    """k-means permutation + centroid top-p + attention over the kept clusters
+    -> (o, lse) in the input token order, plus the intermediate state (labels,
+    sizes, centroids, kept flags) when want_state is set.  `init` is an
+    optional (q_centroids, k_centroids) pair of fp32 [B,h,C,d] tensors."""
+    import ctypes
+    dev = q.device
+    if out is None:
+        out = (torch.empty_like(q),
+               torch.empty((shape.B, shape.heads, shape.N), dtype=torch.float32, device=dev))
+    o, lse = out
+    if workspace is None:
+        workspace = _workspace(cluster_attn_workspace_size(shape, params), dev)
+    B, h, N, d = shape.B, shape.heads, shape.N, shape.d
+    st = None
+    if want_state:
+        i32, f32 = torch.int32, torch.float32
+        st = {"q_labels": torch.empty((B, h, N), dtype=i32, device=dev),
+              "k_labels": torch.empty((B, h, N), dtype=i32, device=dev),
+              "q_counts": torch.empty((B, h, params.Cq), dtype=i32, device=dev),
+              "k_counts": torch.empty((B, h, params.Ck), dtype=i32, device=dev),
+              "q_centroids": torch.empty((B, h, params.Cq, d), dtype=f32, device=dev),
+              "k_centroids": torch.empty((B, h, params.Ck, d), dtype=f32, device=dev),
+              "keep": torch.empty((B, h, params.Cq, params.Ck), dtype=torch.uint8, device=dev)}
+        cst = _lib.vsa_cluster_state(*(t.data_ptr() for t in st.values()))
+        cst_ptr = ctypes.pointer(cst)
+    else:
+        cst_ptr = None
+    iq, ik = (None, None) if init is None else init
+    _lib.check(_lib.load().vsa_cluster_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), shape.c(), params.c(), float(scale),
+        _ptr(iq) if iq is not None else ctypes_void(0),
+        _ptr(ik) if ik is not None else ctypes_void(0), _ptr(o), _ptr(lse), cst_ptr,
+        _ptr(workspace), workspace.numel(), _stream(stream)))
+    return (o, lse, st) if want_state else (o, lse)
 
 
 def device_status(stream=None) -> None:

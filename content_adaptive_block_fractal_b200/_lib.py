@@ -23,7 +23,20 @@ EXPORTS = ("vsa_fractal_flatten", "vsa_fractal_unflatten", "vsa_pool_qk",
            "vsa_sta_mask",
            "vsa_sparse_attn_workspace_size", "vsa_sparse_attn_fwd",
            "vsa_sparse_attn_fwd_noalloc", "vsa_sparse_attn_fwd_rows",
+           "vsa_cluster_attn_workspace_size", "vsa_cluster_attn_fwd",
            "vsa_last_error", "vsa_device_status", "vsa_version")
+
+
+class vsa_cluster_params(ctypes.Structure):
+    _fields_ = [("Cq", ctypes.c_int32), ("Ck", ctypes.c_int32), ("iters", ctypes.c_int32),
+                ("p", ctypes.c_float)]
+
+
+class vsa_cluster_state(ctypes.Structure):
+    _fields_ = [("q_labels", ctypes.c_void_p), ("k_labels", ctypes.c_void_p),
+                ("q_counts", ctypes.c_void_p), ("k_counts", ctypes.c_void_p),
+                ("q_centroids", ctypes.c_void_p), ("k_centroids", ctypes.c_void_p),
+                ("keep", ctypes.c_void_p)]
 
 
 class vsa_shape(ctypes.Structure):
@@ -74,6 +87,8 @@ def load():
         "vsa_sparse_attn_fwd_noalloc": [P, P, P, P, P, vsa_shape, F, P, P, P],
         "vsa_sparse_attn_fwd_rows": [P, P, P, P, P, vsa_shape, F, P, I64, P, P, P, S, P],
         "vsa_device_status": [P],
+        "vsa_cluster_attn_fwd": [P, P, P, vsa_shape, vsa_cluster_params, F, P, P, P, P,
+                                 ctypes.POINTER(vsa_cluster_state), P, S, P],
     }.items():
         fn = getattr(L, name)
         fn.argtypes = args
@@ -82,6 +97,8 @@ def load():
     L.vsa_block_mask_workspace_size.restype = S
     L.vsa_sparse_attn_workspace_size.argtypes = [vsa_shape]
     L.vsa_sparse_attn_workspace_size.restype = S
+    L.vsa_cluster_attn_workspace_size.argtypes = [vsa_shape, vsa_cluster_params]
+    L.vsa_cluster_attn_workspace_size.restype = S
     L.vsa_last_error.restype = ctypes.c_char_p
     L.vsa_version.restype = ctypes.c_char_p
     _lib = L

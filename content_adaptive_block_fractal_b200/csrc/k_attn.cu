@@ -42,6 +42,7 @@
 // and the CTA winds down instead of hanging.
 #include "vsa_device.cuh"
 #include "vsa_internal.h"
+#include "vsa_tma.h"
 
 #include <cmath>
 #include <cstdio>
@@ -60,7 +61,8 @@ constexpr uint32_t kColO = 384;
 struct StepMeta {
   int32_t blk0, blk1;  // key blocks of this step (blk1 = -1 when nb == 1)
   int32_t nb;          // 1 or 2 key blocks; 0 = empty item; -1 = no more work
-  uint32_t flags;      // bit0/1: blk0 kept by query block 0/1; bit2/3: blk1
+  uint32_t flags;      // bit0/1: blk0 kept by query block 0/1; bit2/3: blk1;
+                       // bits 8-14 / 16-22: valid keys of blk0 / blk1 (1..64)
   int32_t bh, r0, r1;  // head slice and query blocks (r1 = -1 if absent)
   int32_t first_last;  // bit0: first step of the item, bit1: last step
   int32_t seq;         // item sequence number within this CTA
@@ -102,6 +104,8 @@ struct AttnArgs {
                           // order[] then holds the list index of each item's lead
   const int32_t *qblocks; // query-subset mode: the listed global query-block rows
   int64_t n_qblocks;
+  const int32_t *kvalid;  // optional: valid keys (1..64) of each key block, the rest
+                          // of the block is masked out; null: all 64
   int64_t N;              // tokens per head
   int Nb, T, HW;          // blocks per head, frames, patches per frame
   int pairs_per_head;
@@ -135,21 +139,33 @@ __device__ __forceinline__ void decode_item(int item, const AttnArgs &a, int &bh
 // reference, adds to the row sums and stores P as 16 packed bf16x2 columns
 // over S columns [16Q, 16Q+16) (scores already read), then waits for `nxt`.
 // Chunks 0-1 are key block 0 (valid when v0), chunks 2-3 key block 1.
+// `lim` is the number of valid key columns in this chunk (32 unless the key
+// block is a partial one); columns past it get P = 0.
 template <int Q>
 __device__ __forceinline__ void softmax_chunk(uint32_t (&cur)[32], uint32_t (&nxt)[32], int nq,
                                               bool v0, bool v1, uint32_t s_addr, float2 c2,
-                                              float2 nm2, float2 (&r4)[4]) {
+                                              float2 nm2, float2 (&r4)[4], int lim) {
   if (Q >= nq) return;
   const bool vq = Q < 2 ? v0 : v1;
   const bool vn = Q + 1 < nq && (Q + 1 < 2 ? v0 : v1);
   if (vn) tmem_ld32_nowait(s_addr + 32 * (Q + 1), nxt);
   uint32_t pk[16];
-  if (vq) {
+  if (vq && lim >= 32) {
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const float2 t =
           ffma2(make_float2(__uint_as_float(cur[2 * j]), __uint_as_float(cur[2 * j + 1])), c2, nm2);
       const float2 p = make_float2(ex2(t.x), ex2(t.y));
+      r4[j & 3] = fadd2(r4[j & 3], p);
+      pk[j] = pack_bf16x2(p.x, p.y);
+    }
+  } else if (vq) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float2 t =
+          ffma2(make_float2(__uint_as_float(cur[2 * j]), __uint_as_float(cur[2 * j + 1])), c2, nm2);
+      const float2 p = make_float2(2 * j < lim ? ex2(t.x) : 0.0f,
+                                   2 * j + 1 < lim ? ex2(t.y) : 0.0f);
       r4[j & 3] = fadd2(r4[j & 3], p);
       pk[j] = pack_bf16x2(p.x, p.y);
     }
@@ -335,13 +351,14 @@ __global__ void __maxnreg__(168)
           if (lane == 0) atomicOr(a.err, kErrBadIndex);
           continue;
         }
+        const uint32_t kv = a.kvalid ? static_cast<uint32_t>(a.kvalid[g0 - r0 + c]) & 0x7Fu : 64u;
         if (cur.nb == 0) {
           cur.blk0 = c;
-          cur.flags = f;
+          cur.flags = f | (kv << 8);
           cur.nb = 1;
         } else {
           cur.blk1 = c;
-          cur.flags |= f << 2;
+          cur.flags |= (f << 2) | (kv << 16);
           cur.nb = 2;
           if (have_pending && !(ok = emit(pend))) break;
           pend = cur;
@@ -508,6 +525,8 @@ __global__ void __maxnreg__(168)
       // warps hold rows of one query block, so v0 / v1 are warp-uniform
       const bool v0 = m.nb > 0 && ((m.flags >> sel) & 1u);
       const bool v1 = m.nb > 1 && ((m.flags >> (2 + sel)) & 1u);
+      const int kv0 = static_cast<int>((m.flags >> 8) & 0x7Fu);    // valid keys per block
+      const int kv1 = static_cast<int>((m.flags >> 16) & 0x7Fu);
       float mx = -INFINITY;
       if (v0 || v1) {
         // pass 1: row max over the valid halves, 64 scores live at a time
@@ -517,6 +536,11 @@ __global__ void __maxnreg__(168)
           if (h ? v1 : v0) {
             float x[64];
             tmem_ld64(s_addr + 64 * h, x);
+            const int kv = h ? kv1 : kv0;
+            if (kv < 64) {
+#pragma unroll
+              for (int j = 0; j < 64; ++j) x[j] = j < kv ? x[j] : -INFINITY;
+            }
 #pragma unroll
             for (int j = 0; j < 64; j += 2)
               m4[(j >> 1) & 3] = fmax3(m4[(j >> 1) & 3], x[j], x[j + 1]);
@@ -567,10 +591,10 @@ __global__ void __maxnreg__(168)
           tmem_ld32_nowait(s_addr, xa);
           tmem_wait_ld_regs(xa);
         }
-        softmax_chunk<0>(xa, xb, nq, v0, v1, s_addr, c2, nm2, r4);
-        softmax_chunk<1>(xb, xa, nq, v0, v1, s_addr, c2, nm2, r4);
-        softmax_chunk<2>(xa, xb, nq, v0, v1, s_addr, c2, nm2, r4);
-        softmax_chunk<3>(xb, xa, nq, v0, v1, s_addr, c2, nm2, r4);
+        softmax_chunk<0>(xa, xb, nq, v0, v1, s_addr, c2, nm2, r4, kv0);
+        softmax_chunk<1>(xb, xa, nq, v0, v1, s_addr, c2, nm2, r4, kv0 - 32);
+        softmax_chunk<2>(xa, xb, nq, v0, v1, s_addr, c2, nm2, r4, kv1);
+        softmax_chunk<3>(xb, xa, nq, v0, v1, s_addr, c2, nm2, r4, kv1 - 32);
       }
       const float rs = ((r4[0].x + r4[0].y) + (r4[1].x + r4[1].y)) +
                        ((r4[2].x + r4[2].y) + (r4[3].x + r4[3].y));
@@ -735,43 +759,6 @@ __global__ void identity_order_kernel(int32_t *order, int64_t n, int *counter) {
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
-using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                              const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                              const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeFn encode_fn() {
-  static EncodeFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeFn>(p);
-  });
-  return fn;
-}
-
-// [rows, d] bf16 viewed as (64 elements, 8 rows, d/64 halves, rows/8 groups):
-// one box {64, 8, d/64, 8} is a whole 64-row block stored as
-// [row group][d-half][8 rows][128 B], i.e. 1 KiB swizzle atoms with the
-// d-halves of a row group side by side.
-bool make_map4(CUtensorMap *m, const void *base, int64_t rows, int d) {
-  EncodeFn enc = encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[4] = {64, 8, static_cast<cuuint64_t>(d / 64),
-                              static_cast<cuuint64_t>(rows / 8)};
-  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, 128,
-                                 static_cast<cuuint64_t>(d) * 2 * 8};
-  const cuuint32_t box[4] = {64, 8, static_cast<cuuint32_t>(d / 64), 8};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
-}
 
 struct AttnLayout {
   int pairs, HW;
@@ -798,7 +785,8 @@ cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
                                const int64_t *row_ptr, const int32_t *col_idx,
                                const Geometry &g, float scale, void *o, float *lse, void *ws,
                                unsigned *err, cudaStream_t st, const char **why,
-                               const int32_t *qblocks, int64_t n_qblocks) {
+                               const int32_t *qblocks, int64_t n_qblocks,
+                               const int32_t *kvalid) {
   const AttnLayout L = attn_layout(g);
   if (L.items == 0 || (qblocks && n_qblocks == 0)) return cudaSuccess;
   if (L.items > 0x7FFFFFFF || g.BH * g.N > 0x7FFFFFFF) {
@@ -840,6 +828,7 @@ cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
   a.n_items = qblocks ? n_items : nullptr;
   a.qblocks = qblocks;
   a.n_qblocks = n_qblocks;
+  a.kvalid = kvalid;
   a.pairs_per_head = L.pairs;
   a.c = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   a.lse_scale = 0.6931471805599453f;

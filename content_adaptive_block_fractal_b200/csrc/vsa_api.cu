@@ -98,6 +98,59 @@ const char *vsa_version(void) { return "0.1.0"; }
 
 const char *vsa_last_error(void) { return g_last_error.c_str(); }
 
+static vsa_status check_cluster(const vsa_shape &s, const vsa_cluster_params &c) {
+  vsa_status st = check_shape(s);
+  if (st != VSA_OK) return st;
+  const vsa::Geometry g = vsa::geometry(s);
+  if (c.Cq < 1 || c.Ck < 1 || c.Cq > 1024 || c.Ck > 1024 || c.Cq > g.N || c.Ck > g.N)
+    return fail(VSA_ERR_INVALID_ARG, "cluster counts (%d, %d) outside [1, min(1024, N)]", c.Cq,
+                c.Ck);
+  if (c.iters < 0 || c.iters > 64) return fail(VSA_ERR_INVALID_ARG, "iters=%d outside [0, 64]", c.iters);
+  if (!(c.p > 0.0f && c.p <= 1.0f))
+    return fail(VSA_ERR_INVALID_ARG, "p=%g outside (0, 1]", static_cast<double>(c.p));
+  const int64_t Np = g.N + 64LL * (c.Cq > c.Ck ? c.Cq : c.Ck);
+  if (g.BH * Np >= (1LL << 31))
+    return fail(VSA_ERR_UNSUPPORTED, "padded sequence too long for 32-bit row coordinates");
+  return VSA_OK;
+}
+
+size_t vsa_cluster_attn_workspace_size(vsa_shape s, vsa_cluster_params c) {
+  if (check_cluster(s, c) != VSA_OK) return 0;
+  return vsa::cluster_workspace_bytes(vsa::geometry(s), c);
+}
+
+vsa_status vsa_cluster_attn_fwd(const void *q, const void *k, const void *v, vsa_shape s,
+                                vsa_cluster_params c, float scale, const float *init_q,
+                                const float *init_k, void *o, float *lse,
+                                const vsa_cluster_state *state, void *workspace,
+                                size_t workspace_bytes, void *stream) {
+  vsa_status st = check_cluster(s, c);
+  if (st != VSA_OK) return st;
+  if (empty(s)) return VSA_OK;
+  if (!q || !k || !v || !o || !lse || !workspace)
+    return fail(VSA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      (init_q && !aligned16(init_q)) || (init_k && !aligned16(init_k)))
+    return fail(VSA_ERR_UNSUPPORTED, "misaligned pointer (tensors 16 B, workspace 256 B)");
+  if (!(scale == scale)) return fail(VSA_ERR_INVALID_ARG, "scale is NaN");
+  const vsa::Geometry g = vsa::geometry(s);
+  const size_t ws = vsa::cluster_workspace_bytes(g, c);
+  if (workspace_bytes < ws)
+    return fail(VSA_ERR_CAPACITY, "cluster attention workspace %zu < %zu bytes", workspace_bytes, ws);
+  if (scale <= 0.0f) scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(s.d)));
+  cudaError_t e;
+  unsigned *err = device_error_word(&e);
+  if (!err) return cuda_fail(e, "device error word");
+  const char *why = nullptr;
+  e = vsa::launch_cluster_attn(q, k, v, g, c, scale, init_q, init_k, o, lse, state, workspace,
+                               err, static_cast<cudaStream_t>(stream), &why);
+  if (e != cudaSuccess)
+    return why ? fail(e == cudaErrorInvalidValue ? VSA_ERR_UNSUPPORTED : VSA_ERR_CUDA, "%s", why)
+               : cuda_fail(e, "cluster attention launch");
+  return VSA_OK;
+}
+
 static vsa_status permute(const void *src, void *dst, vsa_shape s, void *stream, bool inverse) {
   vsa_status st = check_shape(s);
   if (st != VSA_OK) return st;

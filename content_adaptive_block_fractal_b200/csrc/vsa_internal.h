@@ -56,6 +56,15 @@ cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
                                const int64_t *row_ptr, const int32_t *col_idx,
                                const Geometry &g, float scale, void *o, float *lse, void *ws,
                                unsigned *err, cudaStream_t st, const char **why,
-                               const int32_t *qblocks = nullptr, int64_t n_qblocks = 0);
+                               const int32_t *qblocks = nullptr, int64_t n_qblocks = 0,
+                               const int32_t *kvalid = nullptr);
+
+// Semantic-aware permutation attention: workspace and launch.
+size_t cluster_workspace_bytes(const Geometry &g, const vsa_cluster_params &c);
+cudaError_t launch_cluster_attn(const void *q, const void *k, const void *v, const Geometry &g,
+                                const vsa_cluster_params &c, float scale, const float *init_q,
+                                const float *init_k, void *o, float *lse,
+                                const vsa_cluster_state *out_state, void *ws, unsigned *err,
+                                cudaStream_t st, const char **why);
 
 }  // namespace vsa

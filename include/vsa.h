@@ -217,6 +217,45 @@ vsa_status vsa_sparse_attn_fwd_noalloc(const void *qf, const void *kf, const voi
                                        vsa_shape s, float scale, void *o, float *lse,
                                        void *stream);
 
+/* Semantic-aware permutation attention (Sparse VideoGen2, arXiv 2505.18875
+ * summary, sections 2A-2C).  Per (b, h): k-means on Q into Cq clusters and on
+ * K into Ck clusters (Lloyd's iterations from the given centroids -- the
+ * centroid cache of section 2C -- or from the tokens at positions
+ * floor(j*N/C); squared Euclidean distance with the centroids rounded to bf16,
+ * ties to the lower cluster; an empty cluster keeps its centroid), tokens
+ * permuted so that each cluster is contiguous (token order inside a cluster),
+ * key clusters kept per query cluster by the centroids' estimated attention
+ * a_j ~ |K_j| exp(c_q . c_kj / sqrt(d)) until the kept mass reaches p (ties to
+ * the lower index; p = 1 keeps every cluster), and attention of every query
+ * token over the key tokens of its cluster's kept clusters.
+ * q, k, v : device bf16 [B,heads,N,d] in any token order (the result does not
+ *           depend on the order beyond the initial centroids).
+ * o, lse  : device bf16 [B,heads,N,d], fp32 [B,heads,N], same token order.
+ * init_q, init_k : optional device fp32 [B,heads,Cq|Ck,d] initial centroids.
+ * state   : optional; each non-null member receives that intermediate.
+ * Limits: 1 <= Cq, Ck <= min(1024, N), 0 <= iters <= 64, 0 < p <= 1;
+ * the workspace (vsa_cluster_attn_workspace_size, 256-byte aligned) holds the
+ * padded permuted tensors, so it is several times the size of Q. */
+typedef struct {
+    int32_t Cq, Ck;     /* clusters of Q and of K */
+    int32_t iters;      /* Lloyd iterations (assign + update) before the final assignment */
+    float p;            /* kept estimated-attention mass per query cluster */
+} vsa_cluster_params;
+
+typedef struct {
+    int32_t *q_labels, *k_labels;       /* [B,heads,N] */
+    int32_t *q_counts, *k_counts;       /* [B,heads,Cq|Ck] cluster sizes */
+    float *q_centroids, *k_centroids;   /* [B,heads,Cq|Ck,d], the ones labels were assigned with */
+    uint8_t *keep;                      /* [B,heads,Cq,Ck] kept key clusters */
+} vsa_cluster_state;
+
+size_t vsa_cluster_attn_workspace_size(vsa_shape s, vsa_cluster_params c);
+vsa_status vsa_cluster_attn_fwd(const void *q, const void *k, const void *v, vsa_shape s,
+                                vsa_cluster_params c, float scale, const float *init_q,
+                                const float *init_k, void *o, float *lse,
+                                const vsa_cluster_state *state, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
 /* Message for the last non-OK status returned to the calling thread. */
 const char *vsa_last_error(void);
 
