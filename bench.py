@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cluster", action="store_true",
+                    help="only the semantic-aware permutation path at the Wan-14B 720p shape")
     ap.add_argument("--sweep", action="store_true",
                     help="thr x STA sweep at the Wan-14B 720p shape: one JSON line per point "
                          "(mask + attention; inputs generated once)")
@@ -413,6 +415,59 @@ def run_sweep(args):
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peak_tf, "frac": tf / peak_tf,
                          "peak_source": f"{peak_src} bf16 sustained"},
             "clocks": clk.summary()}), flush=True)
+    # the semantic-aware permutation path, on the raster inputs
+    print(json.dumps(run_cluster_point(args, qd, kd, vd, shape, peak_tf, peak_src,
+                                       vsa.ClusterParams(256, 512, 2, 0.9))), flush=True)
+
+
+def run_cluster_point(args, q, k, v, shape, peak_tf, peak_src, params):
+    """The semantic-aware permutation path as one call, timed whole (k-means,
+    permutation, centroid top-p, attention, inverse permutation)."""
+    import torch
+    import content_adaptive_block_fractal_b200 as vsa
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=q.device)
+    ws = vsa._workspace(vsa.cluster_attn_workspace_size(shape, params), q.device)
+    o = torch.empty_like(q)
+    lse = torch.empty((shape.B, shape.heads, shape.N), dtype=torch.float32, device=q.device)
+    _, _, st = vsa.cluster_attention(q, k, v, shape, params, want_state=True, out=(o, lse),
+                                     workspace=ws)
+    for _ in range(max(args.warmup, 3) - 1):
+        vsa.cluster_attention(q, k, v, shape, params, out=(o, lse), workspace=ws)
+    vsa.device_status()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    steps = max(args.steps, 1)
+    total = 0.0
+    with ClockSampler(0) as clk:
+        for _ in range(steps):
+            flush.zero_()
+            e0.record()
+            vsa.cluster_attention(q, k, v, shape, params, out=(o, lse), workspace=ws)
+            e1.record()
+            e1.synchronize()
+            total += e0.elapsed_time(e1)
+    vsa.device_status()
+    ms = total / steps
+    # work: padded 64x64 tiles the attention kernel runs, and the useful
+    # query-key token pairs (each kept cluster pair counted at its true sizes)
+    nq = st["q_counts"].double()
+    nk = st["k_counts"].double()
+    keep = st["keep"].double()
+    tiles = float(((nq / 64).ceil() * (keep @ (nk / 64).ceil().unsqueeze(-1)).squeeze(-1)).sum())
+    pairs = float((nq * (keep @ nk.unsqueeze(-1)).squeeze(-1)).sum())
+    flop_tile = 4 * 64 * 64 * shape.d
+    return {
+        "metric": "semantic-aware permutation attention ms at Wan-14B 720p shape",
+        "value": ms, "unit": "ms", "steps": steps,
+        "mask": f"semantic permutation Cq={params.Cq} Ck={params.Ck} iters={params.iters} "
+                f"p={params.p}",
+        "config": {"workload": "wan14b-720p", "B": shape.B, "heads": shape.heads, "d": shape.d,
+                   "grid": [shape.T, shape.H, shape.W], "data": "synthetic"},
+        "kept_pair_fraction": pairs / (shape.B * shape.heads * shape.N ** 2),
+        "padded_tiles": tiles,
+        "tflops_useful_pairs_whole_call": pairs * 4 * shape.d / (ms * 1e-3) / 1e12,
+        "tflops_padded_tiles_whole_call": tiles * flop_tile / (ms * 1e-3) / 1e12,
+        "peak": peak_tf, "peak_source": f"{peak_src} bf16 sustained",
+        "clocks": clk.summary()}
 
 
 # --------------------------------------------------------------------------- CPU oracle
@@ -488,9 +543,21 @@ def main():
         if rank == 0:
             run_reference(args)
         return
-    if args.sweep:
+    if args.sweep or args.cluster:
         if rank == 0:
-            run_sweep(args)
+            if args.sweep:
+                run_sweep(args)
+            else:
+                import torch
+                import content_adaptive_block_fractal_b200 as vsa
+                from content_adaptive_block_fractal_b200 import workloads
+                wl = workloads.get(WORKLOAD)
+                shape = vsa.Shape.of(wl)
+                q, k, v = (x.cuda() for x in workloads.make_qkv(wl))
+                _, peak_tf, _, peak_src = measured_peaks()
+                print(json.dumps(run_cluster_point(args, q, k, v, shape, peak_tf, peak_src,
+                                                   vsa.ClusterParams(256, 512, 2, 0.9))),
+                      flush=True)
         return
     if world > 1:
         import datetime

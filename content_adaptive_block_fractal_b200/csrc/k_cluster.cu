@@ -282,13 +282,20 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restric
   }
 }
 
-// Member means in fp64, token order (the members are contiguous rows of the
-// permuted tensor); an empty cluster keeps its centroid.  A warp per cluster.
+// Member means in fp64 (the members are contiguous rows of the permuted
+// tensor); an empty cluster keeps its centroid.  A warp per cluster: d/8
+// lanes read a row's 16-byte vectors, so a warp covers 256/d rows per step,
+// each lane keeping 8 fp64 column sums; the partial sums of the row classes
+// are added at the end.
+template <int D>
 __global__ void __launch_bounds__(256)
-    centroid_update_kernel(const __nv_bfloat16 *__restrict__ xp, const int32_t *__restrict__ start,
+    centroid_update_kernel(const uint4 *__restrict__ xp, const int32_t *__restrict__ start,
                            const int32_t *__restrict__ count, int64_t BH, int C, int64_t Np,
-                           int d, float *__restrict__ cent) {
+                           float *__restrict__ cent) {
+  constexpr int kLanesPerRow = D / 8;
+  constexpr int kRowsPerStep = 32 / kLanesPerRow;
   const int lane = threadIdx.x & 31;
+  const int sub = lane / kLanesPerRow, col = lane % kLanesPerRow;
   const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   if (w >= BH * C) return;
   const int64_t bh = w / C;
@@ -296,13 +303,25 @@ __global__ void __launch_bounds__(256)
   const int32_t n = count[w];
   if (n == 0) return;
   const int32_t s0 = start[bh * (C + 1) + j];
-  for (int i0 = 0; i0 < d; i0 += 32) {
-    const int i = i0 + lane;
-    if (i >= d) break;
-    double acc = 0.0;
-    for (int32_t m = 0; m < n; ++m)
-      acc += static_cast<double>(__bfloat162float(xp[(bh * Np + s0 + m) * d + i]));
-    cent[w * d + i] = static_cast<float>(acc / n);
+  double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  const uint4 *base = xp + (bh * Np + s0) * kLanesPerRow + col;
+  for (int32_t m = sub; m < n; m += kRowsPerStep) {
+    const uint4 v = __ldg(base + static_cast<int64_t>(m) * kLanesPerRow);
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc[2 * e] += static_cast<double>(__uint_as_float(u[e] << 16));
+      acc[2 * e + 1] += static_cast<double>(__uint_as_float(u[e] & 0xFFFF0000u));
+    }
+  }
+#pragma unroll
+  for (int off = kLanesPerRow; off < 32; off <<= 1)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xFFFFFFFFu, acc[e], off);
+  if (sub == 0) {
+    float *dst = cent + w * D + col * 8;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) dst[e] = static_cast<float>(acc[e] / n);
   }
 }
 
@@ -327,19 +346,25 @@ __global__ void __launch_bounds__(256)
   int n2 = 1;
   while (n2 < Ck) n2 <<= 1;
   const double inv_sqrt_d = 1.0 / sqrt(static_cast<double>(d));
-  double m = -INFINITY;
-  for (int j = threadIdx.x; j < n2; j += blockDim.x) {
+  // a warp per key cluster: coalesced reads of its centroid, fp64 products
+  for (int j = warp; j < n2; j += 8) {
     double a = -INFINITY;
     if (j < Ck && nk[bh * Ck + j] > 0) {
       const float *kr = ck + (bh * Ck + j) * d;
       double dot = 0.0;
-      for (int e = 0; e < d; ++e) dot += s_q[e] * static_cast<double>(kr[e]);
+      for (int e = lane; e < d; e += 32) dot += s_q[e] * static_cast<double>(kr[e]);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) dot += __shfl_xor_sync(0xFFFFFFFFu, dot, o);
       a = dot * inv_sqrt_d;
     }
-    s_a[j] = a;
-    s_j[j] = j;
-    m = fmax(m, a);
+    if (lane == 0) {
+      s_a[j] = a;
+      s_j[j] = j;
+    }
   }
+  __syncthreads();
+  double m = -INFINITY;
+  for (int j = threadIdx.x; j < n2; j += blockDim.x) m = fmax(m, s_a[j]);
 #pragma unroll
   for (int o = 16; o; o >>= 1) m = fmax(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
   if (lane == 0) s_red[warp] = m;
@@ -648,9 +673,15 @@ static cudaError_t run_kmeans(const void *x, const Geometry &g, int C, int iters
                                                                        start, pos, inv, Np);
     gather_rows_kernel<<<grid_for(BH * Np * 32, 256, 32), 256, 0, st>>>(
         static_cast<const uint4 *>(x), inv, BH, N, Np, vec, static_cast<uint4 *>(xp));
-    if (it < iters)
-      centroid_update_kernel<<<static_cast<int>((BH * C * 32 + 255) / 256), 256, 0, st>>>(
-          static_cast<const __nv_bfloat16 *>(xp), start, count, BH, C, Np, d, cent);
+    if (it < iters) {
+      const int ub = static_cast<int>((BH * C * 32 + 255) / 256);
+      if (d == 128)
+        centroid_update_kernel<128><<<ub, 256, 0, st>>>(static_cast<const uint4 *>(xp), start,
+                                                          count, BH, C, Np, cent);
+      else
+        centroid_update_kernel<64><<<ub, 256, 0, st>>>(static_cast<const uint4 *>(xp), start,
+                                                         count, BH, C, Np, cent);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;
