@@ -19,8 +19,10 @@
 //   tile_hist_kernel, tile_scan_kernel, cluster_start_kernel, position_kernel
 //                          a stable counting sort: positions in cluster order,
 //                          token order inside a cluster, 64-aligned starts
-//   gather_rows_kernel     permuted rows (inverse map; padding rows zero)
-//   centroid_update_kernel member means in fp64 in token order
+//   centroid_update_kernel member means in fp64, members read through the
+//                          inverse map of the permutation
+// and after the final assignment gather_rows_kernel (the permuted rows;
+// padding rows zero)
 // and once: centroid_topp_kernel (fp64 estimated attention, sort, top-p),
 // cluster_csr kernels (block CSR + valid keys), the attention launch, and
 // unpermute_kernel (O and LSE back to token order).
@@ -203,10 +205,21 @@ __global__ void tile_scan_kernel(int32_t *__restrict__ hist, int64_t BH, int C, 
   const int64_t bh = i / C;
   const int j = static_cast<int>(i % C);
   int32_t run = 0;
-  for (int tile = 0; tile < ntile; ++tile) {
-    int32_t *p = hist + (bh * ntile + tile) * C + j;
-    const int32_t v = *p;
-    *p = run;
+  int32_t *col = hist + bh * ntile * C + j;
+  int tile = 0;
+  for (; tile + 8 <= ntile; tile += 8) {     // eight loads in flight, then the prefix
+    int32_t v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = col[static_cast<int64_t>(tile + u) * C];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      col[static_cast<int64_t>(tile + u) * C] = run;
+      run += v[u];
+    }
+  }
+  for (; tile < ntile; ++tile) {
+    const int32_t v = col[static_cast<int64_t>(tile) * C];
+    col[static_cast<int64_t>(tile) * C] = run;
     run += v;
   }
   count[i] = run;
@@ -282,16 +295,16 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restric
   }
 }
 
-// Member means in fp64 (the members are contiguous rows of the permuted
-// tensor); an empty cluster keeps its centroid.  A warp per cluster: d/8
+// Member means in fp64, the members read through the inverse map of the
+// permutation (position -> token); an empty cluster keeps its centroid.  A warp per cluster: d/8
 // lanes read a row's 16-byte vectors, so a warp covers 256/d rows per step,
 // each lane keeping 8 fp64 column sums; the partial sums of the row classes
 // are added at the end.
 template <int D>
 __global__ void __launch_bounds__(256)
-    centroid_update_kernel(const uint4 *__restrict__ xp, const int32_t *__restrict__ start,
-                           const int32_t *__restrict__ count, int64_t BH, int C, int64_t Np,
-                           float *__restrict__ cent) {
+    centroid_update_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ inv,
+                           const int32_t *__restrict__ start, const int32_t *__restrict__ count,
+                           int64_t BH, int64_t N, int C, int64_t Np, float *__restrict__ cent) {
   constexpr int kLanesPerRow = D / 8;
   constexpr int kRowsPerStep = 32 / kLanesPerRow;
   const int lane = threadIdx.x & 31;
@@ -304,9 +317,10 @@ __global__ void __launch_bounds__(256)
   if (n == 0) return;
   const int32_t s0 = start[bh * (C + 1) + j];
   double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  const uint4 *base = xp + (bh * Np + s0) * kLanesPerRow + col;
+  const int32_t *members = inv + bh * Np + s0;      // token of each member, in order
+  const uint4 *head = x + bh * N * kLanesPerRow + col;
   for (int32_t m = sub; m < n; m += kRowsPerStep) {
-    const uint4 v = __ldg(base + static_cast<int64_t>(m) * kLanesPerRow);
+    const uint4 v = __ldg(head + static_cast<int64_t>(members[m]) * kLanesPerRow);
     const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -671,16 +685,19 @@ static cudaError_t run_kmeans(const void *x, const Geometry &g, int C, int iters
       return e;
     position_kernel<<<static_cast<int>(BH * L.ntile), kTile, 0, st>>>(label, N, C, L.ntile, hist,
                                                                        start, pos, inv, Np);
-    gather_rows_kernel<<<grid_for(BH * Np * 32, 256, 32), 256, 0, st>>>(
-        static_cast<const uint4 *>(x), inv, BH, N, Np, vec, static_cast<uint4 *>(xp));
     if (it < iters) {
       const int ub = static_cast<int>((BH * C * 32 + 255) / 256);
+      const uint4 *x4 = static_cast<const uint4 *>(x);
       if (d == 128)
-        centroid_update_kernel<128><<<ub, 256, 0, st>>>(static_cast<const uint4 *>(xp), start,
-                                                          count, BH, C, Np, cent);
+        centroid_update_kernel<128><<<ub, 256, 0, st>>>(x4, inv, start, count, BH, N, C, Np,
+                                                          cent);
       else
-        centroid_update_kernel<64><<<ub, 256, 0, st>>>(static_cast<const uint4 *>(xp), start,
-                                                         count, BH, C, Np, cent);
+        centroid_update_kernel<64><<<ub, 256, 0, st>>>(x4, inv, start, count, BH, N, C, Np,
+                                                         cent);
+    } else {
+      // the final permutation: the permuted, padded tensor itself
+      gather_rows_kernel<<<grid_for(BH * Np * 32, 256, 32), 256, 0, st>>>(
+          static_cast<const uint4 *>(x), inv, BH, N, Np, vec, static_cast<uint4 *>(xp));
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
