@@ -141,7 +141,7 @@ __device__ __forceinline__ void decode_item(int item, const AttnArgs &a, int &bh
 // Chunks 0-1 are key block 0 (valid when v0), chunks 2-3 key block 1.
 // `lim` is the number of valid key columns in this chunk (32 unless the key
 // block is a partial one); columns past it get P = 0.
-template <int Q>
+template <int Q, bool kKeyMask>
 __device__ __forceinline__ void softmax_chunk(uint32_t (&cur)[32], uint32_t (&nxt)[32], int nq,
                                               bool v0, bool v1, uint32_t s_addr, float2 c2,
                                               float2 nm2, float2 (&r4)[4], int lim) {
@@ -150,7 +150,7 @@ __device__ __forceinline__ void softmax_chunk(uint32_t (&cur)[32], uint32_t (&nx
   const bool vn = Q + 1 < nq && (Q + 1 < 2 ? v0 : v1);
   if (vn) tmem_ld32_nowait(s_addr + 32 * (Q + 1), nxt);
   uint32_t pk[16];
-  if (vq && lim >= 32) {
+  if (vq && (!kKeyMask || lim >= 32)) {
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const float2 t =
@@ -159,7 +159,7 @@ __device__ __forceinline__ void softmax_chunk(uint32_t (&cur)[32], uint32_t (&nx
       r4[j & 3] = fadd2(r4[j & 3], p);
       pk[j] = pack_bf16x2(p.x, p.y);
     }
-  } else if (vq) {
+  } else if (kKeyMask && vq) {
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const float2 t =
@@ -177,7 +177,9 @@ __device__ __forceinline__ void softmax_chunk(uint32_t (&cur)[32], uint32_t (&nx
   if (vn) tmem_wait_ld_regs(nxt);
 }
 
-template <int D>
+// kKeyMask: key blocks may be partial (per-block valid counts in AttnArgs);
+// the plain instantiation carries no masking code.
+template <int D, bool kKeyMask>
 __global__ void __maxnreg__(168)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tq,
                        const __grid_constant__ CUtensorMap tk,
@@ -351,7 +353,7 @@ __global__ void __maxnreg__(168)
           if (lane == 0) atomicOr(a.err, kErrBadIndex);
           continue;
         }
-        const uint32_t kv = a.kvalid ? static_cast<uint32_t>(a.kvalid[g0 - r0 + c]) & 0x7Fu : 64u;
+        const uint32_t kv = kKeyMask ? static_cast<uint32_t>(a.kvalid[g0 - r0 + c]) & 0x7Fu : 64u;
         if (cur.nb == 0) {
           cur.blk0 = c;
           cur.flags = f | (kv << 8);
@@ -537,7 +539,7 @@ __global__ void __maxnreg__(168)
             float x[64];
             tmem_ld64(s_addr + 64 * h, x);
             const int kv = h ? kv1 : kv0;
-            if (kv < 64) {
+            if (kKeyMask && kv < 64) {
 #pragma unroll
               for (int j = 0; j < 64; ++j) x[j] = j < kv ? x[j] : -INFINITY;
             }
@@ -591,10 +593,10 @@ __global__ void __maxnreg__(168)
           tmem_ld32_nowait(s_addr, xa);
           tmem_wait_ld_regs(xa);
         }
-        softmax_chunk<0>(xa, xb, nq, v0, v1, s_addr, c2, nm2, r4, kv0);
-        softmax_chunk<1>(xb, xa, nq, v0, v1, s_addr, c2, nm2, r4, kv0 - 32);
-        softmax_chunk<2>(xa, xb, nq, v0, v1, s_addr, c2, nm2, r4, kv1);
-        softmax_chunk<3>(xb, xa, nq, v0, v1, s_addr, c2, nm2, r4, kv1 - 32);
+        softmax_chunk<0, kKeyMask>(xa, xb, nq, v0, v1, s_addr, c2, nm2, r4, kv0);
+        softmax_chunk<1, kKeyMask>(xb, xa, nq, v0, v1, s_addr, c2, nm2, r4, kv0 - 32);
+        softmax_chunk<2, kKeyMask>(xa, xb, nq, v0, v1, s_addr, c2, nm2, r4, kv1);
+        softmax_chunk<3, kKeyMask>(xb, xa, nq, v0, v1, s_addr, c2, nm2, r4, kv1 - 32);
       }
       const float rs = ((r4[0].x + r4[0].y) + (r4[1].x + r4[1].y)) +
                        ((r4[2].x + r4[2].y) + (r4[3].x + r4[3].y));
@@ -835,16 +837,22 @@ cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
   int grid = num_sms();
   const int64_t max_items = qblocks ? (n_qblocks < L.items ? n_qblocks : L.items) : L.items;
   if (max_items < grid) grid = static_cast<int>(max_items);
-  const void *fn = g.d == 128 ? reinterpret_cast<const void *>(sparse_attn_kernel<128>)
-                              : reinterpret_cast<const void *>(sparse_attn_kernel<64>);
+  const bool masked = kvalid != nullptr;
+  const void *fn =
+      g.d == 128 ? (masked ? reinterpret_cast<const void *>(sparse_attn_kernel<128, true>)
+                           : reinterpret_cast<const void *>(sparse_attn_kernel<128, false>))
+                 : (masked ? reinterpret_cast<const void *>(sparse_attn_kernel<64, true>)
+                           : reinterpret_cast<const void *>(sparse_attn_kernel<64, false>));
   const int smem = g.d == 128 ? Smem<128>::kAlloc : Smem<64>::kAlloc;
   if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
       cudaSuccess)
     return e;
   if (g.d == 128)
-    sparse_attn_kernel<128><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+    masked ? sparse_attn_kernel<128, true><<<grid, kThreads, smem, st>>>(mq, mk, mv, a)
+           : sparse_attn_kernel<128, false><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
   else
-    sparse_attn_kernel<64><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+    masked ? sparse_attn_kernel<64, true><<<grid, kThreads, smem, st>>>(mq, mk, mv, a)
+           : sparse_attn_kernel<64, false><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     // report what the kernel needs next to what the launch asked for
