@@ -297,7 +297,7 @@ def run_gpu(args, rank, world, local_rank):
         "kept_tiles": kept,
         "breakdown_ms": {"flatten_pool_qk": parts[0], "flatten_v": parts[1], "mask": parts[2],
                          "sparse_attn": parts[3], "unflatten_o": parts[4]},
-        "roofline": {"bound": "tensor", "kernel": "sparse_attn_kernel<128>",
+        "roofline": {"bound": "tensor", "kernel": "sparse_attn_kernel<128, 0>",
                      "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": achieved_tf / peak_tf, "traffic": traffic,
                      "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long loop)",
