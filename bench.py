@@ -477,6 +477,8 @@ def oracle_sample(wl, heads, n_qblocks, seed=0):
     import oracle
     from content_adaptive_block_fractal_b200 import workloads
     oracle.lib()
+    heads = [h for h in heads if h < wl.heads]          # small workloads have fewer
+    n_qblocks = min(n_qblocks, wl.Nb)
     t_perm = t_pool = t_mask = t_attn = 0.0
     kept_total = kept_sampled = 0
     for h in heads:
