@@ -137,6 +137,23 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
+# --------------------------------------------------------------------------- ranks
+def reduce_over_ranks(values, device):
+    """Max over ranks of each device-timed value: the slowest rank sets the
+    job's time.  Every rank calls it, in the same order."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def job_ms_per_layer(ms_max: float, world: int) -> float:
+    """Weak scaling: each of `world` ranks runs one layer in at most ms_max,
+    so the job turns out a layer every ms_max / world."""
+    return ms_max / world
+
+
 # --------------------------------------------------------------------------- GPU arm
 def run_gpu(args, rank, world, local_rank):
     import torch
@@ -271,12 +288,10 @@ def run_gpu(args, rank, world, local_rank):
                "overlap": "H2D, compute and D2H on separate streams, two buffer sets"}
 
     if world > 1:
-        t = torch.tensor([ms, e2e["value"] if e2e else 0.0], device=qd.device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t[0])
+        ms, e2e_max = reduce_over_ranks([ms, e2e["value"] if e2e else 0.0], qd.device)
         if e2e:
-            e2e["value"] = float(t[1]) / world
-    value = ms / world
+            e2e["value"] = job_ms_per_layer(e2e_max, world)
+    value = job_ms_per_layer(ms, world)
     # The attention kernel runs back to back for the whole timed loop and
     # holds the GPU at its power cap, so the sustained GEMM figure (a
     # seconds-long cuBLAS loop under the same cap) is its denominator.
@@ -571,7 +586,8 @@ def main():
     try:
         result, _ = run_gpu(args, rank, world, local_rank)
         if rank == 0:
-            if not args.no_cpu_baseline:
+            # the oracle's CPU baseline is taken at N = 1 only
+            if not args.no_cpu_baseline and world == 1:
                 import oracle
                 wl = __import__("content_adaptive_block_fractal_b200.workloads",
                                 fromlist=["get"]).get(args.workload)
