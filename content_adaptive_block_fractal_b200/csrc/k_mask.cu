@@ -27,6 +27,7 @@
 #include "vsa_internal.h"
 
 #include <cmath>
+#include <type_traits>
 
 namespace vsa {
 namespace {
@@ -121,10 +122,28 @@ __device__ __forceinline__ int prob_bin(uint32_t key) {
   return b < static_cast<uint32_t>(kBins) ? static_cast<int>(b) : kBins;
 }
 
+// A row's probabilities relative to the row maximum: the slab entry (fp32
+// 2^(s - tile max), L2-resident) times its tile's fp32 rescale factor.  Read
+// again wherever a pass needs them rather than kept in SMEM, so that many
+// more rows fit on an SM; the product is the same every time.
+struct RowView {
+  const float *slab;
+  const float *ts;
+  __device__ __forceinline__ float operator()(int c) const { return slab[c] * ts[c / kCT]; }
+};
+// The same values kept in SMEM by the first pass (rows short enough that the
+// copy costs little occupancy).
+struct SmemRow {
+  const float *e;
+  __device__ __forceinline__ float operator()(int c) const { return e[c]; }
+};
+constexpr int kSmemRowMaxNb = 2048;   // rows up to this many blocks stay in SMEM
+
 // The cut by bisection on the fp32 bit pattern, mass tests in fp64.  Sets
 // vkey (cut value) and need_ties, or keep_all when the sums never reach the
 // target.  General path; used when the histogram path cannot decide.
-__device__ void cut_by_bisection(int Nb, const float *ebuf, uint32_t kmax, double target,
+template <class Row>
+__device__ void cut_by_bisection(int Nb, Row ebuf, uint32_t kmax, double target,
                                  uint32_t *cand_key, int32_t *cand_idx, uint32_t &vkey,
                                  int &need_ties, bool &keep_all) {
   const int lane = threadIdx.x & 31;
@@ -137,7 +156,7 @@ __device__ void cut_by_bisection(int Nb, const float *ebuf, uint32_t kmax, doubl
     double up = 0.0;
     if (ncand < 0) {
       for (int c = lane; c < Nb; c += 32) {
-        const float e = ebuf[c];
+        const float e = ebuf(c);
         const uint32_t k = __float_as_uint(e);
         if (k >= mid && k < hi) up += static_cast<double>(e);
       }
@@ -157,7 +176,7 @@ __device__ void cut_by_bisection(int Nb, const float *ebuf, uint32_t kmax, doubl
     if (ncand < 0 && it >= 5) {
       int cnt = 0;
       for (int c = lane; c < Nb; c += 32) {
-        const uint32_t k = __float_as_uint(ebuf[c]);
+        const uint32_t k = __float_as_uint(ebuf(c));
         cnt += (k >= lo && k < hi);
       }
       cnt = warp_sum_i(cnt);
@@ -165,7 +184,7 @@ __device__ void cut_by_bisection(int Nb, const float *ebuf, uint32_t kmax, doubl
         int pos = 0;
         for (int c0 = 0; c0 < Nb; c0 += 32) {
           const int c = c0 + lane;
-          const uint32_t k = c < Nb ? __float_as_uint(ebuf[c]) : 0u;
+          const uint32_t k = c < Nb ? __float_as_uint(ebuf(c)) : 0u;
           const bool in = c < Nb && k >= lo && k < hi;
           const uint32_t m = __ballot_sync(0xFFFFFFFFu, in);
           if (in) {
@@ -193,8 +212,9 @@ __device__ void cut_by_bisection(int Nb, const float *ebuf, uint32_t kmax, doubl
   }
 }
 
-// Phase B for one row: selection and kept bits.  ebuf: this warp's Nb floats.
-//   1. probabilities relative to the row max into ebuf, their fp64 sum, and a
+// Phase B for one row: selection and kept bits.  ebuf: the row's probabilities
+// relative to the row max, re-read from the slab (RowView).
+//   1. those probabilities, their fp64 sum, and a
 //      histogram of counts / fp32 masses over 1/8-octave bins;
 //   2. the bin b where the cumulative mass reaches 1 - thr; an exact fp64 pass
 //      confirms base = mass above b < target <= base + mass of b and collects
@@ -236,8 +256,9 @@ __device__ void finish_row(const MaskArgs &a, int64_t grow, int r, uint32_t *wbi
   __syncwarp();
 }
 
+template <bool kSmemRow>
 __device__ void select_row(const MaskArgs &a, int64_t grow, int r, const float *slab_row,
-                           const double *tmax_row, float *ebuf, uint32_t *cand_key,
+                           const double *tmax_row, float *erow, uint32_t *cand_key,
                            int32_t *cand_idx, float *tscale, int *hcnt, float *hmass,
                            uint32_t *wbits) {
   const int lane = threadIdx.x & 31;
@@ -252,6 +273,9 @@ __device__ void select_row(const MaskArgs &a, int64_t grow, int r, const float *
     hmass[b] = 0.0f;
   }
   __syncwarp();
+  using Row = typename std::conditional<kSmemRow, SmemRow, RowView>::type;
+  Row ebuf;
+  if constexpr (kSmemRow) ebuf = SmemRow{erow}; else ebuf = RowView{slab_row, tscale};
   const bool need_cut = a.thr > 0.0f;
   double z = 0.0;
   uint32_t kmax = 0;
@@ -278,7 +302,7 @@ __device__ void select_row(const MaskArgs &a, int64_t grow, int r, const float *
         const int c = c0 + 128 * u + j;
         if (c < Nb) {
           const float e = e4[j];
-          ebuf[c] = e;
+          if constexpr (kSmemRow) erow[c] = e;
           const uint32_t k = __float_as_uint(e);
           kmax = max(kmax, k);
           if (need_cut) {
@@ -300,7 +324,7 @@ __device__ void select_row(const MaskArgs &a, int64_t grow, int r, const float *
   bool keep_all = !need_cut;
   uint32_t vkey = 0;
   int need_ties = 0;
-  int cut_bin = -1;       // >= 0: kept = bin < cut_bin, or marked in ebuf (sign bit)
+  int cut_bin = -1;       // >= 0: the histogram path wrote the kept bits
   if (!keep_all) {
     const double target = (1.0 - static_cast<double>(a.thr)) * z;
     // 2. cumulative bin masses (8 bins per lane, then a warp scan)
@@ -330,7 +354,7 @@ __device__ void select_row(const MaskArgs &a, int64_t grow, int r, const float *
       int pos = 0;
       for (int c0 = 0; c0 < Nb; c0 += 32) {
         const int c = c0 + lane;
-        const float e = c < Nb ? ebuf[c] : 0.0f;
+        const float e = c < Nb ? ebuf(c) : 0.0f;
         const int b = c < Nb ? prob_bin(__float_as_uint(e)) : kBins;
         if (b < found) base += static_cast<double>(e);
         // entries above the cut bin are kept whatever the bin's order
@@ -399,7 +423,7 @@ __device__ void select_row(const MaskArgs &a, int64_t grow, int r, const float *
   for (int w = 0; cut_bin < 0 && w < a.words; ++w) {
     const int c = w * 32 + lane;
     const bool valid = c < Nb;
-    const uint32_t k = valid ? __float_as_uint(ebuf[c]) : 0u;
+    const uint32_t k = valid ? __float_as_uint(ebuf(c)) : 0u;
     bool kept;
     if (keep_all) {
       kept = valid;
@@ -564,8 +588,9 @@ __global__ void __launch_bounds__(kThreads, 1) mask_scores_kernel(const MaskArgs
 // over that octave's 2^23 patterns (on its members, compacted when there are
 // at most kCand) finds the k-th largest pattern, and equal patterns at the cut
 // are taken in index order.
+template <bool kSmemRow>
 __device__ void select_row_topk(const MaskArgs &a, int64_t grow, int r, const float *slab_row,
-                                const double *tmax_row, float *ebuf, uint32_t *cand_key,
+                                const double *tmax_row, float *erow, uint32_t *cand_key,
                                 int32_t *cand_idx, float *tscale, int *hist, uint32_t *wbits) {
   const int lane = threadIdx.x & 31;
   const int Nb = a.Nb, k = a.k;
@@ -575,10 +600,13 @@ __device__ void select_row_topk(const MaskArgs &a, int64_t grow, int r, const fl
   for (int t = lane; t < a.ntiles; t += 32) tscale[t] = static_cast<float>(exp2(tmax_row[t] - M));
   for (int b = lane; b < kOctaves; b += 32) hist[b] = 0;
   __syncwarp();
+  using Row = typename std::conditional<kSmemRow, SmemRow, RowView>::type;
+  Row ebuf;
+  if constexpr (kSmemRow) ebuf = SmemRow{erow}; else ebuf = RowView{slab_row, tscale};
   const bool keep_all = k >= Nb;
   for (int c = lane; c < Nb; c += 32) {
     const float e = slab_row[c] * tscale[c / kCT];
-    ebuf[c] = e;
+    if constexpr (kSmemRow) erow[c] = e;
     if (!keep_all) atomicAdd(&hist[__float_as_uint(e) >> 23], 1);
   }
   __syncwarp();
@@ -618,7 +646,7 @@ __device__ void select_row_topk(const MaskArgs &a, int64_t grow, int r, const fl
     int pos = 0;
     for (int c0 = 0; c0 < Nb; c0 += 32) {
       const int c = c0 + lane;
-      const int ex = c < Nb ? static_cast<int>(__float_as_uint(ebuf[c]) >> 23) : -1;
+      const int ex = c < Nb ? static_cast<int>(__float_as_uint(ebuf(c)) >> 23) : -1;
       const uint32_t hi_word = __ballot_sync(0xFFFFFFFFu, ex > found);
       if (lane == 0) wbits[c0 >> 5] = hi_word;
       if (compact) {
@@ -626,7 +654,7 @@ __device__ void select_row_topk(const MaskArgs &a, int64_t grow, int r, const fl
         const uint32_t m = __ballot_sync(0xFFFFFFFFu, in);
         if (in) {
           const int p = pos + __popc(m & ((1u << lane) - 1u));
-          cand_key[p] = __float_as_uint(ebuf[c]);
+          cand_key[p] = __float_as_uint(ebuf(c));
           cand_idx[p] = c;
         }
         pos += __popc(m);
@@ -644,7 +672,7 @@ __device__ void select_row_topk(const MaskArgs &a, int64_t grow, int r, const fl
         for (int i = lane; i < pos; i += 32) cin += cand_key[i] >= mid && cand_key[i] < hi;
       } else {
         for (int c = lane; c < Nb; c += 32) {
-          const uint32_t key = __float_as_uint(ebuf[c]);
+          const uint32_t key = __float_as_uint(ebuf(c));
           cin += key >= mid && key < hi;
         }
       }
@@ -680,7 +708,7 @@ __device__ void select_row_topk(const MaskArgs &a, int64_t grow, int r, const fl
     for (int w = 0; w < a.words; ++w) {
       const int c = w * 32 + lane;
       const bool valid = c < Nb;
-      const uint32_t key = valid ? __float_as_uint(ebuf[c]) : 0u;
+      const uint32_t key = valid ? __float_as_uint(ebuf(c)) : 0u;
       bool kept;
       if (keep_all) {
         kept = valid;
@@ -699,49 +727,58 @@ __device__ void select_row_topk(const MaskArgs &a, int64_t grow, int r, const fl
   finish_row(a, grow, r, wbits);
 }
 
+// Per-warp SMEM of the top-p selection: candidates, tile factors, the bin
+// histogram and the kept-bit row.
+__host__ __device__ inline size_t select_warp_bytes(int ntiles, int row_floats) {
+  return (static_cast<size_t>(kCand) * 8 + static_cast<size_t>(ntiles) * 8 + 16 + kBins * 8 +
+          kMaxWords * 4 + static_cast<size_t>(row_floats) * 4 + 15) & ~static_cast<size_t>(15);
+}
+
+template <bool kSmemRow>
 __global__ void __launch_bounds__(kThreads) mask_select_kernel(const MaskArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int warp = threadIdx.x >> 5;
-  unsigned char *wbase = smem_raw + warp * (static_cast<size_t>(a.Nb) * 4 + kCand * 8 +
-                                            static_cast<size_t>(a.ntiles) * 8 + 16 + kBins * 8 +
-                                            kMaxWords * 4);
-  float *ebuf = reinterpret_cast<float *>(wbase);
-  uint32_t *cand_key = reinterpret_cast<uint32_t *>(ebuf + a.Nb);
+  unsigned char *wbase = smem_raw + warp * select_warp_bytes(a.ntiles, kSmemRow ? a.Nb : 0);
+  uint32_t *cand_key = reinterpret_cast<uint32_t *>(wbase);
   int32_t *cand_idx = reinterpret_cast<int32_t *>(cand_key + kCand);
   float *tscale = reinterpret_cast<float *>(
       (reinterpret_cast<uintptr_t>(cand_idx + kCand) + 15) & ~static_cast<uintptr_t>(15));
   int *hcnt = reinterpret_cast<int *>(tscale + a.ntiles);
   float *hmass = reinterpret_cast<float *>(hcnt + kBins);
   uint32_t *wbits = reinterpret_cast<uint32_t *>(hmass + kBins);
+  float *erow = reinterpret_cast<float *>(wbits + kMaxWords);
   const int64_t rows = a.BH * a.Nb;
   for (int64_t g = static_cast<int64_t>(blockIdx.x) * kWarps + warp; g < rows;
        g += static_cast<int64_t>(gridDim.x) * kWarps) {
-    select_row(a, g, static_cast<int>(g % a.Nb), a.slab + g * a.ld_slab, a.tmax + g * a.ntiles,
-               ebuf, cand_key, cand_idx, tscale, hcnt, hmass, wbits);
+    select_row<kSmemRow>(a, g, static_cast<int>(g % a.Nb), a.slab + g * a.ld_slab,
+                         a.tmax + g * a.ntiles, erow, cand_key, cand_idx, tscale, hcnt, hmass,
+                         wbits);
   }
 }
 
 // Per-warp SMEM of the static-ratio selection (all 4-byte fields).
-__host__ __device__ inline size_t topk_warp_bytes(int Nb, int ntiles) {
-  return (static_cast<size_t>(Nb + 2 * kCand + ntiles + kOctaves + kMaxWords) * 4 + 15) &
+__host__ __device__ inline size_t topk_warp_bytes(int ntiles, int row_floats) {
+  return (static_cast<size_t>(2 * kCand + ntiles + kOctaves + kMaxWords + row_floats) * 4 + 15) &
          ~static_cast<size_t>(15);
 }
 
+template <bool kSmemRow>
 __global__ void __launch_bounds__(kThreads) mask_select_topk_kernel(const MaskArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int warp = threadIdx.x >> 5;
-  unsigned char *wbase = smem_raw + warp * topk_warp_bytes(a.Nb, a.ntiles);
-  float *ebuf = reinterpret_cast<float *>(wbase);
-  uint32_t *cand_key = reinterpret_cast<uint32_t *>(ebuf + a.Nb);
+  unsigned char *wbase = smem_raw + warp * topk_warp_bytes(a.ntiles, kSmemRow ? a.Nb : 0);
+  uint32_t *cand_key = reinterpret_cast<uint32_t *>(wbase);
   int32_t *cand_idx = reinterpret_cast<int32_t *>(cand_key + kCand);
   float *tscale = reinterpret_cast<float *>(cand_idx + kCand);
   int *hist = reinterpret_cast<int *>(tscale + a.ntiles);
   uint32_t *wbits = reinterpret_cast<uint32_t *>(hist + kOctaves);
+  float *erow = reinterpret_cast<float *>(wbits + kMaxWords);
   const int64_t rows = a.BH * a.Nb;
   for (int64_t g = static_cast<int64_t>(blockIdx.x) * kWarps + warp; g < rows;
        g += static_cast<int64_t>(gridDim.x) * kWarps) {
-    select_row_topk(a, g, static_cast<int>(g % a.Nb), a.slab + g * a.ld_slab,
-                    a.tmax + g * a.ntiles, ebuf, cand_key, cand_idx, tscale, hist, wbits);
+    select_row_topk<kSmemRow>(a, g, static_cast<int>(g % a.Nb), a.slab + g * a.ld_slab,
+                              a.tmax + g * a.ntiles, erow, cand_key, cand_idx, tscale, hist,
+                              wbits);
   }
 }
 
@@ -827,10 +864,9 @@ MaskLayout mask_layout(const Geometry &g, int grid) {
   off = align256(off + static_cast<size_t>(g.BH * g.Nb) * 4);
   L.total = off;
   L.smem_a = (static_cast<size_t>(kRT) * (g.d + kPad) + 2 * static_cast<size_t>(kCT) * kLdK) * 8;
-  L.smem_b = static_cast<size_t>(kWarps) *
-             (static_cast<size_t>(g.Nb) * 4 + kCand * 8 + L.ntiles * 8 + 16 + kBins * 8 +
-              kMaxWords * 4);
-  L.smem_k = static_cast<size_t>(kWarps) * topk_warp_bytes(static_cast<int>(g.Nb), L.ntiles);
+  const int row_floats = g.Nb <= kSmemRowMaxNb ? static_cast<int>(g.Nb) : 0;
+  L.smem_b = static_cast<size_t>(kWarps) * select_warp_bytes(L.ntiles, row_floats);
+  L.smem_k = static_cast<size_t>(kWarps) * topk_warp_bytes(L.ntiles, row_floats);
   L.smem = L.smem_a > L.smem_b ? L.smem_a : L.smem_b;
   if (L.smem_k > L.smem) L.smem = L.smem_k;
   if (L.words > kMaxWords) L.smem = ~static_cast<size_t>(0) >> 1;  // reported as unsupported
@@ -881,17 +917,21 @@ cudaError_t launch_block_mask(const double *qp, const double *kp, const Geometry
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int64_t sel_blocks = (rows + kWarps - 1) / kWarps;
   const int sel_grid = static_cast<int>(sel_blocks < 64LL * num_sms() ? sel_blocks : 64LL * num_sms());
+  const bool smem_row = g.Nb <= kSmemRowMaxNb;
+  const void *sel = topk > 0 ? (smem_row ? reinterpret_cast<const void *>(mask_select_topk_kernel<true>)
+                                         : reinterpret_cast<const void *>(mask_select_topk_kernel<false>))
+                             : (smem_row ? reinterpret_cast<const void *>(mask_select_kernel<true>)
+                                         : reinterpret_cast<const void *>(mask_select_kernel<false>));
+  const size_t sel_smem = topk > 0 ? L.smem_k : L.smem_b;
+  if ((e = cudaFuncSetAttribute(sel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(sel_smem))) != cudaSuccess)
+    return e;
   if (topk > 0) {
-    if ((e = cudaFuncSetAttribute(mask_select_topk_kernel,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  static_cast<int>(L.smem_k))) != cudaSuccess)
-      return e;
-    mask_select_topk_kernel<<<sel_grid, kThreads, L.smem_k, st>>>(a);
+    if (smem_row) mask_select_topk_kernel<true><<<sel_grid, kThreads, sel_smem, st>>>(a);
+    else mask_select_topk_kernel<false><<<sel_grid, kThreads, sel_smem, st>>>(a);
   } else {
-    if ((e = cudaFuncSetAttribute(mask_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  static_cast<int>(L.smem_b))) != cudaSuccess)
-      return e;
-    mask_select_kernel<<<sel_grid, kThreads, L.smem_b, st>>>(a);
+    if (smem_row) mask_select_kernel<true><<<sel_grid, kThreads, sel_smem, st>>>(a);
+    else mask_select_kernel<false><<<sel_grid, kThreads, sel_smem, st>>>(a);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   scan_counts_kernel<<<1, 1024, 0, st>>>(a.counts, rows, row_ptr);
