@@ -16,7 +16,8 @@
 //                       mass tests), breaks ties by index, ORs in the STA
 //                       window and writes a kept-bit row and its count.  Small
 //                       SMEM per warp, so many rows are in flight per SM.
-//   scan_counts_kernel  exclusive scan of the counts into row_ptr (int64).
+//   chunk_sums_kernel, chunk_scan_kernel
+//                       exclusive scan of the counts into row_ptr (int64).
 //   expand_bits_kernel  kept bits -> ascending col_idx lists.
 //
 // Precision: scores are exact fp64 dot products of exact pooled means; each
@@ -783,16 +784,47 @@ __global__ void __launch_bounds__(kThreads) mask_select_topk_kernel(const MaskAr
 }
 
 // Exclusive scan of n counts into row_ptr[0..n] by one CTA of 1024 threads.
-__global__ void __launch_bounds__(1024) scan_counts_kernel(const int32_t *__restrict__ counts,
-                                                           int64_t n,
-                                                           int64_t *__restrict__ row_ptr) {
+// Exclusive scan of the kept counts into row_ptr in two launches: per-chunk
+// sums of kScanChunk rows, then every chunk adds up the sums before it (at
+// most a few hundred) and scans its own rows.  Coalesced, no serial walk.
+constexpr int kScanChunk = 1024;
+
+__global__ void __launch_bounds__(kScanChunk) chunk_sums_kernel(const int32_t *__restrict__ counts,
+                                                                int64_t n,
+                                                                int64_t *__restrict__ sums) {
   __shared__ int64_t warp_tot[32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t per = (n + 1023) / 1024;
-  const int64_t b = tid * per, e = b + per < n ? b + per : n;
-  int64_t s = 0;
-  for (int64_t i = b; i < e; ++i) s += counts[i];
-  int64_t x = s;  // inclusive warp scan
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * kScanChunk + threadIdx.x;
+  int64_t v = i < n ? counts[i] : 0;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  if (lane == 0) warp_tot[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int64_t w = warp_tot[lane];
+#pragma unroll
+    for (int o = 16; o; o >>= 1) w += __shfl_xor_sync(0xFFFFFFFFu, w, o);
+    if (lane == 0) sums[blockIdx.x] = w;
+  }
+}
+
+__global__ void __launch_bounds__(kScanChunk) chunk_scan_kernel(const int32_t *__restrict__ counts,
+                                                                int64_t n,
+                                                                const int64_t *__restrict__ sums,
+                                                                int64_t *__restrict__ row_ptr) {
+  __shared__ int64_t warp_tot[32];
+  __shared__ int64_t base;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (warp == 0) {                 // sum of the chunks before this one
+    int64_t b = 0;
+    for (int c = lane; c < static_cast<int>(blockIdx.x); c += 32) b += sums[c];
+#pragma unroll
+    for (int o = 16; o; o >>= 1) b += __shfl_xor_sync(0xFFFFFFFFu, b, o);
+    if (lane == 0) base = b;
+  }
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * kScanChunk + threadIdx.x;
+  const int64_t v = i < n ? counts[i] : 0;
+  int64_t x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int64_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
@@ -810,14 +842,14 @@ __global__ void __launch_bounds__(1024) scan_counts_kernel(const int32_t *__rest
     warp_tot[lane] = w;
   }
   __syncthreads();
-  int64_t run = x - s + (warp ? warp_tot[warp - 1] : 0);
-  for (int64_t i = b; i < e; ++i) {
-    row_ptr[i] = run;
-    run += counts[i];
-  }
-  if (tid == 1023) row_ptr[n] = warp_tot[31];
+  const int64_t incl = base + x + (warp ? warp_tot[warp - 1] : 0);
+  if (i < n) row_ptr[i] = incl - v;
+  if (i == n - 1) row_ptr[n] = incl;
 }
 
+// Kept bits -> ascending column lists.  A warp per row, a lane per 32-bit
+// word: the words' popcounts, a warp scan for their offsets, then each lane
+// writes its own word's set bits in order.
 __global__ void __launch_bounds__(256) expand_bits_kernel(const uint32_t *__restrict__ bits,
                                                           int words, int64_t rows,
                                                           const int64_t *__restrict__ row_ptr,
@@ -829,12 +861,22 @@ __global__ void __launch_bounds__(256) expand_bits_kernel(const uint32_t *__rest
     int64_t pos = row_ptr[r];
     const uint32_t *rb = bits + r * words;
     for (int w0 = 0; w0 < words; w0 += 32) {
-      const uint32_t mine = w0 + lane < words ? rb[w0 + lane] : 0u;
-      for (int i = 0; i < 32 && w0 + i < words; ++i) {
-        const uint32_t word = __shfl_sync(0xFFFFFFFFu, mine, i);
-        if ((word >> lane) & 1u) col_idx[pos + __popc(word & ((1u << lane) - 1u))] = (w0 + i) * 32 + lane;
-        pos += __popc(word);
+      const int w = w0 + lane;
+      uint32_t word = w < words ? rb[w] : 0u;
+      const int n = __popc(word);
+      int incl = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
       }
+      int32_t *dst = col_idx + pos + (incl - n);
+      while (word) {
+        const int b = __ffs(word) - 1;
+        *dst++ = w * 32 + b;
+        word &= word - 1u;
+      }
+      pos += __shfl_sync(0xFFFFFFFFu, incl, 31);
     }
   }
 }
@@ -934,7 +976,13 @@ cudaError_t launch_block_mask(const double *qp, const double *kp, const Geometry
     else mask_select_kernel<false><<<sel_grid, kThreads, sel_smem, st>>>(a);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  scan_counts_kernel<<<1, 1024, 0, st>>>(a.counts, rows, row_ptr);
+  {
+    // chunk sums go to the start of the slab: the selection is done with it
+    int64_t *sums = reinterpret_cast<int64_t *>(a.slab);
+    const int chunks = static_cast<int>((rows + kScanChunk - 1) / kScanChunk);
+    chunk_sums_kernel<<<chunks, kScanChunk, 0, st>>>(a.counts, rows, sums);
+    chunk_scan_kernel<<<chunks, kScanChunk, 0, st>>>(a.counts, rows, sums, row_ptr);
+  }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int64_t want = (rows + 7) / 8;
   const int eg = static_cast<int>(want < 16LL * num_sms() ? want : 16LL * num_sms());
