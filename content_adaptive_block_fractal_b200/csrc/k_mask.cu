@@ -108,13 +108,6 @@ __device__ __forceinline__ float exp2_split(double x) {
   return ex2(f) * __int_as_float((static_cast<int>(n) + 127) << 23);
 }
 
-__device__ __forceinline__ bool sta_keep(int r, int c, const MaskArgs &a) {
-  const int hw = a.Hb * a.Wb;
-  const int tr = r / hw, yr = (r / a.Wb) % a.Hb, xr = r % a.Wb;
-  const int tc = c / hw, yc = (c / a.Wb) % a.Hb, xc = c % a.Wb;
-  return abs(tr - tc) <= a.rt && abs(yr - yc) <= a.rh && abs(xr - xc) <= a.rw;
-}
-
 // key = bits of a probability in [0, 1]; bin 0 holds (7/8, 1], each bin is
 // 1/8 octave; kBins (the tail) collects everything more than 8 octaves down.
 __device__ __forceinline__ int prob_bin(uint32_t key) {
