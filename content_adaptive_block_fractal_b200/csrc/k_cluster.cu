@@ -747,7 +747,6 @@ cudaError_t launch_cluster_attn(const void *q, const void *k, const void *v, con
   gather_rows_kernel<<<grid_for(BH * Np * 32, 256, 32), 256, 0, st>>>(
       static_cast<const uint4 *>(v), inv, BH, N, Np, d / 8, reinterpret_cast<uint4 *>(w + L.xv));
   // the centroids that the final labels were assigned with
-  const int32_t *count_q = reinterpret_cast<const int32_t *>(w + L.count_q);
   const int32_t *count_k = reinterpret_cast<const int32_t *>(w + L.count_k);
   const int32_t *start_q = reinterpret_cast<const int32_t *>(w + L.start_q);
   const int32_t *start_k = reinterpret_cast<const int32_t *>(w + L.start_k);
