@@ -175,9 +175,9 @@ def run_gpu(args, rank, world, local_rank):
     o_raster = torch.empty_like(qd)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=qd.device)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
-    # flatten+pool of Q,K; flatten of V; mask (scores, select, scan, expand);
-    # plan + attention; unflatten of O
-    launches_per_step = 1 + 1 + 4 + 2 + 1
+    # flatten+pool of Q,K; flatten of V; mask (scores, select, chunk sums,
+    # chunk scan, expand); plan + attention; unflatten of O
+    launches_per_step = 1 + 1 + 5 + 2 + 1
 
     def step(record=False):
         if record: ev[0].record(stream)
