@@ -35,8 +35,10 @@ WORKLOAD = "wan14b-720p"
 METRIC = "ms/attention layer and kept-tile TFLOP/s at Wan-14B 720p shape, thr=0.1"
 UNIT = "ms/layer"
 L2_FLUSH_BYTES = 256 << 20
-PROFILE = os.path.join(ROOT, "profiles", "sparse_attn_fwd_wan14b.md")
-# files whose contents make up the attention kernel (hashed against PROFILE)
+# ncu DRAM summaries of the attention launch in each layout
+PROFILES = {lay: os.path.join(ROOT, "profiles", f"sparse_attn_fwd_{lay}_wan14b-720p.md")
+            for lay in ("raster", "flat")}
+# files whose contents make up the attention kernel (hashed against the summary)
 ATTN_SOURCES = [os.path.join(ROOT, "content_adaptive_block_fractal_b200", "csrc", f)
                 for f in ("k_attn.cu", "vsa_device.cuh")]
 
@@ -50,6 +52,9 @@ def parse_args():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layout", default="flat", choices=["flat", "raster"],
+                    help="raster: the kernels gather the fractal blocks from raster q, k, v "
+                         "and write raster o; flat: explicit flatten / unflatten passes")
     ap.add_argument("--cluster", action="store_true",
                     help="only the semantic-aware permutation path at the Wan-14B 720p shape")
     ap.add_argument("--sweep", action="store_true",
@@ -76,11 +81,11 @@ def kernel_source_hash(paths) -> str:
     return h.hexdigest()
 
 
-def profile_traffic(kernel_srcs):
+def profile_traffic(kernel_srcs, profile):
     """DRAM bytes per attention launch from the committed ncu summary, if it was
     taken on the current kernel source (same hash of the kernel's files); else None."""
     try:
-        text = open(PROFILE).read()
+        text = open(profile).read()
     except OSError:
         return None
     h = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
@@ -170,33 +175,54 @@ def run_gpu(args, rank, world, local_rank):
     qh, kh, vh = (x.pin_memory() for x in (q, k, v))
     qd, kd, vd = (x.cuda() for x in (qh, kh, vh))
     stream = torch.cuda.current_stream()
-    qf, kf, vf = (torch.empty_like(qd) for _ in range(3))
-    layer = vsa.Layer(shape, params, qd.device)
-    o_raster = torch.empty_like(qd)
+    raster = args.layout == "raster"
+    layer = vsa.Layer(shape, params, qd.device, layout=args.layout)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=qd.device)
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
-    # flatten+pool of Q,K; flatten of V; mask (scores, select, chunk sums,
-    # chunk scan, expand); plan + attention; unflatten of O
-    launches_per_step = 1 + 1 + 5 + 2 + 1
+    csr, o, lse = layer.csr, layer.o, layer.lse
+    if raster:
+        # pool straight from raster; the attention gathers each fractal block
+        # with one patch-shaped TMA box and writes O and LSE in raster order
+        o_raster = o
+        stages = [
+            ("pool_qk", lambda x: vsa.pool_qk_raster(x[0], x[1], shape, out=(layer.qp, layer.kp))),
+            ("mask", lambda x: vsa.block_mask(layer.qp, layer.kp, shape, params, out=csr,
+                                              workspace=layer.ws_mask)),
+            ("sparse_attn", lambda x: vsa.sparse_attn_fwd_raster(
+                x[0], x[1], x[2], csr.row_ptr, csr.col_idx, shape, 0.0, out=(o, lse),
+                workspace=layer.ws_attn)),
+        ]
+        # pool; mask (scores, select, chunk sums, chunk scan, expand); plan + attention
+        launches_per_step = 1 + 5 + 2
+    else:
+        qf, kf, vf = (torch.empty_like(qd) for _ in range(3))
+        o_raster = torch.empty_like(qd)
+        stages = [
+            ("flatten_pool_qk", lambda x: vsa.flatten_pool_qk(x[0], x[1], shape,
+                                                              out=(qf, kf, layer.qp, layer.kp))),
+            ("flatten_v", lambda x: vsa.fractal_flatten(x[2], shape, out=vf)),
+            ("mask", lambda x: vsa.block_mask(layer.qp, layer.kp, shape, params, out=csr,
+                                              workspace=layer.ws_mask)),
+            ("sparse_attn", lambda x: vsa.sparse_attn_fwd(
+                qf, kf, vf, csr.row_ptr, csr.col_idx, shape, 0.0, out=(o, lse),
+                workspace=layer.ws_attn)),
+            ("unflatten_o", lambda x: vsa.fractal_unflatten(o, shape, out=o_raster)),
+        ]
+        # flatten+pool of Q,K; flatten of V; mask (5); plan + attention; unflatten of O
+        launches_per_step = 1 + 1 + 5 + 2 + 1
+    n_st = len(stages)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_st + 1)]
+    inputs = (qd, kd, vd)
 
     def step(record=False):
         if record: ev[0].record(stream)
-        vsa.flatten_pool_qk(qd, kd, shape, out=(qf, kf, layer.qp, layer.kp))
-        if record: ev[1].record(stream)
-        vsa.fractal_flatten(vd, shape, out=vf)
-        if record: ev[2].record(stream)
-        vsa.block_mask(layer.qp, layer.kp, shape, params, out=layer.csr, workspace=layer.ws_mask)
-        if record: ev[3].record(stream)
-        vsa.sparse_attn_fwd(qf, kf, vf, layer.csr.row_ptr, layer.csr.col_idx, shape, 0.0,
-                            out=(layer.o, layer.lse), workspace=layer.ws_attn)
-        if record: ev[4].record(stream)
-        vsa.fractal_unflatten(layer.o, shape, out=o_raster)
-        if record: ev[5].record(stream)
+        for i, (_, fn) in enumerate(stages):
+            fn(inputs)
+            if record: ev[i + 1].record(stream)
 
     for _ in range(args.warmup):
         step()
     vsa.device_status()
-    kept = int(layer.csr.row_ptr[-1].item())
+    kept = int(csr.row_ptr[-1].item())
     rows = shape.B * shape.heads * shape.Nb
     kept_frac = kept / (rows * shape.Nb)
     flop_per_tile = 4 * 64 * 64 * shape.d
@@ -206,20 +232,19 @@ def run_gpu(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    parts = np.zeros(5)
+    parts = np.zeros(n_st)
     total = 0.0
     with ClockSampler(local_rank) as clk:
         for _ in range(args.steps):
             flush.zero_()
             step(record=True)
-            ev[5].synchronize()
-            t = [ev[i].elapsed_time(ev[i + 1]) for i in range(5)]
-            parts += t
-            total += ev[0].elapsed_time(ev[5])
+            ev[n_st].synchronize()
+            parts += [ev[i].elapsed_time(ev[i + 1]) for i in range(n_st)]
+            total += ev[0].elapsed_time(ev[n_st])
     torch.cuda.synchronize()
     vsa.device_status()
     ms = total / args.steps
-    parts /= args.steps
+    parts = {name: t / args.steps for (name, _), t in zip(stages, parts)}
 
     # end to end through the public API with host buffers: every step copies
     # its raster Q, K, V in from pinned memory and its O and LSE back out.
@@ -231,13 +256,13 @@ def run_gpu(args, rank, world, local_rank):
         n_e2e = max(3, min(args.steps, 10))
         ins = [(qd, kd, vd), tuple(torch.empty_like(qd) for _ in range(3))]
         outs_o = [o_raster, torch.empty_like(o_raster)]
-        outs_l = [torch.empty_like(layer.lse) for _ in range(2)]
+        outs_l = [torch.empty_like(lse) for _ in range(2)]
         o_host = [torch.empty(qh.shape, dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
-        l_host = [torch.empty(layer.lse.shape, dtype=torch.float32, pin_memory=True)
+        l_host = [torch.empty(lse.shape, dtype=torch.float32, pin_memory=True)
                   for _ in range(2)]
         s_h2d, s_d2h = torch.cuda.Stream(), torch.cuda.Stream()
         ev_in = [torch.cuda.Event() for _ in range(2)]     # inputs landed
-        ev_used = [torch.cuda.Event() for _ in range(2)]   # inputs flattened (buffer free)
+        ev_used = [torch.cuda.Event() for _ in range(2)]   # inputs consumed (buffer free)
         ev_out = [torch.cuda.Event() for _ in range(2)]    # outputs written
         ev_read = [torch.cuda.Event() for _ in range(2)]   # outputs copied out (buffer free)
 
@@ -251,16 +276,26 @@ def run_gpu(args, rank, world, local_rank):
                 ev_in[b].record(s_h2d)
                 stream.wait_event(ev_in[b])
                 qx, kx, vx = ins[b]
-                vsa.flatten_pool_qk(qx, kx, shape, out=(qf, kf, layer.qp, layer.kp))
-                vsa.fractal_flatten(vx, shape, out=vf)
-                ev_used[b].record(stream)
-                vsa.block_mask(layer.qp, layer.kp, shape, params, out=layer.csr,
-                               workspace=layer.ws_mask)
-                vsa.sparse_attn_fwd(qf, kf, vf, layer.csr.row_ptr, layer.csr.col_idx, shape,
-                                    0.0, out=(layer.o, layer.lse), workspace=layer.ws_attn)
-                stream.wait_event(ev_read[b])
-                vsa.fractal_unflatten(layer.o, shape, out=outs_o[b])
-                outs_l[b].copy_(layer.lse)
+                if raster:
+                    vsa.pool_qk_raster(qx, kx, shape, out=(layer.qp, layer.kp))
+                    vsa.block_mask(layer.qp, layer.kp, shape, params, out=csr,
+                                   workspace=layer.ws_mask)
+                    stream.wait_event(ev_read[b])
+                    vsa.sparse_attn_fwd_raster(qx, kx, vx, csr.row_ptr, csr.col_idx, shape, 0.0,
+                                               out=(outs_o[b], outs_l[b]),
+                                               workspace=layer.ws_attn)
+                    ev_used[b].record(stream)
+                else:
+                    vsa.flatten_pool_qk(qx, kx, shape, out=(qf, kf, layer.qp, layer.kp))
+                    vsa.fractal_flatten(vx, shape, out=vf)
+                    ev_used[b].record(stream)
+                    vsa.block_mask(layer.qp, layer.kp, shape, params, out=csr,
+                                   workspace=layer.ws_mask)
+                    vsa.sparse_attn_fwd(qf, kf, vf, csr.row_ptr, csr.col_idx, shape,
+                                        0.0, out=(o, lse), workspace=layer.ws_attn)
+                    stream.wait_event(ev_read[b])
+                    vsa.fractal_unflatten(o, shape, out=outs_o[b])
+                    outs_l[b].copy_(lse)
                 ev_out[b].record(stream)
                 s_d2h.wait_event(ev_out[b])
                 with torch.cuda.stream(s_d2h):
@@ -296,22 +331,34 @@ def run_gpu(args, rank, world, local_rank):
     # holds the GPU at its power cap, so the sustained GEMM figure (a
     # seconds-long cuBLAS loop under the same cap) is its denominator.
     burst_tf, peak_tf, peak_gbs, peak_src = measured_peaks()
-    attn_ms = parts[3]
+    attn_ms = parts["sparse_attn"]
     achieved_tf = kept_flop / (attn_ms * 1e-3) / 1e12
-    traffic = profile_traffic(ATTN_SOURCES)
+    traffic = profile_traffic(ATTN_SOURCES, PROFILES[args.layout])
+    pooled_bytes = 2 * rows * shape.d * 8
+    if raster:
+        # pooling reads Q and K and writes the means; nothing else moves
+        hbm = {"pool_qk": (2 * tensor_bytes + pooled_bytes) / (parts["pool_qk"] * 1e-3) / 1e9}
+        step_desc = ("pool q,k + mask + sparse attention on raster q,k,v -> raster o,lse "
+                     "(the fractal order is applied by the kernels' addressing)")
+    else:
+        hbm = {"flatten_pool_qk": (4 * tensor_bytes + pooled_bytes)
+               / (parts["flatten_pool_qk"] * 1e-3) / 1e9,
+               "flatten_v": 2 * tensor_bytes / (parts["flatten_v"] * 1e-3) / 1e9,
+               "unflatten_o": 2 * tensor_bytes / (parts["unflatten_o"] * 1e-3) / 1e9}
+        step_desc = "flatten q,k,v + pool + mask + sparse attention + unflatten o"
+    hbm["peak"] = peak_gbs
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {**wl.describe(), "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": "256 MiB flush written between timed steps; Q/K/V 2.5 GB > L2",
-                   "step": "flatten q,k,v + pool + mask + sparse attention + unflatten o"},
+                   "layout": args.layout, "step": step_desc},
         "kept_tile_tflops": achieved_tf,
         "kept_tile_tflops_layer": kept_flop / (ms * 1e-3) / 1e12,
         "kept_fraction": kept_frac,
         "kept_tiles": kept,
-        "breakdown_ms": {"flatten_pool_qk": parts[0], "flatten_v": parts[1], "mask": parts[2],
-                         "sparse_attn": parts[3], "unflatten_o": parts[4]},
+        "breakdown_ms": parts,
         "roofline": {"bound": "tensor", "kernel": "sparse_attn_kernel<128, 0>",
                      "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": achieved_tf / peak_tf, "traffic": traffic,
@@ -319,11 +366,7 @@ def run_gpu(args, rank, world, local_rank):
                      "frac_of_burst": achieved_tf / burst_tf,
                      "flop_per_kept_tile": flop_per_tile},
         # HBM kernels: algorithmic bytes / time (read + write, each byte once)
-        "hbm_gbs": {"flatten_pool_qk": (4 * tensor_bytes + 2 * rows * shape.d * 8)
-                    / (parts[0] * 1e-3) / 1e9,
-                    "flatten_v": 2 * tensor_bytes / (parts[1] * 1e-3) / 1e9,
-                    "unflatten_o": 2 * tensor_bytes / (parts[4] * 1e-3) / 1e9,
-                    "peak": peak_gbs},
+        "hbm_gbs": hbm,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }

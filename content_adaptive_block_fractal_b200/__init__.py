@@ -19,7 +19,7 @@ from . import _lib
 from ._lib import VsaError, vsa_mask_params, vsa_shape
 
 __all__ = ["Shape", "MaskParams", "VsaError", "fractal_flatten", "fractal_unflatten",
-           "flatten_pool_qk",
+           "flatten_pool_qk", "pool_qk_raster", "sparse_attn_fwd_raster", "Layer",
            "pool_qk", "block_mask", "block_mask_topk", "sta_mask", "sta_mask_nnz",
            "block_mask_workspace_size", "sparse_attn_fwd", "sparse_attn_fwd_rows",
            "ClusterParams", "cluster_attention", "cluster_attn_workspace_size",
@@ -128,6 +128,20 @@ def flatten_pool_qk(q: torch.Tensor, k: torch.Tensor, shape: Shape, out=None, st
     return qf, kf, qp, kp
 
 
+def pool_qk_raster(q: torch.Tensor, k: torch.Tensor, shape: Shape, out=None, stream=None):
+    """64-token block means of the fractal blocks read straight from raster Q
+    and K -> (qp, kp); identical to the means of flatten_pool_qk, with no
+    flattened copy written."""
+    if out is None:
+        sz = (shape.B, shape.heads, shape.Nb, shape.d)
+        out = (torch.empty(sz, dtype=torch.float64, device=q.device),
+               torch.empty(sz, dtype=torch.float64, device=q.device))
+    qp, kp = out
+    _lib.check(_lib.load().vsa_pool_qk_raster(_ptr(q), _ptr(k), _ptr(qp), _ptr(kp), shape.c(),
+                                              _stream(stream)))
+    return qp, kp
+
+
 def block_mask_workspace_size(shape: Shape) -> int:
     return int(_lib.load().vsa_block_mask_workspace_size(shape.c()))
 
@@ -219,6 +233,23 @@ def sparse_attn_fwd(qf, kf, vf, row_ptr, col_idx, shape: Shape, scale: float = 0
     return o, lse
 
 
+def sparse_attn_fwd_raster(q, k, v, row_ptr, col_idx, shape: Shape, scale: float = 0.0,
+                           out=None, workspace=None, stream=None):
+    """sparse_attn_fwd on raster-order q, k, v -> raster-order (o, lse); the
+    mask still indexes fractal blocks.  Equals flattening, sparse_attn_fwd and
+    unflattening, bit for bit, without the permuted copies."""
+    if out is None:
+        out = (torch.empty_like(q),
+               torch.empty((shape.B, shape.heads, shape.N), dtype=torch.float32, device=q.device))
+    o, lse = out
+    if workspace is None:
+        workspace = _workspace(sparse_attn_workspace_size(shape), q.device)
+    _lib.check(_lib.load().vsa_sparse_attn_fwd_raster(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr), _ptr(col_idx), shape.c(), float(scale),
+        _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return o, lse
+
+
 def sparse_attn_fwd_rows(qf, kf, vf, row_ptr, col_idx, shape: Shape, qblocks: torch.Tensor,
                          scale: float = 0.0, out=None, workspace=None, stream=None):
     """Attention for the listed query blocks only (int32 global block rows,
@@ -301,10 +332,17 @@ def device_status(stream=None) -> None:
 
 
 class Layer:
-    """Preallocated buffers for one attention layer: pool, mask, sparse attention."""
+    """Preallocated buffers for one attention layer: pool, mask, sparse attention.
 
-    def __init__(self, shape: Shape, params: MaskParams, device="cuda", scale: float = 0.0):
-        self.shape, self.params, self.scale = shape, params, scale
+    layout "flat": q, k, v, o and lse in fractal-flattened token order;
+    "raster": in raster order (the fractal blocks are gathered by the kernels'
+    own addressing, so no permuted copy is made)."""
+
+    def __init__(self, shape: Shape, params: MaskParams, device="cuda", scale: float = 0.0,
+                 layout: str = "flat"):
+        if layout not in ("flat", "raster"):
+            raise ValueError(f"layout must be 'flat' or 'raster', not {layout!r}")
+        self.shape, self.params, self.scale, self.layout = shape, params, scale, layout
         B, h, Nb, d, N = shape.B, shape.heads, shape.Nb, shape.d, shape.N
         f64 = dict(dtype=torch.float64, device=device)
         self.qp = torch.empty((B, h, Nb, d), **f64)
@@ -318,12 +356,15 @@ class Layer:
         self.o = torch.empty((B, h, N, d), dtype=torch.bfloat16, device=device)
         self.lse = torch.empty((B, h, N), dtype=torch.float32, device=device)
 
-    def __call__(self, qf, kf, vf, stream=None):
-        pool_qk(qf, kf, self.shape, out=(self.qp, self.kp), stream=stream)
+    def __call__(self, q, k, v, stream=None):
+        raster = self.layout == "raster"
+        (pool_qk_raster if raster else pool_qk)(q, k, self.shape, out=(self.qp, self.kp),
+                                                stream=stream)
         block_mask(self.qp, self.kp, self.shape, self.params, out=self.csr,
                    workspace=self.ws_mask, stream=stream)
-        sparse_attn_fwd(qf, kf, vf, self.csr.row_ptr, self.csr.col_idx, self.shape,
-                        self.scale, out=(self.o, self.lse), workspace=self.ws_attn, stream=stream)
+        (sparse_attn_fwd_raster if raster else sparse_attn_fwd)(
+            q, k, v, self.csr.row_ptr, self.csr.col_idx, self.shape, self.scale,
+            out=(self.o, self.lse), workspace=self.ws_attn, stream=stream)
         return self.o, self.lse
 
 

@@ -18,11 +18,12 @@ STATUS_NAMES = {0: "VSA_OK", 1: "VSA_ERR_INVALID_ARG", 2: "VSA_ERR_UNSUPPORTED",
 
 # Every symbol include/vsa.h declares.
 EXPORTS = ("vsa_fractal_flatten", "vsa_fractal_unflatten", "vsa_pool_qk",
-           "vsa_flatten_pool_qk",
+           "vsa_flatten_pool_qk", "vsa_pool_qk_raster",
            "vsa_block_mask_workspace_size", "vsa_block_mask", "vsa_block_mask_topk",
            "vsa_sta_mask",
            "vsa_sparse_attn_workspace_size", "vsa_sparse_attn_fwd",
            "vsa_sparse_attn_fwd_noalloc", "vsa_sparse_attn_fwd_rows",
+           "vsa_sparse_attn_fwd_raster",
            "vsa_cluster_attn_workspace_size", "vsa_cluster_attn_fwd",
            "vsa_last_error", "vsa_device_status", "vsa_version")
 
@@ -78,12 +79,14 @@ def load():
         "vsa_fractal_unflatten": [P, P, vsa_shape, P],
         "vsa_pool_qk": [P, P, P, P, vsa_shape, P],
         "vsa_flatten_pool_qk": [P, P, P, P, P, P, vsa_shape, P],
+        "vsa_pool_qk_raster": [P, P, P, P, vsa_shape, P],
         "vsa_block_mask": [P, P, vsa_shape, vsa_mask_params, P, P, I64, P, P, S, P],
         "vsa_block_mask_topk": [P, P, vsa_shape, ctypes.c_int32, vsa_mask_params, P, P, I64, P,
                                 P, S, P],
         "vsa_sta_mask": [vsa_shape, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P, I64,
                          P, P],
         "vsa_sparse_attn_fwd": [P, P, P, P, P, vsa_shape, F, P, P, P, S, P],
+        "vsa_sparse_attn_fwd_raster": [P, P, P, P, P, vsa_shape, F, P, P, P, S, P],
         "vsa_sparse_attn_fwd_noalloc": [P, P, P, P, P, vsa_shape, F, P, P, P],
         "vsa_sparse_attn_fwd_rows": [P, P, P, P, P, vsa_shape, F, P, I64, P, P, P, S, P],
         "vsa_device_status": [P],

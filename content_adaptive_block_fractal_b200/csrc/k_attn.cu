@@ -108,6 +108,9 @@ struct AttnArgs {
                           // of the block is masked out; null: all 64
   int64_t N;              // tokens per head
   int Nb, T, HW;          // blocks per head, frames, patches per frame
+  int H, W, Wb;           // raster rows and columns per frame, patches per row
+  uint64_t hw_mul, wb_mul;  // ceil(2^32 / HW), ceil(2^32 / Wb): exact quotients
+                            // n / HW and n / Wb as (n * mul) >> 32 while n * HW < 2^32
   int pairs_per_head;
   float c;                // scale * log2(e)
   float lse_scale;        // ln(2)
@@ -132,6 +135,44 @@ __device__ __forceinline__ void decode_item(int item, const AttnArgs &a, int &bh
   const int t2 = p / a.HW, sp = p % a.HW;
   r0 = 2 * t2 * a.HW + sp;
   r1 = (2 * t2 + 1 < a.T) ? r0 + a.HW : -1;
+}
+
+// Frame and patch of 64-token block r (fractal order: frame-major, then the
+// patches of the frame row-major).
+__device__ __forceinline__ void block_patch(int r, const AttnArgs &a, int &t, int &py, int &px) {
+  t = static_cast<int>((static_cast<uint64_t>(r) * a.hw_mul) >> 32);
+  const int sp = r - t * a.HW;
+  py = static_cast<int>((static_cast<uint64_t>(sp) * a.wb_mul) >> 32);
+  px = sp - py * a.Wb;
+}
+
+// TMA load of 64-token block r of head slice bh into one operand stage.
+// Flattened layout: the block's 8 row groups are consecutive.  Raster layout:
+// the block is the 8 x 8 patch of its frame, so the box is placed by
+// (column, row, frame) coordinates and lands in the same SMEM order.
+template <bool kRaster>
+__device__ __forceinline__ void load_block(uint32_t dst, const CUtensorMap *m, uint32_t bar,
+                                           const AttnArgs &a, int bh, int r) {
+  if constexpr (kRaster) {
+    int t, py, px;
+    block_patch(r, a, t, py, px);
+    tma_load_5d(dst, m, bar, 0, px * 8, 0, py * 8, bh * a.T + t);
+  } else {
+    tma_load_4d(dst, m, bar, 0, 0, 0, static_cast<int>(static_cast<int64_t>(bh) * a.N / 8) + r * 8);
+  }
+}
+
+// Token index within its head of position i (= 8 * patch row + column) of
+// block r.
+template <bool kRaster>
+__device__ __forceinline__ int64_t block_token(const AttnArgs &a, int r, int i) {
+  if constexpr (!kRaster) {
+    return static_cast<int64_t>(r) * 64 + i;
+  } else {
+    int t, py, px;
+    block_patch(r, a, t, py, px);
+    return (static_cast<int64_t>(t) * a.H + py * 8 + (i >> 3)) * a.W + px * 8 + (i & 7);
+  }
 }
 
 // One 32-column chunk Q of the softmax's second pass: starts the load of
@@ -178,8 +219,9 @@ __device__ __forceinline__ void softmax_chunk(uint32_t (&cur)[32], uint32_t (&nx
 }
 
 // kKeyMask: key blocks may be partial (per-block valid counts in AttnArgs);
-// the plain instantiation carries no masking code.
-template <int D, bool kKeyMask>
+// the plain instantiation carries no masking code.  kRaster: Q, K, V, O and
+// LSE in raster token order (blocks fetched as patches), else flattened.
+template <int D, bool kKeyMask, bool kRaster>
 __global__ void __maxnreg__(168)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tq,
                        const __grid_constant__ CUtensorMap tk,
@@ -276,9 +318,8 @@ __global__ void __maxnreg__(168)
         const uint32_t kf = k_full(s3);
         mbar_arrive_expect_tx(kf, static_cast<uint32_t>(nb * L::kBlockBytes));
         const uint32_t kbase = sbase + L::kKOff + s3 * L::kKVBytes;
-        const int head_grp = static_cast<int>(static_cast<int64_t>(r.bh) * a.N / 8);
-        if (nb > 0) tma_load_4d(kbase, &tk, kf, 0, 0, 0, head_grp + r.blk0 * 8);
-        if (nb > 1) tma_load_4d(kbase + L::kBlockBytes, &tk, kf, 0, 0, 0, head_grp + r.blk1 * 8);
+        if (nb > 0) load_block<kRaster>(kbase, &tk, kf, a, r.bh, r.blk0);
+        if (nb > 1) load_block<kRaster>(kbase + L::kBlockBytes, &tk, kf, a, r.bh, r.blk1);
       }
       __syncwarp();
       ++m;
@@ -308,10 +349,8 @@ __global__ void __maxnreg__(168)
       if (lane == 0) {
         const int nq = r1 >= 0 ? 2 : 1;
         mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(nq * 64 * D * 2));
-        const int head_grp = static_cast<int>(static_cast<int64_t>(bh) * a.N / 8);
         for (int j = 0; j < nq; ++j)
-          tma_load_4d(sbase + L::kQOff + j * L::kBlockBytes, &tq, q_full, 0, 0, 0,
-                      head_grp + (j ? r1 : r0) * 8);
+          load_block<kRaster>(sbase + L::kQOff + j * L::kBlockBytes, &tq, q_full, a, bh, j ? r1 : r0);
       }
       // merge the two ascending lists, two union entries per step
       const int64_t g0 = static_cast<int64_t>(bh) * a.Nb + r0;
@@ -493,9 +532,8 @@ __global__ void __maxnreg__(168)
         const uint32_t vf = v_full(b);
         mbar_arrive_expect_tx(vf, static_cast<uint32_t>(nb * L::kBlockBytes));
         const uint32_t vbase = sbase + L::kVOff + b * L::kKVBytes;
-        const int head_grp = static_cast<int>(static_cast<int64_t>(r.bh) * a.N / 8);
-        if (nb > 0) tma_load_4d(vbase, &tv, vf, 0, 0, 0, head_grp + r.blk0 * 8);
-        if (nb > 1) tma_load_4d(vbase + L::kBlockBytes, &tv, vf, 0, 0, 0, head_grp + r.blk1 * 8);
+        if (nb > 0) load_block<kRaster>(vbase, &tv, vf, a, r.bh, r.blk0);
+        if (nb > 1) load_block<kRaster>(vbase + L::kBlockBytes, &tv, vf, a, r.bh, r.blk1);
       }
       __syncwarp();
     }
@@ -641,8 +679,8 @@ __global__ void __maxnreg__(168)
         const bool store = rblk >= 0;
         const bool has_keys = l_run > 0.0f;
         const float inv = has_keys ? 1.0f / l_run : 0.0f;
-        const int64_t tok = static_cast<int64_t>(m.bh) * a.N + static_cast<int64_t>(rblk) * 64 +
-                            (row & 63);
+        const int64_t tok =
+            static_cast<int64_t>(m.bh) * a.N + (store ? block_token<kRaster>(a, rblk, row & 63) : 0);
         uint4 *orow = reinterpret_cast<uint4 *>(a.o + tok * D);
 #pragma unroll 1
         for (int cc = 0; cc < D; cc += 32) {
@@ -788,17 +826,24 @@ cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
                                const Geometry &g, float scale, void *o, float *lse, void *ws,
                                unsigned *err, cudaStream_t st, const char **why,
                                const int32_t *qblocks, int64_t n_qblocks,
-                               const int32_t *kvalid) {
+                               const int32_t *kvalid, bool raster) {
   const AttnLayout L = attn_layout(g);
   if (L.items == 0 || (qblocks && n_qblocks == 0)) return cudaSuccess;
   if (L.items > 0x7FFFFFFF || g.BH * g.N > 0x7FFFFFFF) {
     *why = "sparse attention: too many tokens for 32-bit TMA row coordinates";
     return cudaErrorInvalidValue;
   }
+  if (raster && g.Nb * L.HW >= (1LL << 32)) {
+    *why = "sparse attention: too many blocks per head for the raster layout";
+    return cudaErrorInvalidValue;
+  }
   CUtensorMap mq, mk, mv;
   const int64_t rows = g.BH * g.N;
-  if (!make_map4(&mq, qf, rows, g.d) || !make_map4(&mk, kf, rows, g.d) ||
-      !make_map4(&mv, vf, rows, g.d)) {
+  const auto map = [&](CUtensorMap *m, const void *base) {
+    return raster ? make_map_raster(m, base, g.BH * g.T, g.H, g.W, g.d)
+                  : make_map4(m, base, rows, g.d);
+  };
+  if (!map(&mq, qf) || !map(&mk, kf) || !map(&mv, vf)) {
     *why = "sparse attention: cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
   }
@@ -827,6 +872,9 @@ cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
   a.o = static_cast<__nv_bfloat16 *>(o); a.lse = lse;
   a.order = order; a.counter = counter; a.err = err;
   a.items = L.items; a.N = g.N; a.Nb = static_cast<int>(g.Nb); a.T = g.T; a.HW = L.HW;
+  a.H = g.H; a.W = g.W; a.Wb = g.Wb;
+  a.hw_mul = ((1ull << 32) + L.HW - 1) / L.HW;
+  a.wb_mul = ((1ull << 32) + g.Wb - 1) / g.Wb;
   a.n_items = qblocks ? n_items : nullptr;
   a.qblocks = qblocks;
   a.n_qblocks = n_qblocks;
@@ -838,21 +886,38 @@ cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
   const int64_t max_items = qblocks ? (n_qblocks < L.items ? n_qblocks : L.items) : L.items;
   if (max_items < grid) grid = static_cast<int>(max_items);
   const bool masked = kvalid != nullptr;
-  const void *fn =
-      g.d == 128 ? (masked ? reinterpret_cast<const void *>(sparse_attn_kernel<128, true>)
-                           : reinterpret_cast<const void *>(sparse_attn_kernel<128, false>))
-                 : (masked ? reinterpret_cast<const void *>(sparse_attn_kernel<64, true>)
-                           : reinterpret_cast<const void *>(sparse_attn_kernel<64, false>));
-  const int smem = g.d == 128 ? Smem<128>::kAlloc : Smem<64>::kAlloc;
+  if (raster && masked) {
+    *why = "sparse attention: key masking is not available in the raster layout";
+    return cudaErrorInvalidValue;
+  }
+  // (masked, raster): the plain kernel, key masking (flattened), raster layout
+  const void *fn;
+  int smem;
+  if (g.d == 128) {
+    using L128 = Smem<128>;
+    fn = masked   ? reinterpret_cast<const void *>(sparse_attn_kernel<128, true, false>)
+         : raster ? reinterpret_cast<const void *>(sparse_attn_kernel<128, false, true>)
+                  : reinterpret_cast<const void *>(sparse_attn_kernel<128, false, false>);
+    smem = L128::kAlloc;
+  } else {
+    using L64 = Smem<64>;
+    fn = masked   ? reinterpret_cast<const void *>(sparse_attn_kernel<64, true, false>)
+         : raster ? reinterpret_cast<const void *>(sparse_attn_kernel<64, false, true>)
+                  : reinterpret_cast<const void *>(sparse_attn_kernel<64, false, false>);
+    smem = L64::kAlloc;
+  }
   if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
       cudaSuccess)
     return e;
-  if (g.d == 128)
-    masked ? sparse_attn_kernel<128, true><<<grid, kThreads, smem, st>>>(mq, mk, mv, a)
-           : sparse_attn_kernel<128, false><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
-  else
-    masked ? sparse_attn_kernel<64, true><<<grid, kThreads, smem, st>>>(mq, mk, mv, a)
-           : sparse_attn_kernel<64, false><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+  if (g.d == 128) {
+    if (masked) sparse_attn_kernel<128, true, false><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+    else if (raster) sparse_attn_kernel<128, false, true><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+    else sparse_attn_kernel<128, false, false><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+  } else {
+    if (masked) sparse_attn_kernel<64, true, false><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+    else if (raster) sparse_attn_kernel<64, false, true><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+    else sparse_attn_kernel<64, false, false><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     // report what the kernel needs next to what the launch asked for

@@ -75,7 +75,9 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint4 *__restrict__ q,
 // l always holds 16-byte column group l % (D/8) of its tokens, which keeps
 // its 8 fp64 accumulators on fixed columns (the same split as pool_kernel,
 // hence the same exact sums).  Units [0, blocks) are Q, [blocks, 2*blocks) K.
-template <int D>
+// kFlat false: the flattened copies are not written (the attention then reads
+// the raster tensors through patch-addressed TMA boxes), only the means.
+template <int D, bool kFlat>
 __global__ void __launch_bounds__(256)
     flatten_pool_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ k,
                         uint4 *__restrict__ qf, uint4 *__restrict__ kf, double *__restrict__ qp,
@@ -97,7 +99,7 @@ __global__ void __launch_bounds__(256)
     const int py = static_cast<int>(rem / Wb), px = static_cast<int>(rem % Wb);
     const int64_t head = bh * Nb * 64;           // first token of the head
     const uint4 *src = (is_k ? k : q) + (head + (t * H + py * 8) * W + px * 8) * kVecPerRow;
-    uint4 *dst = (is_k ? kf : qf) + (head + blk * 64) * kVecPerRow;
+    uint4 *dst = kFlat ? (is_k ? kf : qf) + (head + blk * 64) * kVecPerRow : nullptr;
     double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll 2
     for (int i = 0; i < 8; ++i) {                // patch row i: raster row py*8 + i
@@ -107,7 +109,7 @@ __global__ void __launch_bounds__(256)
       for (int j = 0; j < kPerLane; ++j) v[j] = __ldcs(run + lane + 32 * j);
 #pragma unroll
       for (int j = 0; j < kPerLane; ++j) {
-        __stcs(dst + i * kVecPerRun + lane + 32 * j, v[j]);
+        if (kFlat) __stcs(dst + i * kVecPerRun + lane + 32 * j, v[j]);
         const uint32_t u[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -141,12 +143,17 @@ cudaError_t launch_flatten_pool_qk(const void *q, const void *k, void *qf, void 
   const uint4 *k4 = static_cast<const uint4 *>(k);
   uint4 *qf4 = static_cast<uint4 *>(qf);
   uint4 *kf4 = static_cast<uint4 *>(kf);
+  const bool flat = qf != nullptr;
   if (g.d == 128)
-    flatten_pool_kernel<128><<<grid, 256, 0, st>>>(q4, k4, qf4, kf4, qp, kp, blocks, g.Nb, g.H,
-                                                   g.W);
+    flat ? flatten_pool_kernel<128, true><<<grid, 256, 0, st>>>(q4, k4, qf4, kf4, qp, kp, blocks,
+                                                                g.Nb, g.H, g.W)
+         : flatten_pool_kernel<128, false><<<grid, 256, 0, st>>>(q4, k4, qf4, kf4, qp, kp, blocks,
+                                                                 g.Nb, g.H, g.W);
   else
-    flatten_pool_kernel<64><<<grid, 256, 0, st>>>(q4, k4, qf4, kf4, qp, kp, blocks, g.Nb, g.H,
-                                                  g.W);
+    flat ? flatten_pool_kernel<64, true><<<grid, 256, 0, st>>>(q4, k4, qf4, kf4, qp, kp, blocks,
+                                                               g.Nb, g.H, g.W)
+         : flatten_pool_kernel<64, false><<<grid, 256, 0, st>>>(q4, k4, qf4, kf4, qp, kp, blocks,
+                                                                g.Nb, g.H, g.W);
   return cudaGetLastError();
 }
 

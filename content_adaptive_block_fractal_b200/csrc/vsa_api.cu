@@ -223,6 +223,26 @@ vsa_status vsa_flatten_pool_qk(const void *q, const void *k, void *qf, void *kf,
   return e == cudaSuccess ? VSA_OK : cuda_fail(e, "flatten+pool launch");
 }
 
+vsa_status vsa_pool_qk_raster(const void *q, const void *k, double *qp, double *kp, vsa_shape s,
+                              void *stream) {
+  vsa_status st = check_shape(s);
+  if (st != VSA_OK) return st;
+  if (empty(s)) return VSA_OK;
+  if (!q || !k || !qp || !kp) return fail(VSA_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(qp) || !aligned16(kp))
+    return fail(VSA_ERR_UNSUPPORTED, "tensor pointers must be 16-byte aligned");
+  const vsa::Geometry g = vsa::geometry(s);
+  const size_t bytes = static_cast<size_t>(g.BH * g.N) * g.d * 2;
+  const size_t pbytes = static_cast<size_t>(g.BH * g.Nb) * g.d * 8;
+  if (overlap(qp, pbytes, q, bytes) || overlap(qp, pbytes, k, bytes) ||
+      overlap(kp, pbytes, q, bytes) || overlap(kp, pbytes, k, bytes))
+    return fail(VSA_ERR_INVALID_ARG, "an output overlaps an input");
+  if (overlap(qp, pbytes, kp, pbytes)) return fail(VSA_ERR_INVALID_ARG, "outputs overlap");
+  cudaError_t e = vsa::launch_flatten_pool_qk(q, k, nullptr, nullptr, qp, kp, g,
+                                              static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? VSA_OK : cuda_fail(e, "raster pool launch");
+}
+
 size_t vsa_block_mask_workspace_size(vsa_shape s) {
   if (check_shape(s) != VSA_OK) return 0;
   return vsa::block_mask_workspace_bytes(vsa::geometry(s));
@@ -341,7 +361,8 @@ size_t vsa_sparse_attn_workspace_size(vsa_shape s) {
 static vsa_status sparse_attn(const void *qf, const void *kf, const void *vf,
                               const int64_t *row_ptr, const int32_t *col_idx, vsa_shape s,
                               float scale, const int32_t *qblocks, int64_t n_qblocks, void *o,
-                              float *lse, void *workspace, size_t workspace_bytes, void *stream);
+                              float *lse, void *workspace, size_t workspace_bytes, void *stream,
+                              bool raster = false);
 
 vsa_status vsa_sparse_attn_fwd(const void *qf, const void *kf, const void *vf,
                                const int64_t *row_ptr, const int32_t *col_idx, vsa_shape s,
@@ -349,6 +370,14 @@ vsa_status vsa_sparse_attn_fwd(const void *qf, const void *kf, const void *vf,
                                size_t workspace_bytes, void *stream) {
   return sparse_attn(qf, kf, vf, row_ptr, col_idx, s, scale, nullptr, 0, o, lse, workspace,
                      workspace_bytes, stream);
+}
+
+vsa_status vsa_sparse_attn_fwd_raster(const void *q, const void *k, const void *v,
+                                      const int64_t *row_ptr, const int32_t *col_idx,
+                                      vsa_shape s, float scale, void *o, float *lse,
+                                      void *workspace, size_t workspace_bytes, void *stream) {
+  return sparse_attn(q, k, v, row_ptr, col_idx, s, scale, nullptr, 0, o, lse, workspace,
+                     workspace_bytes, stream, true);
 }
 
 vsa_status vsa_sparse_attn_fwd_rows(const void *qf, const void *kf, const void *vf,
@@ -375,7 +404,8 @@ vsa_status vsa_sparse_attn_fwd_rows(const void *qf, const void *kf, const void *
 static vsa_status sparse_attn(const void *qf, const void *kf, const void *vf,
                               const int64_t *row_ptr, const int32_t *col_idx, vsa_shape s,
                               float scale, const int32_t *qblocks, int64_t n_qblocks, void *o,
-                              float *lse, void *workspace, size_t workspace_bytes, void *stream) {
+                              float *lse, void *workspace, size_t workspace_bytes, void *stream,
+                              bool raster) {
   vsa_status st = check_shape(s);
   if (st != VSA_OK) return st;
   if (empty(s)) return VSA_OK;
@@ -396,7 +426,8 @@ static vsa_status sparse_attn(const void *qf, const void *kf, const void *vf,
   if (!err) return cuda_fail(e, "device error word");
   const char *why = nullptr;
   e = vsa::launch_sparse_attn(qf, kf, vf, row_ptr, col_idx, g, scale, o, lse, workspace, err,
-                              static_cast<cudaStream_t>(stream), &why, qblocks, n_qblocks);
+                              static_cast<cudaStream_t>(stream), &why, qblocks, n_qblocks,
+                              nullptr, raster);
   if (e != cudaSuccess)
     return why ? fail(e == cudaErrorInvalidValue ? VSA_ERR_UNSUPPORTED : VSA_ERR_CUDA, "%s", why)
                : cuda_fail(e, "sparse attention launch");

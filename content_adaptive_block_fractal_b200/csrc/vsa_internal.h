@@ -34,6 +34,7 @@ cudaError_t launch_fractal_permute(const void *src, void *dst, const Geometry &g
                                    cudaStream_t st);
 cudaError_t launch_pool_qk(const void *qf, const void *kf, double *qp, double *kp,
                            const Geometry &g, cudaStream_t st);
+// qf, kf null: only the block means are written (pooling straight from raster).
 cudaError_t launch_flatten_pool_qk(const void *q, const void *k, void *qf, void *kf, double *qp,
                                    double *kp, const Geometry &g, cudaStream_t st);
 
@@ -57,7 +58,7 @@ cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
                                const Geometry &g, float scale, void *o, float *lse, void *ws,
                                unsigned *err, cudaStream_t st, const char **why,
                                const int32_t *qblocks = nullptr, int64_t n_qblocks = 0,
-                               const int32_t *kvalid = nullptr);
+                               const int32_t *kvalid = nullptr, bool raster = false);
 
 // Semantic-aware permutation attention: workspace and launch.
 size_t cluster_workspace_bytes(const Geometry &g, const vsa_cluster_params &c);

@@ -16,6 +16,9 @@
  *   5. vsa_sparse_attn_fwd       attention forward over the kept 64 x 64 tiles,
  *                                returning O and the log-sum-exp;
  *   and vsa_fractal_unflatten    to bring O back to raster order.
+ * Steps 1 and 5's unflattening can also be left to the attention's own
+ * loads and stores: vsa_pool_qk_raster and vsa_sparse_attn_fwd_raster take
+ * raster tensors and give the same results with no permuted copy written.
  *
  * Conventions shared by every entry point
  *   - Pointers marked "device" are CUDA device pointers on the current device;
@@ -104,6 +107,17 @@ vsa_status vsa_pool_qk(const void *qf, const void *kf, double *qp, double *kp,
 vsa_status vsa_flatten_pool_qk(const void *q, const void *k, void *qf, void *kf, double *qp,
                                double *kp, vsa_shape s, void *stream);
 
+/* 1.+2. without the copies: the block means of the fractal blocks read
+ * straight from raster Q and K (NABLA, Methodology items 1-2: block r of a
+ * head is the P x P patch (r % (H/P*W/P)) of frame r / (H/P*W/P), patches
+ * row-major).  Bit-identical to the qp, kp of vsa_flatten_pool_qk; for use
+ * with vsa_sparse_attn_fwd_raster, which needs no flattened tensors.
+ * q, k   : device bf16 [B,heads,N,d], raster order (may alias each other).
+ * qp, kp : device fp64 [B,heads,Nb,d] (outputs); neither may overlap an input
+ *          or the other (VSA_ERR_INVALID_ARG). */
+vsa_status vsa_pool_qk_raster(const void *q, const void *k, double *qp, double *kp,
+                              vsa_shape s, void *stream);
+
 /* 3.-4. Block mask (NABLA, Methodology items 2-3).
  * For every (b, h) and query block r: A[r,:] = softmax(qp_r . kp_c / sqrt(d))
  * over the Nb key blocks c, CDF selection at thr, union with the STA window
@@ -175,6 +189,22 @@ vsa_status vsa_sparse_attn_fwd(const void *qf, const void *kf, const void *vf,
                                vsa_shape s, float scale, void *o, float *lse,
                                void *workspace, size_t workspace_bytes,
                                void *stream);
+
+/* 5. with raster tensors: the same computation as vsa_sparse_attn_fwd, with
+ * q, k, v, o : device bf16 [B,heads,N,d] and lse : fp32 [B,heads,N] in
+ * raster token order n = (t*H + y)*W + x instead of flattened order.  The
+ * mask (row_ptr, col_idx) is unchanged: it indexes fractal blocks, block r of
+ * a head being the P x P patch (r % (H/P*W/P)) of frame r / (H/P*W/P).  Each
+ * block is fetched by one patch-shaped TMA box and each output row is stored
+ * at its raster position, so
+ *   vsa_sparse_attn_fwd_raster(q, k, v -> o, lse)
+ * equals, bit for bit, vsa_fractal_flatten of q, k and v, vsa_sparse_attn_fwd,
+ * then vsa_fractal_unflatten of o and the same permutation of lse.  Workspace
+ * and errors as vsa_sparse_attn_fwd. */
+vsa_status vsa_sparse_attn_fwd_raster(const void *q, const void *k, const void *v,
+                                      const int64_t *row_ptr, const int32_t *col_idx,
+                                      vsa_shape s, float scale, void *o, float *lse,
+                                      void *workspace, size_t workspace_bytes, void *stream);
 
 /* Query-subset attention (HSA, arXiv 2605.06892 summary, section 2.2 "KV cache
  * synchronisation": only the active tokens form queries, against the whole

@@ -128,3 +128,26 @@ def test_query_subset_validation():
     assert call(P((1 << 12) + 2), 4) == 1       # misaligned list
     assert call(P(1 << 12), 33) == 1            # more entries than query blocks
     assert call(None, 0) == 0                   # nothing to do
+
+
+def test_raster_pool_and_attention_validation():
+    L = _lib.load()
+    s = Shape(1, 2, 4, 16, 16, 64)              # 256 KiB per bf16 tensor, 16 KiB pooled
+    P = ctypes.c_void_p
+    MB = 1 << 20
+    def pool(q=1 * MB, k=2 * MB, qp=3 * MB, kp=4 * MB):
+        return L.vsa_pool_qk_raster(P(q), P(k), P(qp), P(kp), s.c(), None)
+    assert pool(q=0) == 1
+    assert pool(kp=0) == 1
+    assert pool(qp=3 * MB + 8) == 2                 # misaligned
+    assert pool(qp=1 * MB + 4096) == 1              # output inside an input
+    assert pool(kp=3 * MB + 4096) == 1              # the two outputs overlap
+    def attn(ws_bytes=1 << 20, q=1 << 12, lse=1 << 29):
+        return L.vsa_sparse_attn_fwd_raster(P(q), P(1 << 16), P(1 << 20), P(1 << 24), P(1 << 26),
+                                            s.c(), 0.0, P(1 << 28), P(lse), P(1 << 30), ws_bytes,
+                                            None)
+    assert attn(q=0) == 1
+    assert attn(q=(1 << 12) + 8) == 2
+    assert attn(lse=(1 << 29) + 2) == 2
+    assert attn(ws_bytes=8) == 3                    # workspace too small
+    assert len(L.vsa_last_error()) > 0

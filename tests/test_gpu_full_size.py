@@ -1,5 +1,5 @@
 """Parity at the full workload sizes, through the same calls and launch
-configuration that bench.py times (fused flatten+pool of Q and K, flatten of V,
+configuration that `bench.py --layout flat` times (fused flatten+pool of Q and K, flatten of V,
 block mask, sparse attention, unflatten of O, all heads in one launch each).
 
 The oracle cannot run a whole 40-head or 24-head layer in a test, so it checks
