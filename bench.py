@@ -359,7 +359,8 @@ def run_gpu(args, rank, world, local_rank):
         "kept_fraction": kept_frac,
         "kept_tiles": kept,
         "breakdown_ms": parts,
-        "roofline": {"bound": "tensor", "kernel": "sparse_attn_kernel<128, 0>",
+        "roofline": {"bound": "tensor",
+                     "kernel": f"sparse_attn_kernel<{shape.d}, 0, {int(raster)}>",
                      "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": achieved_tf / peak_tf, "traffic": traffic,
                      "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long loop)",

@@ -151,3 +151,8 @@ def test_raster_pool_and_attention_validation():
     assert attn(lse=(1 << 29) + 2) == 2
     assert attn(ws_bytes=8) == 3                    # workspace too small
     assert len(L.vsa_last_error()) > 0
+
+
+def test_layer_layout_is_checked_before_allocating():
+    with pytest.raises(ValueError, match="layout"):
+        vsa.Layer(Shape(1, 2, 4, 16, 16, 64), MaskParams(0.2), "cpu", layout="fractal")
