@@ -25,7 +25,9 @@
 //               d/64 halves x 8 row groups), stored 128B-swizzled as
 //               [row group][d-half][8 rows][128 B]: the rows of two blocks
 //               then sit at one uniform group stride of 16*d bytes (the SBO)
-//               and the d-halves 1 KiB apart;
+//               and the d-halves 1 KiB apart.  In the raster layout the
+//               block is the 8 x 8 patch of its frame, fetched by one 5-D box
+//               that lands in the same SMEM order;
 //   warp 11     V producer: follows the step records and loads V per step
 //               into its own 3-deep ring;
 //   warp 1      allocates 512 TMEM columns; one lane issues the S MMAs;

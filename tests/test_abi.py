@@ -156,3 +156,11 @@ def test_raster_pool_and_attention_validation():
 def test_layer_layout_is_checked_before_allocating():
     with pytest.raises(ValueError, match="layout"):
         vsa.Layer(Shape(1, 2, 4, 16, 16, 64), MaskParams(0.2), "cpu", layout="fractal")
+
+
+def test_raster_entry_points_accept_an_empty_shape():
+    L = _lib.load()
+    s = Shape(1, 2, 0, 16, 16, 64).c()            # T = 0: nothing to do, nothing touched
+    assert L.vsa_pool_qk_raster(None, None, None, None, s, None) == 0
+    assert L.vsa_sparse_attn_fwd_raster(None, None, None, None, None, s, 0.0, None, None, None,
+                                        0, None) == 0
