@@ -839,6 +839,11 @@ cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
     *why = "sparse attention: too many blocks per head for the raster layout";
     return cudaErrorInvalidValue;
   }
+  const bool masked = kvalid != nullptr;
+  if (raster && masked) {
+    *why = "sparse attention: key masking is not available in the raster layout";
+    return cudaErrorInvalidValue;
+  }
   CUtensorMap mq, mk, mv;
   const int64_t rows = g.BH * g.N;
   const auto map = [&](CUtensorMap *m, const void *base) {
@@ -887,26 +892,20 @@ cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
   int grid = num_sms();
   const int64_t max_items = qblocks ? (n_qblocks < L.items ? n_qblocks : L.items) : L.items;
   if (max_items < grid) grid = static_cast<int>(max_items);
-  const bool masked = kvalid != nullptr;
-  if (raster && masked) {
-    *why = "sparse attention: key masking is not available in the raster layout";
-    return cudaErrorInvalidValue;
-  }
-  // (masked, raster): the plain kernel, key masking (flattened), raster layout
+  // three instantiations per d: flattened, flattened with key masking (the
+  // cluster path), raster
   const void *fn;
   int smem;
   if (g.d == 128) {
-    using L128 = Smem<128>;
     fn = masked   ? reinterpret_cast<const void *>(sparse_attn_kernel<128, true, false>)
          : raster ? reinterpret_cast<const void *>(sparse_attn_kernel<128, false, true>)
                   : reinterpret_cast<const void *>(sparse_attn_kernel<128, false, false>);
-    smem = L128::kAlloc;
+    smem = Smem<128>::kAlloc;
   } else {
-    using L64 = Smem<64>;
     fn = masked   ? reinterpret_cast<const void *>(sparse_attn_kernel<64, true, false>)
          : raster ? reinterpret_cast<const void *>(sparse_attn_kernel<64, false, true>)
                   : reinterpret_cast<const void *>(sparse_attn_kernel<64, false, false>);
-    smem = L64::kAlloc;
+    smem = Smem<64>::kAlloc;
   }
   if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
       cudaSuccess)
