@@ -94,7 +94,7 @@ int num_sms() {
 
 extern "C" {
 
-const char *vsa_version(void) { return "0.1.0"; }
+const char *vsa_version(void) { return "0.2.0"; }
 
 const char *vsa_last_error(void) { return g_last_error.c_str(); }
 
