@@ -368,7 +368,7 @@ def run_gpu(args, rank, world, local_rank):
                      "flop_per_kept_tile": flop_per_tile},
         # HBM kernels: algorithmic bytes / time (read + write, each byte once)
         "hbm_gbs": hbm,
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": launches_per_step * args.steps * world,   # all ranks
         "clocks": clk.summary(),
     }
     if e2e:
