@@ -84,9 +84,9 @@ struct Smem {
   static constexpr int kXchgOff = kListOff + 2 * kListWin * 4;   // m_sh[2][128], l_sh[2][128]
   static constexpr int kBarOff = (kXchgOff + 4 * 128 * 4 + 7) & ~7;
   // k_full[3] v_full[3] s_full[3] pv_buf[3] meta_full[8] meta_empty[8]
-  // q_full q_empty p_full[4] o_full o_empty m_full[2] l_full[2]
+  // q_full q_empty p_full[4] o_full[0] o_empty m_full[2] l_full[2] o_full[1]
   // (s_full also frees K stages and pv_buf V stages: same completions)
-  static constexpr int kNumBars = 4 * kRing + 2 * kMetaRing + 2 + 4 + 2 + 4;
+  static constexpr int kNumBars = 4 * kRing + 2 * kMetaRing + 2 + 4 + 3 + 4;
   static constexpr int kTmemSlotOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kTmemSlotOff + 16;
   static constexpr int kAlloc = kBytes;                   // base is 1 KiB aligned
@@ -254,7 +254,10 @@ __global__ void __maxnreg__(168)
   const uint32_t q_full = bar + 8u * (4 * kRing + 2 * kMetaRing);
   const uint32_t q_empty = q_full + 8;
   auto p_full = [&](int s) { return q_full + 16u + 8u * s; };   // 4 slots
-  const uint32_t o_full = q_full + 48;
+  // O complete, one barrier per item parity: item s completes phase s/2 of
+  // o_full(s & 1), so the phase before the one an epilogue waits for belongs
+  // to item s - 2, which is ordered before it (see the epilogue's wait)
+  auto o_full = [&](int s) { return s ? q_full + 96u : q_full + 48u; };
   const uint32_t o_empty = q_full + 56;
   auto m_full = [&](int s) { return q_full + 64u + 8u * s; };
   auto l_full = [&](int s) { return q_full + 80u + 8u * s; };
@@ -280,7 +283,8 @@ __global__ void __maxnreg__(168)
       mbar_init(m_full(s), 4);            // one arrival per softmax warp
       mbar_init(l_full(s), 4);
     }
-    mbar_init(o_full, 1);
+    mbar_init(o_full(0), 1);
+    mbar_init(o_full(1), 1);
     mbar_init(o_empty, 128);
     fence_mbar_init();
   }
@@ -512,8 +516,10 @@ __global__ void __maxnreg__(168)
               mma_bf16_ts(tmem + kColO, pcol + k * 8, vd + k * kKStep, kIdescO, true);
           }
         }
+        // O complete before the step's own commit: every later pv_buf
+        // arrival then follows this item's O-complete arrival
+        if (r.first_last & 2) mma_commit(o_full(r.seq & 1));
         mma_commit(pv_buf(b));          // also frees V stage b
-        if (r.first_last & 2) mma_commit(o_full);
       }
       __syncwarp();
     }
@@ -675,7 +681,15 @@ __global__ void __maxnreg__(168)
         // is in the scale of step n-1's reference m_prev <= m_run
         float l_run = l_own;
         if (l_other > 0.0f) l_run += l_other * ex2(m_prev - m_run);
-        if (!mbar_wait(o_full, static_cast<uint32_t>(m.seq) & 1u, a.err, kErrWaitMma)) break;
+        // Item seq is phase seq/2 of o_full(seq & 1).  The parity wait can
+        // only be early if that barrier's previous phase, item seq - 2, were
+        // still open.  It is not: if item seq - 2 ended at step n - 2, this
+        // group ran its epilogue and saw that phase complete; if it ended at
+        // step n - 3 or before, S_n waited for PV_(n-3)'s commit, which the PV
+        // issuer made after item seq - 2's O-complete commit.
+        if (!mbar_wait(o_full(m.seq & 1), (static_cast<uint32_t>(m.seq) >> 1) & 1u, a.err,
+                       kErrWaitMma))
+          break;
         tc_fence_after();
         const int rblk = sel ? m.r1 : m.r0;
         const bool store = rblk >= 0;
@@ -766,7 +780,6 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int64_t *__restrict__ 
         bh * pairs + static_cast<int32_t>(keys[p] & 0xFFFFFFFFu);
 }
 
-// Fallback order (no per-head sort) for very large heads.
 // Query-subset planner: the listed query blocks (global rows, strictly
 // ascending) are paired in list order within each head -- the block of even
 // rank within its head leads an item, the next one joins it -- so every item
@@ -794,6 +807,8 @@ __global__ void plan_rows_kernel(const int32_t *__restrict__ qblocks, int64_t n,
   order[pos] = static_cast<int32_t>(i);
 }
 
+// Fallback order (no per-head sort) for heads with more than 4096 query-tile
+// pairs, beyond the planner's single-CTA bitonic sort.
 __global__ void identity_order_kernel(int32_t *order, int64_t n, int *counter) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i == 0) *counter = 0;

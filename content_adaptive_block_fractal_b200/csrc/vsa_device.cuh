@@ -395,24 +395,6 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-// 2^x on the FMA and integer pipes, for x <= 9 (the softmax's range), so
-// that part of the exponentials can bypass the 16/clk/SM MUFU unit.  Range
-// reduction x = j + f with j = rint(x) (the 1.5*2^23 rounding trick: j lands
-// in the low mantissa bits of t), |f| <= 1/2; 2^f from a degree-3 polynomial
-// fitted to 2^f on [-1/2, 1/2] by the Remez exchange algorithm for minimal
-// relative error (7.5e-5 when evaluated in fp32, below half a bf16 ulp); 2^j
-// added to the exponent field with one integer shift-add.  x is clamped at
-// -125 so the exponent never wraps; results below 2^-125 come out as tiny
-// normals instead of exact underflow, which no sum of these values can see.
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -125.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  const float p = fmaf(fmaf(fmaf(5.517166853e-02f, f, 2.426111251e-01f), f, 6.932609677e-01f), f,
-                       9.999280572e-01f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&h);

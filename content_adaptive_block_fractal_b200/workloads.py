@@ -198,3 +198,22 @@ def random_csr(n_rows: int, nb: int, density: float, seed: int):
     np.cumsum(counts, out=row_ptr[1:])
     col_idx = np.nonzero(keep)[1].astype(np.int32)
     return row_ptr, col_idx
+
+
+def short_csr(n_rows: int, nb: int, k_min: int, k_max: int, seed: int):
+    """Seeded random block lists with k_min..k_max distinct blocks per row
+    (row_ptr int64, col_idx int32, ascending per row), drawn row by row so
+    that wide grids need no n_rows x nb matrix."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    counts = rng.integers(k_min, k_max + 1, size=n_rows)
+    row_ptr = np.zeros(n_rows + 1, dtype=np.int64)
+    np.cumsum(counts, out=row_ptr[1:])
+    col_idx = np.empty(int(row_ptr[-1]), dtype=np.int32)
+    # k_max draws per row, duplicates replaced until each row has distinct blocks
+    draw = rng.integers(0, nb, size=(n_rows, k_max))
+    for r in range(n_rows):
+        cols = np.unique(draw[r, :counts[r]])
+        while cols.size < counts[r]:
+            cols = np.unique(np.append(cols, rng.integers(0, nb)))
+        col_idx[row_ptr[r]:row_ptr[r + 1]] = cols
+    return row_ptr, col_idx

@@ -14,9 +14,11 @@ Checks: every role finishes (no deadlock); every parity wait succeeds on
 exactly the phase it names (neither early nor lapped); no K/V stage, step
 record slot or TMEM S buffer is reused before its previous user is done; every
 MMA finds its operands loaded.  With `check_epilogue` the epilogue's wait on
-the O-complete barrier is the kernel's parity wait and is checked like the
-others; without it, it is modelled as a wait for its own item's phase, so the
-rest of the protocol is checked on its own."""
+the O-complete barriers (one per item parity) is the kernel's parity wait and
+is checked like the others; without it, it is modelled as a wait for its own
+item's phase, so the rest of the protocol is checked on its own.  A variant
+with a single O-complete barrier (`single_o_full`) reproduces the ordering gap
+that the per-parity pair closes."""
 import random
 
 RING, META = 3, 8
@@ -53,8 +55,9 @@ class Barrier:
 
 
 class Model:
-    def __init__(self, items, rng, check_epilogue):
+    def __init__(self, items, rng, check_epilogue, single_o_full=False):
         self.items, self.rng, self.check_epilogue = items, rng, check_epilogue
+        self.single_o_full = single_o_full
         self.t = 0
         self.events = []
         mk = Barrier
@@ -66,7 +69,8 @@ class Model:
         self.meta_empty = [mk(f"meta_empty{i}", 1) for i in range(META)]  # 4 warps of a group
         self.q_full, self.q_empty = mk("q_full", 1), mk("q_empty", 1)
         self.p_full = [mk(f"p_full{i}", 1) for i in range(4)]
-        self.o_full, self.o_empty = mk("o_full", 1), mk("o_empty", 1)
+        self.o_full = [mk(f"o_full{i}", 1) for i in range(1 if single_o_full else 2)]
+        self.o_empty = mk("o_empty", 1)
         self.m_full = [mk(f"m_full{i}", 1) for i in range(2)]
         self.l_full = [mk(f"l_full{i}", 1) for i in range(2)]
         self.meta = [None] * META
@@ -88,6 +92,10 @@ class Model:
         assert r is not None and r["n"] == n, f"{who} read a stale record for step {n}"
         self.readers.setdefault(n, set()).add(who)
         return r
+
+    def o_slot(self, seq):
+        """The O-complete barrier of item `seq`."""
+        return 0 if self.single_o_full else seq & 1
 
     # ------------------------------------------------------------------ roles
     def producer(self):
@@ -164,11 +172,13 @@ class Model:
             yield from self.wait(self.v_full[b], (n // RING) & 1, n // RING)
             assert r["nb"] == 0 or ("V", n) in self.done, "PV MMA before its V landed"
 
-            def finish(b=b, n=n, last=r["last"]):
+            def finish(b=b, n=n, last=r["last"], seq=r["seq"]):
+                # the kernel commits O complete before the step's pv_buf, and
+                # commits arrive in issue order
                 self.done.add(("PV", n))
-                self.pv_buf[b].arrive()
                 if last:
-                    self.o_full.arrive()
+                    self.o_full[self.o_slot(seq)].arrive()
+                self.pv_buf[b].arrive()
             self.later(finish, 5, 60)
             n += 1
 
@@ -218,10 +228,12 @@ class Model:
                 assert ("PV", p) in self.done
             self.p_full[n & 3].arrive()
             if r["last"]:
+                ob = self.o_full[self.o_slot(r["seq"])]
+                ph = r["seq"] if self.single_o_full else r["seq"] >> 1
                 if self.check_epilogue:      # the kernel's parity wait, checked
-                    yield from self.wait(self.o_full, r["seq"] & 1, r["seq"])
+                    yield from self.wait(ob, ph & 1, ph)
                 else:                        # an ordered wait for this item's phase
-                    while self.o_full.phase < r["seq"] + 1:
+                    while ob.phase < ph + 1:
                         yield
                 assert ("PV", n) in self.done, "epilogue read O before its last PV finished"
                 self.o_empty.arrive()
@@ -231,7 +243,7 @@ class Model:
     def state(self, live):
         bars = (self.k_full + self.v_full + self.s_full + self.pv_buf + self.meta_full +
                 self.meta_empty + self.p_full + self.m_full + self.l_full +
-                [self.q_full, self.q_empty, self.o_full, self.o_empty])
+                self.o_full + [self.q_full, self.q_empty, self.o_empty])
         return (len(live),) + tuple((b.phase, b.arrived, b.tx) for b in bars)
 
     def run(self):
@@ -272,7 +284,8 @@ def random_items(rng):
     return items
 
 
-def run_schedules(count, seed, check_epilogue):
+def run_schedules(count, seed, check_epilogue, single_o_full=False):
     rng = random.Random(seed)
     for _ in range(count):
-        Model(random_items(rng), random.Random(rng.random()), check_epilogue).run()
+        Model(random_items(rng), random.Random(rng.random()), check_epilogue,
+              single_o_full).run()

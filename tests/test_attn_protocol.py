@@ -14,11 +14,15 @@ def test_protocol_has_no_deadlock_early_wait_or_early_reuse():
     run_schedules(300, seed=2026, check_epilogue=False)
 
 
-@pytest.mark.xfail(strict=True, raises=AssertionError,
-                   reason="known gap: the O-complete barrier advances once per item, so an "
-                          "epilogue whose item starts right after the previous item's last step "
-                          "(other softmax group) can pass its parity wait one phase early if "
-                          "that item's last PV is late; the kernel's Q reload gives it a timing "
-                          "margin, not an ordering.  Fix: one O-complete barrier per item parity.")
 def test_epilogue_wait_names_its_item():
-    run_schedules(300, seed=2026, check_epilogue=True)
+    """With one O-complete barrier per item parity, the epilogue's parity wait
+    succeeds on exactly its own item's phase, under every schedule."""
+    run_schedules(600, seed=2026, check_epilogue=True)
+
+
+def test_single_o_complete_barrier_is_caught():
+    """The model tells the two designs apart: with a single O-complete barrier
+    advancing once per item, some schedule lets an epilogue whose item starts
+    right after the previous item's last step pass its wait one phase early."""
+    with pytest.raises(AssertionError, match="o_full0"):
+        run_schedules(300, seed=2026, check_epilogue=True, single_o_full=True)

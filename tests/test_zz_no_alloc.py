@@ -13,8 +13,6 @@ import torch
 from content_adaptive_block_fractal_b200 import _lib, workloads
 import content_adaptive_block_fractal_b200 as vsa
 
-O_MAX, O_MEAN, LSE_TOL = 2e-2, 2e-3, 1e-3
-
 
 def _p(t):
     return ctypes.c_void_p(t.data_ptr())
@@ -46,14 +44,13 @@ def _no_alloc(L, shape, qf, kf, vf, rp, ci, stream):
     return o, lse
 
 
-def _close(a, b):
+def _same(a, b):
+    """Both entry points run the same kernel on the same inputs, and each
+    128-row tile is computed by one CTA in a fixed order, so O and LSE must
+    agree bit for bit (a stale plan or an aliased scratch would not)."""
     (oa, la), (ob, lb) = a, b
-    err = (oa.float() - ob.float()).abs()
-    assert err.max().item() <= O_MAX and err.mean().item() <= O_MEAN
-    fin = torch.isfinite(lb)
-    assert torch.equal(torch.isfinite(la), fin)
-    if fin.any():
-        assert (la[fin] - lb[fin]).abs().max().item() <= LSE_TOL
+    assert torch.equal(oa, ob)
+    assert torch.equal(la, lb)
 
 
 @pytest.mark.gpu
@@ -73,8 +70,8 @@ def test_no_alloc_matches_workspace_entry_point_twice():
         second = _no_alloc(L, shape, qf, kf, vf, rp, ci, stream)
         torch.cuda.synchronize()
         _lib.check(L.vsa_device_status(stream))
-        _close(first, ref)
-        _close(second, ref)
+        _same(first, ref)
+        _same(second, ref)
 
 
 @pytest.mark.gpu
