@@ -21,7 +21,6 @@ import hashlib
 import json
 import math
 import os
-import re
 import subprocess
 import sys
 import time
@@ -35,10 +34,10 @@ WORKLOAD = "wan14b-720p"
 METRIC = "ms/attention layer and kept-tile TFLOP/s at Wan-14B 720p shape, thr=0.1"
 UNIT = "ms/layer"
 L2_FLUSH_BYTES = 256 << 20
-# ncu DRAM summaries of the attention launch in each layout
-PROFILES = {lay: os.path.join(ROOT, "profiles", f"sparse_attn_fwd_{lay}_wan14b-720p.md")
-            for lay in ("raster", "flat")}
-# files whose contents make up the attention kernel (hashed against the summary)
+# DRAM bytes per launch of each benchmarked kernel, from ncu captures, with a
+# hash of the kernel's source files at capture time
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "dram_traffic.json")
+# files whose contents make up the attention kernel (hashed against the record)
 ATTN_SOURCES = [os.path.join(ROOT, "content_adaptive_block_fractal_b200", "csrc", f)
                 for f in ("k_attn.cu", "vsa_device.cuh")]
 
@@ -57,6 +56,9 @@ def parse_args():
                          "and write raster o; flat: explicit flatten / unflatten passes")
     ap.add_argument("--cluster", action="store_true",
                     help="only the semantic-aware permutation path at the Wan-14B 720p shape")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="N > 1: every rank runs its own layer (replicas, weak scaling), or the "
+                         "ranks split one layer's heads (heads, strong scaling)")
     ap.add_argument("--sweep", action="store_true",
                     help="thr x STA sweep at the Wan-14B 720p shape: one JSON line per point "
                          "(mask + attention; inputs generated once)")
@@ -81,19 +83,18 @@ def kernel_source_hash(paths) -> str:
     return h.hexdigest()
 
 
-def profile_traffic(kernel_srcs, profile):
-    """DRAM bytes per attention launch from the committed ncu summary, if it was
-    taken on the current kernel source (same hash of the kernel's files); else None."""
+def profile_traffic(kernel, kernel_srcs, record=TRAFFIC_RECORD):
+    """DRAM bytes per launch of `kernel` from the traffic record, if they were
+    captured on the current kernel source (same hash of the kernel's files);
+    else None."""
     try:
-        text = open(profile).read()
-    except OSError:
+        with open(record) as f:
+            entry = json.load(f)["kernels"][kernel]
+    except (OSError, KeyError, ValueError, TypeError):
         return None
-    h = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
-    b = re.search(r"dram_bytes_per_launch_full:\s*([0-9.eE+]+)", text)
-    if not h or not b:
+    if kernel_source_hash(kernel_srcs) != entry.get("source_sha256"):
         return None
-    cur = kernel_source_hash(kernel_srcs)
-    return float(b.group(1)) if cur.startswith(h.group(1)) else None
+    return float(entry["dram_bytes_per_launch"])
 
 
 class ClockSampler:
@@ -153,10 +154,29 @@ def reduce_over_ranks(values, device):
     return [float(x) for x in t]
 
 
-def job_ms_per_layer(ms_max: float, world: int) -> float:
-    """Weak scaling: each of `world` ranks runs one layer in at most ms_max,
-    so the job turns out a layer every ms_max / world."""
-    return ms_max / world
+def sum_over_ranks(values, device):
+    """Sum over ranks (work counts of a layer split across ranks)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return [float(x) for x in t]
+
+
+def head_slice(heads: int, rank: int, world: int):
+    """Heads [h0, h1) of one layer that `rank` computes when `world` ranks
+    split the layer by heads: contiguous, disjoint, sizes differing by at most
+    one.  Every step of the path is independent per head, so no data crosses
+    ranks."""
+    return heads * rank // world, heads * (rank + 1) // world
+
+
+def job_ms_per_layer(ms_max: float, world: int, shard: str = "replicas") -> float:
+    """Replicas (weak scaling): each of `world` ranks runs one layer in at most
+    ms_max, so the job turns out a layer every ms_max / world.  Heads (strong
+    scaling): the ranks share one layer, which is done when the slowest rank
+    is, after ms_max."""
+    return ms_max / world if shard == "replicas" else ms_max
 
 
 # --------------------------------------------------------------------------- GPU arm
@@ -168,10 +188,12 @@ def run_gpu(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     wl = workloads.get(args.workload)
-    shape = vsa.Shape.of(wl)
     params = vsa.MaskParams(wl.thr, wl.use_sta, wl.sta)
+    shard = args.shard if world > 1 else "replicas"
+    h0, h1 = head_slice(wl.heads, rank, world) if shard == "heads" else (0, wl.heads)
+    shape = vsa.Shape(wl.B, h1 - h0, wl.T, wl.H, wl.W, wl.d)
 
-    q, k, v = workloads.make_qkv(wl)                       # host bf16, raster order
+    q, k, v = workloads.make_qkv(wl, heads=range(h0, h1))   # host bf16, raster order
     qh, kh, vh = (x.pin_memory() for x in (q, k, v))
     qd, kd, vd = (x.cuda() for x in (qh, kh, vh))
     stream = torch.cuda.current_stream()
@@ -191,8 +213,8 @@ def run_gpu(args, rank, world, local_rank):
                 x[0], x[1], x[2], csr.row_ptr, csr.col_idx, shape, 0.0, out=(o, lse),
                 workspace=layer.ws_attn)),
         ]
-        # pool; mask (scores, select, chunk sums, chunk scan, expand); plan + attention
-        launches_per_step = 1 + 5 + 2
+        # pool; mask (digits, select, recheck, chunk sums, chunk scan, expand); plan + attention
+        launches_per_step = 1 + 6 + 2
     else:
         qf, kf, vf = (torch.empty_like(qd) for _ in range(3))
         o_raster = torch.empty_like(qd)
@@ -207,8 +229,8 @@ def run_gpu(args, rank, world, local_rank):
                 workspace=layer.ws_attn)),
             ("unflatten_o", lambda x: vsa.fractal_unflatten(o, shape, out=o_raster)),
         ]
-        # flatten+pool of Q,K; flatten of V; mask (5); plan + attention; unflatten of O
-        launches_per_step = 1 + 1 + 5 + 2 + 1
+        # flatten+pool of Q,K; flatten of V; mask (6); plan + attention; unflatten of O
+        launches_per_step = 1 + 1 + 6 + 2 + 1
     n_st = len(stages)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_st + 1)]
     inputs = (qd, kd, vd)
@@ -323,17 +345,28 @@ def run_gpu(args, rank, world, local_rank):
                "overlap": "H2D, compute and D2H on separate streams, two buffer sets"}
 
     if world > 1:
-        ms, e2e_max = reduce_over_ranks([ms, e2e["value"] if e2e else 0.0], qd.device)
+        names = list(parts)
+        maxed = reduce_over_ranks([ms, e2e["value"] if e2e else 0.0] + [parts[n] for n in names],
+                                  qd.device)
+        ms, e2e_max = maxed[0], maxed[1]
+        parts = dict(zip(names, maxed[2:]))
         if e2e:
-            e2e["value"] = job_ms_per_layer(e2e_max, world)
-    value = job_ms_per_layer(ms, world)
-    # The attention kernel runs back to back for the whole timed loop and
-    # holds the GPU at its power cap, so the sustained GEMM figure (a
-    # seconds-long cuBLAS loop under the same cap) is its denominator.
-    burst_tf, peak_tf, peak_gbs, peak_src = measured_peaks()
+            e2e["value"] = job_ms_per_layer(e2e_max, world, shard)
+        if shard == "heads":
+            # the layer's kept tiles are the sum of the ranks' slices
+            kept = int(sum_over_ranks([kept], qd.device)[0])
+            kept_flop = kept * flop_per_tile
+            rows = wl.B * wl.heads * shape.Nb
+            kept_frac = kept / (rows * shape.Nb)
+    value = job_ms_per_layer(ms, world, shard)
+    # The attention kernel is one launch of ~10 ms per step, timed alone by
+    # CUDA events between L2 flushes; its clocks stay near the maximum, so the
+    # burst GEMM figure is its denominator (the sustained one is printed too).
+    burst_tf, sus_tf, peak_gbs, peak_src = measured_peaks()
     attn_ms = parts["sparse_attn"]
     achieved_tf = kept_flop / (attn_ms * 1e-3) / 1e12
-    traffic = profile_traffic(ATTN_SOURCES, PROFILES[args.layout])
+    attn_kernel = f"sparse_attn_kernel<{shape.d}, 0, {int(raster)}>"
+    traffic = profile_traffic(attn_kernel, ATTN_SOURCES)
     pooled_bytes = 2 * rows * shape.d * 8
     if raster:
         # pooling reads Q and K and writes the means; nothing else moves
@@ -349,9 +382,13 @@ def run_gpu(args, rank, world, local_rank):
     hbm["peak"] = peak_gbs
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False,
+        "scaling": "strong" if shard == "heads" else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {**wl.describe(), "parallelism": f"replicas{world}" if world > 1 else "single",
+        "config": {**wl.describe(),
+                   "parallelism": (f"{shard}{world}" if world > 1 else "single"),
+                   **({"heads_per_rank": [wl.heads * r // world for r in range(world + 1)]}
+                      if shard == "heads" else {}),
                    "l2": "256 MiB flush written between timed steps; Q/K/V 2.5 GB > L2",
                    "layout": args.layout, "step": step_desc},
         "kept_tile_tflops": achieved_tf,
@@ -359,12 +396,12 @@ def run_gpu(args, rank, world, local_rank):
         "kept_fraction": kept_frac,
         "kept_tiles": kept,
         "breakdown_ms": parts,
-        "roofline": {"bound": "tensor",
-                     "kernel": f"sparse_attn_kernel<{shape.d}, 0, {int(raster)}>",
-                     "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
-                     "frac": achieved_tf / peak_tf, "traffic": traffic,
-                     "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long loop)",
-                     "frac_of_burst": achieved_tf / burst_tf,
+        "roofline": {"bound": "tensor", "kernel": attn_kernel,
+                     "achieved": achieved_tf, "peak": burst_tf, "unit": "TFLOP/s",
+                     "frac": achieved_tf / burst_tf, "traffic": traffic,
+                     "peak_source": f"{peak_src} bf16 burst (one launch timed by CUDA events)",
+                     "frac_of_sustained": achieved_tf / sus_tf,
+                     "algorithmic_bytes": 4 * tensor_bytes + rows * 4 * 64,
                      "flop_per_kept_tile": flop_per_tile},
         # HBM kernels: algorithmic bytes / time (read + write, each byte once)
         "hbm_gbs": hbm,
@@ -398,7 +435,7 @@ def run_sweep(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=qd.device)
     stream = torch.cuda.current_stream()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-    burst_tf, peak_tf, _, peak_src = measured_peaks()
+    peak_tf, _, _, peak_src = measured_peaks()       # burst: single timed launches
     flop_per_tile = 4 * 64 * 64 * shape.d
     steps = max(args.steps, 1)
     k10 = shape.Nb // 10
@@ -472,7 +509,7 @@ def run_sweep(args):
             "query_blocks": int(qblocks.numel()) if qblocks is not None else rows_all,
             "mask_ms": t_mask, "sparse_attn_ms": t_attn, "kept_tile_tflops": tf,
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peak_tf, "frac": tf / peak_tf,
-                         "peak_source": f"{peak_src} bf16 sustained"},
+                         "peak_source": f"{peak_src} bf16 burst"},
             "clocks": clk.summary()}), flush=True)
     # the semantic-aware permutation path, on the raster inputs
     print(json.dumps(run_cluster_point(args, qd, kd, vd, shape, peak_tf, peak_src,
@@ -525,7 +562,7 @@ def run_cluster_point(args, q, k, v, shape, peak_tf, peak_src, params):
         "padded_tiles": tiles,
         "tflops_useful_pairs_whole_call": pairs * 4 * shape.d / (ms * 1e-3) / 1e12,
         "tflops_padded_tiles_whole_call": tiles * flop_tile / (ms * 1e-3) / 1e12,
-        "peak": peak_tf, "peak_source": f"{peak_src} bf16 sustained",
+        "peak": peak_tf, "peak_source": f"{peak_src} bf16 burst",
         "clocks": clk.summary()}
 
 
@@ -615,7 +652,7 @@ def main():
                 wl = workloads.get(WORKLOAD)
                 shape = vsa.Shape.of(wl)
                 q, k, v = (x.cuda() for x in workloads.make_qkv(wl))
-                _, peak_tf, _, peak_src = measured_peaks()
+                peak_tf, _, _, peak_src = measured_peaks()
                 print(json.dumps(run_cluster_point(args, q, k, v, shape, peak_tf, peak_src,
                                                    vsa.ClusterParams(256, 512, 2, 0.9))),
                       flush=True)

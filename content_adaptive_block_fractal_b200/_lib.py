@@ -25,7 +25,7 @@ EXPORTS = ("vsa_fractal_flatten", "vsa_fractal_unflatten", "vsa_pool_qk",
            "vsa_sparse_attn_fwd_noalloc", "vsa_sparse_attn_fwd_rows",
            "vsa_sparse_attn_fwd_raster",
            "vsa_cluster_attn_workspace_size", "vsa_cluster_attn_fwd",
-           "vsa_last_error", "vsa_device_status", "vsa_version")
+           "vsa_last_error", "vsa_device_status", "vsa_wait_probe", "vsa_version")
 
 
 class vsa_cluster_params(ctypes.Structure):
@@ -90,6 +90,7 @@ def load():
         "vsa_sparse_attn_fwd_noalloc": [P, P, P, P, P, vsa_shape, F, P, P, P],
         "vsa_sparse_attn_fwd_rows": [P, P, P, P, P, vsa_shape, F, P, I64, P, P, P, S, P],
         "vsa_device_status": [P],
+        "vsa_wait_probe": [I64, P],
         "vsa_cluster_attn_fwd": [P, P, P, vsa_shape, vsa_cluster_params, F, P, P, P, P,
                                  ctypes.POINTER(vsa_cluster_state), P, S, P],
     }.items():

@@ -1,87 +1,102 @@
 // k_mask.cu -- content-adaptive block mask (NABLA, Methodology item 2:
 // reduced attention over pooled blocks and the per-row CDF threshold; item 3:
-// union with the sliding-tile window; Sparse VideoGen2 section 2B: top-p).
+// union with the sliding-tile window; Sparse VideoGen2 section 2B: top-p;
+// DynamicRad section 2, Static-Ratio mode: a fixed number of blocks per row).
 //
-// Four kernels:
-//   mask_scores_kernel  persistent; one work unit = 64 query blocks x 128 key
-//                       blocks of one (batch, head), units split evenly over
-//                       the CTAs.  Forms the pooled scores with fp64
-//                       tensor-core MMAs (m8n8k4), K streamed in slices,
-//                       writes each tile's row maxima in fp64 and
-//                       2^(t - tile max) as fp32 to the workspace slab.
-//   mask_select_kernel  one warp per row: rescales the slab row to the row
-//                       maximum, finds the CDF cut (histogram of the top 8
-//                       octaves + exact fp64 check + warp sort of the cut
-//                       bin, or bisection on the fp32 bit pattern with fp64
-//                       mass tests), breaks ties by index, ORs in the STA
-//                       window and writes a kept-bit row and its count.  Small
-//                       SMEM per warp, so many rows are in flight per SM.
-//   chunk_sums_kernel, chunk_scan_kernel
-//                       exclusive scan of the counts into row_ptr (int64).
-//   expand_bits_kernel  kept bits -> ascending col_idx lists.
+// Exact scores from integer tensor-core products.  Every pooled row x (fp64,
+// d values) is written as y = x * 2^(6-e), max|x| < 2^e, and split into four
+// signed base-2^7 digits:
+//     y = D0 + D1 b + D2 b^2 + D3 b^3 + rho b^3,   b = 2^-7, |Dj| <= 64, |rho| <= 1/2
+// (each step exact in fp64).  The score q.k = 2^(eq+ek-12) sum_i y_i y'_i is
+// then, up to the dropped products of weight b^4 and below, the fixed-point
+// value  A0 + b A1 + b^2 A2 + b^3 A3,  A_k = sum_{j+l=k} Dq_j . Dk_l, whose ten
+// int8 dot products are exact int32 tcgen05.mma (kind::i8) results.  Per term
+// the dropped part is at most 4096 (3 b^4 + 2 b^5 + b^6) + 64.001 b^3 < 7.7e-5,
+// so |score error| <= d * 7.7e-5 * 2^(eq+ek-12): a bound that holds for every
+// input, not an estimate.  With the fp32 combination of the A_k and the
+// scaling, each log2-score t carries a known error bound eps (per row).
 //
-// Precision: scores are exact fp64 dot products of exact pooled means; each
-// probability carries a relative error of a few 1e-7 (fp32 storage and the
-// hardware exp2 on a reduced argument), so the kept set equals the exact one
-// except for rows whose cut is within that of 1 - thr or of a tie.
+// Kernels, in launch order:
+//   mask_digits_kernel   fp64 Qp, Kp -> int8 digit planes [4][rows][128] and
+//                        per-row exponents (a warp per row).
+//   mask_scores_kernel   persistent, warp-specialised; a work unit is 128
+//                        query blocks of one head.  TMA loads the Q digit tile
+//                        once and the K digit chunks (64 key blocks) into a
+//                        4-deep ring; one thread issues the 40 int8 MMAs of a
+//                        chunk into one of two TMEM accumulator sets; sixteen
+//                        epilogue warps (thread = query row, 16 columns each)
+//                        combine the four class accumulators into the fp32
+//                        log2-score t = s log2(e) and store it to a row-major
+//                        score slab, with the row's max, min and eps.
+//   mask_select_kernel   a warp per row (rows in reverse, so the most recently
+//                        written part of the slab is still in L2): 2^(t - R)
+//                        in SMEM and their exact fp64 sum; 1/8-octave bins of
+//                        those values, window by window (8 octaves each), find
+//                        the bin holding the cut; one exact pass marks the
+//                        blocks above it and collects the bin's blocks, which
+//                        are sorted (t desc, index asc) and cut.  A row whose
+//                        decision is not certain under eps (a near tie at the
+//                        cut, a cut mass within the error of 1 - thr, an
+//                        overfull cut bin) is listed for the recheck instead.
+//                        Then the STA union, the kept-bit row and its count.
+//   mask_recheck_kernel  a CTA per listed row: the oracle's computation in
+//                        fp64 (scores, softmax, sort by probability then
+//                        index, prefix mass), kept bits, STA union, count.
+//   chunk_sums_kernel, chunk_scan_kernel, expand_bits_kernel
+//                        counts -> row_ptr (int64) -> ascending col_idx.
 #include "vsa_device.cuh"
 #include "vsa_internal.h"
+#include "vsa_tma.h"
 
+#include <climits>
 #include <cmath>
-#include <type_traits>
 
 namespace vsa {
 namespace {
 
-constexpr int kRT = 64;       // query blocks per work item
-constexpr int kCT = 128;      // key blocks per phase-A column tile
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
-constexpr int kPad = 4;       // fp64 padding per smem row (conflict-free fragments)
-constexpr int kKS = 32;       // columns of d per K slice in the score kernel
-constexpr int kLdK = kKS + kPad;
-constexpr int kCand = 256;    // per-warp candidate list capacity
-constexpr int kBins = 64;     // 1/8-octave probability bins (8 octaves below the max)
-constexpr int kMaxWords = 256;  // kept-bit words per row held in SMEM (Nb <= 8192)
-constexpr int kOctaves = 256;   // fp32 exponent bins of the static-ratio selection
-constexpr int kMaxGrid = 160; // persistent score CTAs
+constexpr int kDigits = 4;        // digit planes per pooled tensor
+constexpr int kRowBytes = 128;    // one digit row: d int8 values, zero-padded to 128
+constexpr int kTileRows = 128;    // query blocks per work unit (MMA M)
+constexpr int kChunk = 64;        // key blocks per MMA chunk (MMA N)
+constexpr int kStages = 4;        // K chunk ring
+constexpr int kEpiWarps = 16;     // four per TMEM lane quarter, 16 columns each
+constexpr int kThreadsA = (2 + kEpiWarps) * 32;
+constexpr int kEpiBarrier = 1;    // named barrier of the epilogue warps
+constexpr int kSelWarps = 8;      // rows in flight per select CTA
+constexpr int kWin = 64;          // 1/8-octave bins per window (8 octaves)
+constexpr int kCand = 64;         // cut-bin blocks sorted per row
+constexpr int kMaxNb = 8192;      // blocks per head (kept-bit rows and per-warp rows in SMEM)
 
-struct MaskArgs {
-  const double *qp, *kp;
-  int64_t BH;
-  int Nb, d, Hb, Wb;
-  float thr;
-  int use_sta, rt, rh, rw;
-  double c;          // scale * log2(e)
-  float *slab;       // [BH*Nb][ld_slab]
-  double *tmax;      // [BH*Nb][ntiles]
-  int ld_slab, ntiles;
-  uint32_t *bits;    // [BH*Nb][words]
-  int words;
-  int32_t *counts;   // [BH*Nb]
-  int64_t items, tiles_per_head;
-  int k;             // static-ratio selection: blocks kept per row (0: top-p)
+struct RowRec {
+  float tmax, tmin;   // extremes of the row's log2-scores
+  float eps;          // error bound of every t of the row (log2 units)
+  int pad;
 };
 
-__device__ __forceinline__ void dmma(double (&c)[2], double a, double b) {
-  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
-               : "+d"(c[0]), "+d"(c[1])
-               : "d"(a), "d"(b));
-}
-
-__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool valid) {
-  const uint32_t s = smem_u32(smem);
-  const int n = valid ? 16 : 0;  // src size 0 -> zero fill
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem), "r"(n)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
+struct MaskArgs {
+  int64_t BH, rows;
+  int Nb, d, Hb, Wb, T;
+  float thr;        // top-p threshold (topk == 0)
+  int topk;         // static ratio: blocks per row (0: top-p)
+  int use_sta, rt, rh, rw;
+  float c_log2;     // log2(e) / sqrt(d)
+  double scale;     // 1 / sqrt(d), the recheck's fp64 scale
+  const double *qp, *kp;
+  const int *qexp, *kexp;
+  const float *kscale;      // [BH][ldk]: 2^(K row exponent), exact
+  int ldk;
+  float *slab;              // [rows][ld] log2-scores
+  int ld;
+  RowRec *rec;              // [rows]
+  uint32_t *bits;           // [rows][words]
+  int words;
+  int32_t *counts;          // [rows]
+  int32_t *flagged;         // rows listed for the recheck
+  int *nflag;
+  int tiles_per_head, nch, np2;
+  int64_t units;
+  unsigned *err;
+};
 
 __device__ __forceinline__ double warp_sum(double v) {
 #pragma unroll
@@ -99,684 +114,917 @@ __device__ __forceinline__ int warp_sum_i(int v) {
   return v;
 }
 
-// 2^x for x <= 0 in fp64 argument, fp32 result with relative error ~2e-7:
-// split x = n + f with f in [0, 1), hardware exp2 of f, exact scaling by 2^n.
-__device__ __forceinline__ float exp2_split(double x) {
-  if (!(x > -126.0)) return 0.0f;  // also maps -inf / NaN to 0
-  const double n = floor(x);
-  const float f = static_cast<float>(x - n);
-  return ex2(f) * __int_as_float((static_cast<int>(n) + 127) << 23);
+__device__ __forceinline__ void epi_sync() {
+  asm volatile("bar.sync %0, %1;" ::"n"(kEpiBarrier), "n"(kEpiWarps * 32) : "memory");
 }
 
-// key = bits of a probability in [0, 1]; bin 0 holds (7/8, 1], each bin is
-// 1/8 octave; kBins (the tail) collects everything more than 8 octaves down.
-__device__ __forceinline__ int prob_bin(uint32_t key) {
-  const uint32_t d = key < 0x3F800000u ? 0x3F800000u - key : 0u;
-  const uint32_t b = d >> 20;
-  return b < static_cast<uint32_t>(kBins) ? static_cast<int>(b) : kBins;
+// exact int32 -> fp32 for |a| < 2^22
+__device__ __forceinline__ float i2f_small(int32_t a) {
+  return __int_as_float(a + 0x4B400000) - 12582912.0f;
 }
 
-// A row's probabilities relative to the row maximum: the slab entry (fp32
-// 2^(s - tile max), L2-resident) times its tile's fp32 rescale factor.  Read
-// again wherever a pass needs them rather than kept in SMEM, so that many
-// more rows fit on an SM; the product is the same every time.
-struct RowView {
-  const float *slab;
-  const float *ts;
-  __device__ __forceinline__ float operator()(int c) const { return slab[c] * ts[c / kCT]; }
-};
-// The same values kept in SMEM by the first pass (rows short enough that the
-// copy costs little occupancy).
-struct SmemRow {
-  const float *e;
-  __device__ __forceinline__ float operator()(int c) const { return e[c]; }
-};
-constexpr int kSmemRowMaxNb = 2048;   // rows up to this many blocks stay in SMEM
+// D[tmem] (+)= A[smem] . B[smem] with s8 operands, s32 accumulate.
+__device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(static_cast<uint32_t>(accumulate))
+      : "memory");
+}
 
-// The cut by bisection on the fp32 bit pattern, mass tests in fp64.  Sets
-// vkey (cut value) and need_ties, or keep_all when the sums never reach the
-// target.  General path; used when the histogram path cannot decide.
-template <class Row>
-__device__ void cut_by_bisection(int Nb, Row ebuf, uint32_t kmax, double target,
-                                 uint32_t *cand_key, int32_t *cand_idx, uint32_t &vkey,
-                                 int &need_ties, bool &keep_all) {
+// Instruction descriptor for kind::i8: s32 accumulator, s8 A and B, K-major.
+__host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
+  return (2u << 4)                                   // D format: s32
+         | (1u << 7)                                 // A: s8
+         | (1u << 10)                                // B: s8
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
+#define VSA_R16(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), \
+                   "=r"(r[i + 4]), "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7]), \
+                   "=r"(r[i + 8]), "=r"(r[i + 9]), "=r"(r[i + 10]), "=r"(r[i + 11]), \
+                   "=r"(r[i + 12]), "=r"(r[i + 13]), "=r"(r[i + 14]), "=r"(r[i + 15])
+// 16 columns at each of two TMEM addresses, one wait for both.
+__device__ __forceinline__ void tmem_ld2x16(uint32_t a0, uint32_t a1, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : VSA_R16(0), VSA_R16(16)
+      : "r"(a0), "r"(a1)
+      : "memory");
+}
+#undef VSA_R16
+
+// ---------------------------------------------------------------- digits
+// A warp per pooled row (Q rows first, then K rows); lane l converts values
+// 4l .. 4l+3 and writes byte 4l.. of each digit row (zeros past d).
+__global__ void __launch_bounds__(256)
+    mask_digits_kernel(const double *__restrict__ qp, const double *__restrict__ kp,
+                       int64_t rows, int64_t plane_rows, int d, int Nb, int ldk,
+                       int8_t *__restrict__ qdig, int8_t *__restrict__ kdig,
+                       int *__restrict__ qexp, int *__restrict__ kexp,
+                       float *__restrict__ kscale, int *nflag) {
   const int lane = threadIdx.x & 31;
-  // Invariant: the cut key lies in [lo, hi); mass(key >= hi) = base < target.
-  uint32_t lo = 0, hi = kmax + 1;
-  double base = 0.0;
-  int ncand = -1;  // -1: scan the whole row
-  for (int it = 0; hi - lo > 1; ++it) {
-    const uint32_t mid = lo + ((hi - lo) >> 1);
-    double up = 0.0;
-    if (ncand < 0) {
-      for (int c = lane; c < Nb; c += 32) {
-        const float e = ebuf(c);
-        const uint32_t k = __float_as_uint(e);
-        if (k >= mid && k < hi) up += static_cast<double>(e);
-      }
-    } else {
-      for (int i = lane; i < ncand; i += 32) {
-        const uint32_t k = cand_key[i];
-        if (k >= mid && k < hi) up += static_cast<double>(__uint_as_float(k));
-      }
+  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (w == 0 && lane == 0) *nflag = 0;
+  if (w >= 2 * rows) return;
+  const bool isk = w >= rows;
+  const int64_t row = isk ? w - rows : w;
+  const double *src = (isk ? kp : qp) + row * d;
+  double x[4] = {0.0, 0.0, 0.0, 0.0};
+  if (4 * lane < d) {
+    const double2 u = *reinterpret_cast<const double2 *>(src + 4 * lane);
+    const double2 v = *reinterpret_cast<const double2 *>(src + 4 * lane + 2);
+    x[0] = u.x; x[1] = u.y; x[2] = v.x; x[3] = v.y;
+  }
+  double m = fmax(fmax(fabs(x[0]), fabs(x[1])), fmax(fabs(x[2]), fabs(x[3])));
+  m = warp_max(m);
+  int e = 0;
+  if (m > 0.0) frexp(m, &e);           // m < 2^e
+  uint32_t packed[kDigits] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    double y = ldexp(x[i], 6 - e);       // |y| < 64, exact
+#pragma unroll
+    for (int j = 0; j < kDigits; ++j) {
+      const double dj = rint(y);         // |dj| <= 64
+      packed[j] |= (static_cast<uint32_t>(static_cast<int>(dj)) & 0xFFu) << (8 * i);
+      y = (y - dj) * 128.0;              // exact: |y - dj| <= 1/2
     }
-    up = warp_sum(up);
-    if (base + up >= target) {
-      lo = mid;
+  }
+  int8_t *dig = isk ? kdig : qdig;
+#pragma unroll
+  for (int j = 0; j < kDigits; ++j)
+    reinterpret_cast<uint32_t *>(dig + (static_cast<int64_t>(j) * plane_rows + row) * kRowBytes)[lane] =
+        packed[j];
+  if (lane == 0) {
+    if (isk) {
+      kexp[row] = e;
+      // per head, padded to ldk entries so a chunk's scales are aligned
+      kscale[(row / Nb) * ldk + row % Nb] = (e > -127 && e < 128) ? __int_as_float((e + 127) << 23) : 0.0f;
     } else {
-      base += up;
-      hi = mid;
+      qexp[row] = e;
     }
-    if (ncand < 0 && it >= 5) {
-      int cnt = 0;
-      for (int c = lane; c < Nb; c += 32) {
-        const uint32_t k = __float_as_uint(ebuf(c));
-        cnt += (k >= lo && k < hi);
-      }
-      cnt = warp_sum_i(cnt);
-      if (cnt <= kCand) {
-        int pos = 0;
-        for (int c0 = 0; c0 < Nb; c0 += 32) {
-          const int c = c0 + lane;
-          const uint32_t k = c < Nb ? __float_as_uint(ebuf(c)) : 0u;
-          const bool in = c < Nb && k >= lo && k < hi;
-          const uint32_t m = __ballot_sync(0xFFFFFFFFu, in);
-          if (in) {
-            const int p = pos + __popc(m & ((1u << lane) - 1u));
-            cand_key[p] = k;
-            cand_idx[p] = c;
+  }
+}
+
+// ---------------------------------------------------------------- scores
+struct SmemA {
+  static constexpr int kQBytes = kDigits * kTileRows * kRowBytes;   // 64 KiB
+  static constexpr int kKStage = kDigits * kChunk * kRowBytes;       // 32 KiB
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + kQBytes;
+  static constexpr int kX = kK + kStages * kKStage;   // per-slice max / min [2][4][128]
+  static constexpr int kXBytes = 2 * 4 * kTileRows * 4 + 64;
+  static constexpr int kBar = (kX + kXBytes + 7) & ~7;
+  // q_full q_empty k_full[4] k_empty[4] acc_full[2] acc_empty[2]
+  static constexpr int kNumBars = 2 + 2 * kStages + 4;
+  static constexpr int kTmemSlot = kBar + kNumBars * 8;
+  static constexpr int kAlloc = kTmemSlot + 16;
+  static_assert(kAlloc <= 232448, "mask score kernel shared memory exceeds 227 KiB");
+};
+
+// 18 warps: at most five share a scheduler's 16K registers, so 96 each
+__global__ void __maxnreg__(96)
+    mask_scores_kernel(const __grid_constant__ CUtensorMap tq,
+                       const __grid_constant__ CUtensorMap tk, const MaskArgs a) {
+  using L = SmemA;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(a.err, kErrSmemAlign);
+    return;
+  }
+  unsigned char *smem = smem_raw;
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar = sbase + L::kBar;
+  const uint32_t q_full = bar, q_empty = bar + 8;
+  auto k_full = [&](int s) { return bar + 16u + 8u * s; };
+  auto k_empty = [&](int s) { return bar + 16u + 8u * (kStages + s); };
+  auto acc_full = [&](int s) { return bar + 16u + 8u * (2 * kStages + s); };
+  auto acc_empty = [&](int s) { return bar + 16u + 8u * (2 * kStages + 2 + s); };
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemSlot);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(k_full(s), 1);
+      mbar_init(k_empty(s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(acc_full(s), 1);
+      mbar_init(acc_empty(s), kEpiWarps * 32);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tq);
+      tma_prefetch_desc(&tk);
+      int n = 0, uu = 0;
+      bool ok = true;
+      for (int64_t u = blockIdx.x; ok && u < a.units; u += gridDim.x, ++uu) {
+        const int64_t bh = u / a.tiles_per_head;
+        const int tile = static_cast<int>(u % a.tiles_per_head);
+        if (uu > 0 && !mbar_wait(q_empty, (uu - 1) & 1, a.err, kErrWaitMma)) break;
+        mbar_arrive_expect_tx(q_full, L::kQBytes);
+        tma_load_3d(sbase + L::kQ, &tq, q_full, 0,
+                    static_cast<int>(bh * a.Nb + tile * kTileRows), 0);
+        for (int j = 0; j < a.nch; ++j, ++n) {
+          const int s = n % kStages;
+          if (n >= kStages &&
+              !mbar_wait(k_empty(s), ((n - kStages) / kStages) & 1, a.err, kErrWaitMma)) {
+            ok = false;
+            break;
           }
-          pos += __popc(m);
+          mbar_arrive_expect_tx(k_full(s), L::kKStage);
+          tma_load_3d(sbase + L::kK + s * L::kKStage, &tk, k_full(s), 0,
+                      static_cast<int>(bh * a.Nb + j * kChunk), 0);
         }
-        ncand = pos;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t kIdesc = idesc_i8(kTileRows, kChunk);
+    // K-major, 128-byte swizzle: 8-row groups 1 KiB apart, K slices of 32
+    // bytes (2 units of 16 B) inside the 128-byte row
+    const uint64_t q_desc = smem_desc(sbase + L::kQ, 16, 1024);
+    const uint64_t k_desc = smem_desc(sbase + L::kK, 16, 1024);
+    constexpr uint32_t kQPlane = (kTileRows * kRowBytes) >> 4;
+    constexpr uint32_t kKPlane = (kChunk * kRowBytes) >> 4;
+    constexpr uint32_t kKStageU = L::kKStage >> 4;
+    const int ksteps = a.d / 32;
+    int n = 0, uu = 0;
+    bool ok = true;
+    for (int64_t u = blockIdx.x; ok && u < a.units; u += gridDim.x, ++uu) {
+      if (!mbar_wait(q_full, uu & 1, a.err, kErrWaitTma)) break;
+      for (int j = 0; j < a.nch; ++j, ++n) {
+        const int s = n % kStages, b = n & 1;
+        if (!mbar_wait(k_full(s), (n / kStages) & 1, a.err, kErrWaitTma) ||
+            (n >= 2 && !mbar_wait(acc_empty(b), ((n - 2) >> 1) & 1, a.err, kErrWaitSoftmax))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t acc = tmem + static_cast<uint32_t>(b) * 256u;
+          const uint64_t kd = k_desc + static_cast<uint32_t>(s) * kKStageU;
+#pragma unroll
+          for (int cls = 0; cls < kDigits; ++cls) {
+            bool first = true;
+#pragma unroll
+            for (int j2 = 0; j2 <= cls; ++j2) {
+              const int l = cls - j2;
+              for (int ks = 0; ks < ksteps; ++ks) {
+                mma_i8_ss(acc + cls * kChunk, q_desc + j2 * kQPlane + ks * 2,
+                          kd + l * kKPlane + ks * 2, kIdesc, !first);
+                first = false;
+              }
+            }
+          }
+          mma_commit(k_empty(s));
+          mma_commit(acc_full(b));
+          if (j == a.nch - 1) mma_commit(q_empty);
+        }
         __syncwarp();
       }
     }
-  }
-  vkey = lo;
-  if (vkey == 0u) {
-    keep_all = true;  // the sums never reach 1 - thr: keep every block
   } else {
-    const double v = static_cast<double>(__uint_as_float(vkey));
-    int j = static_cast<int>(ceil((target - base) / v));
-    if (j < 1) j = 1;
-    while (j > 1 && base + (j - 1) * v >= target) --j;
-    while (base + j * v < target && j < Nb) ++j;
-    need_ties = j;
-  }
-}
-
-// Phase B for one row: selection and kept bits.  ebuf: the row's probabilities
-// relative to the row max, re-read from the slab (RowView).
-//   1. those probabilities, their fp64 sum, and a
-//      histogram of counts / fp32 masses over 1/8-octave bins;
-//   2. the bin b where the cumulative mass reaches 1 - thr; an exact fp64 pass
-//      confirms base = mass above b < target <= base + mass of b and collects
-//      the bin's entries;
-//   3. with at most 32 entries: a warp bitonic sort on (probability desc,
-//      index asc) and an fp64 prefix scan mark the kept ones.  Otherwise (or
-//      if the fp32 histogram misled step 2) the bisection path decides.
-// Shared end of both selections: OR in the STA window, write the kept-bit
-// row and its count.  wbits holds the selection's bits (warp-synchronised).
-__device__ void finish_row(const MaskArgs &a, int64_t grow, int r, uint32_t *wbits) {
-  const int lane = threadIdx.x & 31;
-  const int Nb = a.Nb;
-  if (a.use_sta) {
-    // the window: at most (2rt+1)(2rh+1)(2rw+1) blocks around the row's own
-    const int hw = a.Hb * a.Wb;
-    const int tr = r / hw, yr = (r / a.Wb) % a.Hb, xr = r % a.Wb;
-    const int nt = 2 * a.rt + 1, ny = 2 * a.rh + 1, nx = 2 * a.rw + 1;
-    const int T = Nb / hw;
-    for (int i = lane; i < nt * ny * nx; i += 32) {
-      const int t = tr - a.rt + i / (ny * nx);
-      const int y = yr - a.rh + (i / nx) % ny;
-      const int x = xr - a.rw + i % nx;
-      if (t >= 0 && t < T && y >= 0 && y < a.Hb && x >= 0 && x < a.Wb) {
-        const int c = (t * a.Hb + y) * a.Wb + x;
-        atomicOr(&wbits[c >> 5], 1u << (c & 31));
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - 2;
+    const int slice = e >> 2;                  // 16-column slice of each chunk
+    const int quarter = warp & 3;              // TMEM lane quarter
+    const int row = quarter * 32 + lane;       // query row within the tile
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    float *x_mx = reinterpret_cast<float *>(smem + L::kX);   // [4][128]
+    float *x_mn = x_mx + 4 * kTileRows;                        // [4][128]
+    int *x_head = reinterpret_cast<int *>(x_mn + 4 * kTileRows);
+    const int tid = e * 32 + lane;
+    int n = 0;
+    // A wait that gives up clears ok; the warps then run the rest of their
+    // loops without waiting or writing, so every epilogue warp still reaches
+    // each named barrier and the CTA winds down.
+    bool ok = true;
+    for (int64_t u = blockIdx.x; u < a.units; u += gridDim.x) {
+      const int64_t bh = u / a.tiles_per_head;
+      const int tile = static_cast<int>(u % a.tiles_per_head);
+      const int r_local = tile * kTileRows + row;
+      const bool valid = r_local < a.Nb;
+      const int64_t g = bh * a.Nb + r_local;
+      // the head's largest K exponent (for the error bound)
+      {
+        int emax = INT_MIN;
+        for (int c = tid; c < a.Nb; c += kEpiWarps * 32) emax = max(emax, a.kexp[bh * a.Nb + c]);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) emax = max(emax, __shfl_xor_sync(0xFFFFFFFFu, emax, o));
+        if (tid == 0) x_head[0] = INT_MIN;
+        epi_sync();
+        if (lane == 0) atomicMax(&x_head[0], emax);
+        epi_sync();
       }
-    }
-    __syncwarp();
-  }
-  uint32_t *out = a.bits + grow * a.words;
-  int count = 0;
-  for (int w = lane; w < a.words; w += 32) {
-    const uint32_t word = wbits[w];
-    out[w] = word;
-    count += __popc(word);
-  }
-  count = warp_sum_i(count);
-  if (lane == 0) a.counts[grow] = count;
-  __syncwarp();
-}
-
-template <bool kSmemRow>
-__device__ void select_row(const MaskArgs &a, int64_t grow, int r, const float *slab_row,
-                           const double *tmax_row, float *erow, uint32_t *cand_key,
-                           int32_t *cand_idx, float *tscale, int *hcnt, float *hmass,
-                           uint32_t *wbits) {
-  const int lane = threadIdx.x & 31;
-  const int Nb = a.Nb;
-  // row maximum over the tile maxima, per-tile rescale factors in fp64
-  double M = -INFINITY;
-  for (int t = lane; t < a.ntiles; t += 32) M = fmax(M, tmax_row[t]);
-  M = warp_max(M);
-  for (int t = lane; t < a.ntiles; t += 32) tscale[t] = static_cast<float>(exp2(tmax_row[t] - M));
-  for (int b = lane; b < kBins; b += 32) {
-    hcnt[b] = 0;
-    hmass[b] = 0.0f;
-  }
-  __syncwarp();
-  using Row = typename std::conditional<kSmemRow, SmemRow, RowView>::type;
-  Row ebuf;
-  if constexpr (kSmemRow) ebuf = SmemRow{erow}; else ebuf = RowView{slab_row, tscale};
-  const bool need_cut = a.thr > 0.0f;
-  double z = 0.0;
-  uint32_t kmax = 0;
-  // the slab row sits in L2: 16-byte loads, four in flight per lane, before
-  // any use (the row is padded to a multiple of 4 floats)
-  constexpr int kU = 4;
-  for (int c0 = 4 * lane; c0 < Nb; c0 += 128 * kU) {
-    float4 v[kU];
+      const int ke_max = x_head[0];
+      const int qe = valid ? a.qexp[g] : 0;
+      const float rowf = ldexpf(a.c_log2, qe - 12);
+      const float *ks_head = a.kscale + bh * a.ldk;
+      float *srow = a.slab + g * a.ld;
+      float tmx = -INFINITY, tmn = INFINITY;
+      // the K scales of this thread's 16 columns, loaded one chunk ahead so
+      // the load is off the path from the accumulators to the stores
+      float4 ksn[4];
 #pragma unroll
-    for (int u = 0; u < kU; ++u)
-      if (c0 + 128 * u < Nb) v[u] = *reinterpret_cast<const float4 *>(slab_row + c0 + 128 * u);
+      for (int q = 0; q < 4; ++q)
+        ksn[q] = __ldg(reinterpret_cast<const float4 *>(ks_head + slice * 16) + q);
+      for (int j = 0; j < a.nch; ++j, ++n) {
+        const int b = n & 1;
+        if (ok && !mbar_wait(acc_full(b), (n >> 1) & 1, a.err, kErrWaitMma)) ok = false;
+        tc_fence_after();
+        // classes 3 and 2 first, then 1 and 0 (half the registers live)
+        const uint32_t base = lane_addr + static_cast<uint32_t>(b) * 256u + slice * 16;
+        uint32_t A[32];
+        float u[16];
+        tmem_ld2x16(base + 2 * kChunk, base + 3 * kChunk, A);
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const float x4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-      // the four entries share a 128-column tile (c0 is a multiple of 4)
-      const float ts = c0 + 128 * u < Nb ? tscale[(c0 + 128 * u) / kCT] : 0.0f;
-      float e4[4];
+        for (int i = 0; i < 16; ++i)
+          u[i] = fmaf(i2f_small(static_cast<int32_t>(A[16 + i])), 0.0078125f,
+                      i2f_small(static_cast<int32_t>(A[i])));
+        tmem_ld2x16(base, base + kChunk, A);
+        tc_fence_before();
+        mbar_arrive(acc_empty(b));
+        const int c0 = j * kChunk + slice * 16;
+        if (!ok || !valid || c0 >= a.Nb) continue;
+        float t[16];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) e4[j] = c0 + 128 * u + j < Nb ? x4[j] * ts : 0.0f;
-      // row mass: fp32 sums of four, fp64 across (relative error ~1e-7)
-      z += static_cast<double>((e4[0] + e4[1]) + (e4[2] + e4[3]));
+        for (int i = 0; i < 16; ++i) {
+          const float sfix = fmaf(fmaf(u[i], 0.0078125f, i2f_small(static_cast<int32_t>(A[16 + i]))),
+                                  0.0078125f, i2f_small(static_cast<int32_t>(A[i])));
+          const float4 kq = ksn[i >> 2];
+          const float ksi = (i & 3) == 0 ? kq.x : (i & 3) == 1 ? kq.y : (i & 3) == 2 ? kq.z : kq.w;
+          t[i] = sfix * ksi * rowf;
+        }
+        if (j + 1 < a.nch) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int c = c0 + 128 * u + j;
-        if (c < Nb) {
-          const float e = e4[j];
-          if constexpr (kSmemRow) erow[c] = e;
-          const uint32_t k = __float_as_uint(e);
-          kmax = max(kmax, k);
-          if (need_cut) {
-            const int b = prob_bin(k);
-            if (b < kBins) {         // the tail needs no histogram
-              atomicAdd(&hcnt[b], 1);
-              atomicAdd(&hmass[b], e);
+          for (int q = 0; q < 4; ++q)
+            ksn[q] = __ldg(reinterpret_cast<const float4 *>(ks_head + (j + 1) * kChunk + slice * 16) + q);
+        }
+        if (c0 + 16 <= a.Nb) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            tmx = fmaxf(tmx, t[i]);
+            tmn = fminf(tmn, t[i]);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            if (c0 + i < a.Nb) {
+              tmx = fmaxf(tmx, t[i]);
+              tmn = fminf(tmn, t[i]);
             }
           }
         }
+        // the row is padded to a multiple of 16 entries; padding is never read
+        float4 *dst = reinterpret_cast<float4 *>(srow + c0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          dst[q] = make_float4(t[4 * q], t[4 * q + 1], t[4 * q + 2], t[4 * q + 3]);
       }
+      x_mx[slice * kTileRows + row] = tmx;
+      x_mn[slice * kTileRows + row] = tmn;
+      epi_sync();
+      if (ok && slice == 0 && valid) {
+        float mx = x_mx[row], mn = x_mn[row];
+#pragma unroll
+        for (int s = 1; s < 4; ++s) {
+          mx = fmaxf(mx, x_mx[s * kTileRows + row]);
+          mn = fminf(mn, x_mn[s * kTileRows + row]);
+        }
+        const double tabs = fmax(fabs(static_cast<double>(mx)), fabs(static_cast<double>(mn)));
+        // error of a value 2^(t - R) in log2 units: d (7.7e-5 digit
+        // truncation + 5.9e-6 fp32 combination of the classes) in y units,
+        // times 2^(eq+ek-12) log2(e)/sqrt(d); the two fp32 roundings of t
+        // (2^-23 |t|), the rounding of t - R (2^-24 (|t| + |R|), |R| <= |t| + 1),
+        // the hardware exp2 (relative 2^-22, 3.4e-7 in log2 units) and the
+        // fp32 partial sums of four values in the row total (3 * 2^-24)
+        const double kr = ldexp(static_cast<double>(a.c_log2), qe + ke_max - 12);
+        const double eps = a.d * 8.3e-5 * kr + ldexp(tabs + 1.0, -22) + 7e-7;
+        const bool range_ok = qe > -100 && qe < 100 && ke_max < 100 && tabs < 1.0e5;
+        RowRec r;
+        r.tmax = mx;
+        r.tmin = mn;
+        r.eps = range_ok ? static_cast<float>(eps) : INFINITY;
+        r.pad = 0;
+        a.rec[g] = r;
+      }
+      // x_mx / x_mn are rewritten only after the next unit's two barriers
     }
   }
-  z = warp_sum(z);
-#pragma unroll
-  for (int o = 16; o; o >>= 1) kmax = max(kmax, __shfl_xor_sync(0xFFFFFFFFu, kmax, o));
-  __syncwarp();
 
-  bool keep_all = !need_cut;
-  uint32_t vkey = 0;
-  int need_ties = 0;
-  int cut_bin = -1;       // >= 0: the histogram path wrote the kept bits
-  if (!keep_all) {
-    const double target = (1.0 - static_cast<double>(a.thr)) * z;
-    // 2. cumulative bin masses (8 bins per lane, then a warp scan)
-    double loc = 0.0;
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- select
+// Bins of a value p = 2^(t - R) in [0, 1) from its fp32 bit pattern.  The
+// 1/8-octave bin: bin 0 holds [15/16, 1), larger bins smaller values, p = 0
+// falls in the last bin (1015).  The fine key splits every bin into 64
+// (key / 64 = bin).  Both are monotone: a larger p never has a larger key.
+__device__ __forceinline__ int value_bin(float p) {
+  const uint32_t k = __float_as_uint(p);
+  const int ex = static_cast<int>(k >> 23);      // biased exponent, <= 126 for p < 1
+  const int m3 = static_cast<int>((k >> 20) & 7u);
+  return (126 - ex) * 8 + (7 - m3);
+}
+__device__ __forceinline__ int value_key(float p) {
+  const uint32_t k = __float_as_uint(p);
+  const int ex = static_cast<int>(k >> 23);
+  const int m9 = static_cast<int>((k >> 14) & 511u);
+  return (126 - ex) * 512 + (511 - m9);
+}
+// t - R implied by p = 2^(t - R), with the bound of its error: fp32 rounding
+// of t - R and the hardware exp2 (relative 2^-21 at most)
+__device__ __forceinline__ double log2_of(float p) { return log2(static_cast<double>(p)); }
+__device__ __forceinline__ double log2_slack(double l) { return ldexp(fabs(l), -23) + 1e-6; }
+
+// Per-warp SMEM of the selection: the row's 2^(t - R), the window histogram,
+// the cut-bin candidates and the kept-bit row.
+__host__ __device__ inline size_t select_warp_bytes(int ldp, int words) {
+  return (static_cast<size_t>(ldp) * 4 + kWin * 4 + kCand * 8 + static_cast<size_t>(words) * 4 +
+          15) & ~static_cast<size_t>(15);
+}
+
+// Cumulative scan of the 64 bins of `hist` (two per lane) from `above`: the
+// first bin whose inclusive mass reaches `target`, or kWin - 1 (fp32 bin
+// sums only place the cut; exact passes confirm it).
+__device__ __forceinline__ int first_bin_reaching(const float *hist, double above, double target) {
+  const int lane = threadIdx.x & 31;
+  const double h0 = hist[2 * lane], h1 = hist[2 * lane + 1];
+  double incl = h0 + h1;
 #pragma unroll
-    for (int i = 0; i < kBins / 32; ++i) loc += static_cast<double>(hmass[lane * (kBins / 32) + i]);
-    double incl = loc;
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const double excl = incl - h0 - h1;
+  int found = 1 << 30;
+  if (above + excl + h0 >= target) found = 2 * lane;
+  else if (above + incl >= target) found = 2 * lane + 1;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const double y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    double run = incl - loc;
-    int found = kBins;
-#pragma unroll
-    for (int i = 0; i < kBins / 32; ++i) {
-      const int b = lane * (kBins / 32) + i;
-      run += static_cast<double>(hmass[b]);
-      if (found == kBins && run >= target) found = b;
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) found = min(found, __shfl_xor_sync(0xFFFFFFFFu, found, o));
-    bool decided = false;
-    if (found < kBins && hcnt[found] <= 32) {
-      // exact mass above the bin and the bin's entries
-      double base = 0.0;
-      int pos = 0;
-      for (int c0 = 0; c0 < Nb; c0 += 32) {
-        const int c = c0 + lane;
-        const float e = c < Nb ? ebuf(c) : 0.0f;
-        const int b = c < Nb ? prob_bin(__float_as_uint(e)) : kBins;
-        if (b < found) base += static_cast<double>(e);
-        // entries above the cut bin are kept whatever the bin's order
-        const uint32_t above = __ballot_sync(0xFFFFFFFFu, b < found);
-        if (lane == 0) wbits[c0 >> 5] = above;
-        const bool in = b == found;
-        const uint32_t m = __ballot_sync(0xFFFFFFFFu, in);
-        if (in) {
-          const int p = pos + __popc(m & ((1u << lane) - 1u));
-          if (p < 32) {
-            cand_key[p] = __float_as_uint(e);
-            cand_idx[p] = c;
-          }
-        }
-        pos += __popc(m);
-      }
-      base = warp_sum(base);
+  for (int o = 16; o; o >>= 1) found = min(found, __shfl_xor_sync(0xFFFFFFFFu, found, o));
+  return found < kWin ? found : kWin - 1;
+}
+
+// kCount: the static-ratio rule (the k largest), else top-p (mass 1 - thr).
+template <bool kCount>
+__global__ void __launch_bounds__(kSelWarps * 32) mask_select_kernel(const MaskArgs a, int ldp) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nw = blockDim.x >> 5;                 // rows in flight per CTA
+  unsigned char *wb = smem_raw + warp * select_warp_bytes(ldp, a.words);
+  float *ph = reinterpret_cast<float *>(wb);                   // [ldp]
+  float *hist = ph + ldp;                                      // [kWin]
+  int32_t *cand_c = reinterpret_cast<int32_t *>(hist + kWin);  // [kCand]
+  float *cand_t = reinterpret_cast<float *>(cand_c + kCand);   // [kCand]
+  uint32_t *bits = reinterpret_cast<uint32_t *>(cand_t + kCand);
+  const int Nb = a.Nb;
+  const bool keep_all_rule = kCount ? a.topk >= Nb : a.thr <= 0.0f;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * nw;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * nw + warp; i < a.rows; i += warps) {
+    const int64_t g = a.rows - 1 - i;          // newest slab rows first
+    const int r = static_cast<int>(g % Nb);
+    const float *srow = a.slab + g * a.ld;
+    bool recheck = false;
+    if (keep_all_rule) {
+      for (int w = lane; w < a.words; w += 32)
+        bits[w] = (w + 1) * 32 <= Nb ? 0xFFFFFFFFu : ((1u << (Nb & 31)) - 1u);
+    } else {
+      const RowRec rc = a.rec[g];
+      const double eps = rc.eps;
+      if (!(eps < 1.0) || !(fabsf(rc.tmax) < 1.0e5f)) recheck = true;
+      const int R = recheck ? 0 : static_cast<int>(floorf(rc.tmax)) + 1;   // every t < R
+      const float Rf = static_cast<float>(R);
+      // 1. the row's values 2^(t - R) in SMEM, their exact total and the
+      // histogram of the top window (8 octaves)
+      for (int b = lane; b < kWin; b += 32) hist[b] = 0.0f;
       __syncwarp();
-      if (pos <= 32 && base < target) {
-        // one entry per lane; sort by (probability desc, index asc)
-        uint64_t key = ~0ull;
-        if (lane < pos)
-          key = (static_cast<uint64_t>(0xFFFFFFFFu - cand_key[lane]) << 32) |
-                static_cast<uint32_t>(cand_idx[lane]);
+      double z = 0.0, wmass = 0.0;
+      if (!recheck) {
+        // 16-byte loads, two in flight per lane (the row is padded to 16)
+        for (int c0 = 4 * lane; c0 < Nb; c0 += 256) {
+          float4 v[2];
 #pragma unroll
-        for (int size = 2; size <= 32; size <<= 1)
+          for (int u = 0; u < 2; ++u)
+            if (c0 + 128 * u < Nb) v[u] = *reinterpret_cast<const float4 *>(srow + c0 + 128 * u);
 #pragma unroll
-          for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            const uint64_t other = __shfl_xor_sync(0xFFFFFFFFu, key, stride);
-            const bool up = (lane & size) == 0;
-            const bool lower = (lane & stride) == 0;
-            const uint64_t lo_v = key < other ? key : other;
-            const uint64_t hi_v = key < other ? other : key;
-            key = (lower == up) ? lo_v : hi_v;
+          for (int u = 0; u < 2; ++u) {
+            const int cb = c0 + 128 * u;
+            if (cb >= Nb) continue;
+            const float x4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+            float p4[4];
+            float z4 = 0.0f, w4 = 0.0f;    // fp32 sums of four, fp64 across
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const bool in = cb + q < Nb;
+              const float p = in ? ex2(x4[q] - Rf) : 0.0f;
+              p4[q] = p;
+              const float w = kCount ? (in ? 1.0f : 0.0f) : p;
+              z4 += w;
+              const int b = value_bin(p);
+              if (in && b < kWin) {
+                atomicAdd(&hist[b], w);
+                w4 += w;
+              }
+            }
+            z += static_cast<double>(z4);
+            wmass += static_cast<double>(w4);
+            // ph is padded to a multiple of 32 entries
+            *reinterpret_cast<float4 *>(ph + cb) = make_float4(p4[0], p4[1], p4[2], p4[3]);
           }
-        const bool valid = key != ~0ull;
-        const double p = valid ? static_cast<double>(__uint_as_float(0xFFFFFFFFu - static_cast<uint32_t>(key >> 32)))
-                               : 0.0;
-        double inc = p;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const double y = __shfl_up_sync(0xFFFFFFFFu, inc, o);
-          if (lane >= o) inc += y;
         }
-        const double total = __shfl_sync(0xFFFFFFFFu, inc, 31);
-        if (base + total >= target) {
-          // kept while the mass before the entry is still below the target
+        z = warp_sum(z);
+        wmass = warp_sum(wmass);
+      }
+      __syncwarp();
+      const double target = kCount ? static_cast<double>(a.topk)
+                                   : (1.0 - static_cast<double>(a.thr)) * z;
+      // 2. windows of 64 bins, top down, until one holds the cut
+      double above = 0.0;      // mass (count) of the windows above
+      int bstar = -1;
+      for (int wlo = 0; !recheck && bstar < 0 && wlo < 1024; wlo += kWin) {
+        if (wlo > 0) {
+          for (int b = lane; b < kWin; b += 32) hist[b] = 0.0f;
           __syncwarp();
-          if (valid && base + (inc - p) < target) {
-            const int c = static_cast<int>(key & 0xFFFFFFFFu);
-            atomicOr(&wbits[c >> 5], 1u << (c & 31));
+          wmass = 0.0;
+          for (int c = lane; c < Nb; c += 32) {
+            const float p = ph[c];
+            const int b = value_bin(p) - wlo;
+            if (b >= 0 && b < kWin) {
+              const float w = kCount ? 1.0f : p;
+              atomicAdd(&hist[b], w);
+              wmass += static_cast<double>(w);
+            }
           }
-          cut_bin = found;
-          decided = true;
+          wmass = warp_sum(wmass);
+          __syncwarp();
         }
+        if (above + wmass >= target) bstar = wlo + first_bin_reaching(hist, above, target);
+        else above += wmass;
         __syncwarp();
       }
-    }
-    if (!decided)
-      cut_by_bisection(Nb, ebuf, kmax, target, cand_key, cand_idx, vkey, need_ties, keep_all);
-  }
-
-  // kept bits (the histogram path wrote them already): everything, or above
-  // the bisection cut with ties by index
-  int ties_seen = 0;
-  for (int w = 0; cut_bin < 0 && w < a.words; ++w) {
-    const int c = w * 32 + lane;
-    const bool valid = c < Nb;
-    const uint32_t k = valid ? __float_as_uint(ebuf(c)) : 0u;
-    bool kept;
-    if (keep_all) {
-      kept = valid;
-    } else {
-      kept = valid && k > vkey;
-      const bool tie = valid && k == vkey;
-      const uint32_t tm = __ballot_sync(0xFFFFFFFFu, tie);
-      if (tie && ties_seen + __popc(tm & ((1u << lane) - 1u)) < need_ties) kept = true;
-      ties_seen += __popc(tm);
-    }
-    const uint32_t word = __ballot_sync(0xFFFFFFFFu, kept);
-    if (lane == 0) wbits[w] = word;
-  }
-  __syncwarp();
-  finish_row(a, grow, r, wbits);
-}
-
-// Work unit = (batch-head, 64-row tile, 128-column tile), numbered row-tile
-// major; CTA i takes the contiguous range [i*U/G, (i+1)*U/G), so the units
-// are spread evenly and a CTA meets a new row tile (and reloads Q) only a few
-// times.  K comes in slices of kKS columns of d through two cp.async buffers:
-// the next slice (the next unit's first one at a unit's end) is in flight
-// while the current one feeds the DMMAs.
-__global__ void __launch_bounds__(kThreads, 1) mask_scores_kernel(const MaskArgs a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  double *sQ = reinterpret_cast<double *>(smem_raw);
-  const int ld = a.d + kPad;
-  double *sK = sQ + kRT * ld;                  // [2][kCT][kLdK]
-  __shared__ double sRed[kRT][4];
-  __shared__ double sTileMax[kRT];
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int g = lane >> 2, tq = lane & 3;
-  const int wm = warp >> 2, wn = warp & 3;
-  const int nslices = a.d / kKS;
-  const int64_t units = a.items * a.ntiles;
-  const int64_t u_begin = units * blockIdx.x / gridDim.x;
-  const int64_t u_end = units * (blockIdx.x + 1) / gridDim.x;
-  if (u_begin >= u_end) return;
-
-  // K slice s (columns [s*kKS, s*kKS + kKS) of d) of unit u into buffer b
-  auto load_slice = [&](int64_t u, int sl, int b) {
-    const int64_t item = u / a.ntiles;
-    const int c0 = static_cast<int>(u % a.ntiles) * kCT;
-    const double *ksrc = a.kp + (item / a.tiles_per_head) * a.Nb * a.d + sl * kKS;
-    double *dst = sK + b * (kCT * kLdK);
-    for (int i = tid; i < kCT * (kKS / 2); i += kThreads) {
-      const int row = i / (kKS / 2), ch = i % (kKS / 2);
-      const bool ok = c0 + row < a.Nb;
-      cp_async16(dst + row * kLdK + ch * 2,
-                 ok ? ksrc + static_cast<int64_t>(c0 + row) * a.d + ch * 2 : a.kp, ok);
-    }
-    cp_async_commit();
-  };
-
-  load_slice(u_begin, 0, 0);
-  int buf = 0;
-  int64_t q_item = -1;
-  for (int64_t u = u_begin; u < u_end; ++u) {
-    const int64_t item = u / a.ntiles;
-    const int ct = static_cast<int>(u % a.ntiles);
-    const int64_t bh = item / a.tiles_per_head;
-    const int r0 = static_cast<int>(item % a.tiles_per_head) * kRT;
-    const int c0 = ct * kCT;
-    if (item != q_item) {
-      // every warp finished the previous unit (barrier at its end)
-      const double *qsrc = a.qp + (bh * a.Nb + r0) * a.d;
-      const int vec_per_row = a.d / 2;
-      for (int i = tid; i < kRT * vec_per_row; i += kThreads) {
-        const int row = i / vec_per_row, ch = i % vec_per_row;
-        const bool ok = r0 + row < a.Nb;
-        cp_async16(sQ + row * ld + ch * 2, ok ? qsrc + row * a.d + ch * 2 : a.qp, ok);
-      }
-      cp_async_commit();
-      q_item = item;
-    }
-
-    double acc[4][4][2];
-#pragma unroll
-    for (int mi = 0; mi < 4; ++mi)
-#pragma unroll
-      for (int ni = 0; ni < 4; ++ni) acc[mi][ni][0] = acc[mi][ni][1] = 0.0;
-    for (int sl = 0; sl < nslices; ++sl) {
-      // prefetch the next slice (the next unit's first at the last slice)
-      bool more = true;
-      if (sl + 1 < nslices) load_slice(u, sl + 1, buf ^ 1);
-      else if (u + 1 < u_end) load_slice(u + 1, 0, buf ^ 1);
-      else more = false;
-      // everything but the prefetch has landed: this slice (and Q)
-      if (more) cp_async_wait_group<1>();
-      else cp_async_wait_group<0>();
-      __syncthreads();
-      const double *qa = sQ + (wm * 32 + g) * ld + sl * kKS + tq;
-      const double *kb = sK + buf * (kCT * kLdK) + (wn * 32 + g) * kLdK + tq;
-#pragma unroll 2
-      for (int k = 0; k < kKS; k += 4) {
-        double af[4], bf[4];
-#pragma unroll
-        for (int mi = 0; mi < 4; ++mi) af[mi] = qa[mi * 8 * ld + k];
-#pragma unroll
-        for (int ni = 0; ni < 4; ++ni) bf[ni] = kb[ni * 8 * kLdK + k];
-#pragma unroll
-        for (int mi = 0; mi < 4; ++mi)
-#pragma unroll
-          for (int ni = 0; ni < 4; ++ni) dmma(acc[mi][ni], af[mi], bf[ni]);
-      }
-      __syncthreads();   // this buffer is refilled by the prefetch after next
-      buf ^= 1;
-    }
-
-    // scaled log2 scores; columns past Nb do not exist
-    float *slab = a.slab + (bh * a.Nb + r0) * a.ld_slab;
-    double *tmax = a.tmax + (bh * a.Nb + r0) * a.ntiles;
-#pragma unroll
-    for (int mi = 0; mi < 4; ++mi) {
-      double m = -INFINITY;
-#pragma unroll
-      for (int ni = 0; ni < 4; ++ni)
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int col = c0 + wn * 32 + ni * 8 + 2 * tq + j;
-          acc[mi][ni][j] = col < a.Nb ? acc[mi][ni][j] * a.c : -INFINITY;
-          m = fmax(m, acc[mi][ni][j]);
+      if (bstar < 0) recheck = true;     // the sums never reach the target
+      // 3. exact passes over the fine keys: bits of the blocks above the cut
+      // range [klo, khi), their exact mass, the nearest values on either
+      // side and the range's blocks, with a histogram of the range's 64 fine
+      // keys; a range with more blocks than the list holds is narrowed to
+      // the fine key holding the cut and passed once more
+      int ncand = 0;
+      double above_x = 0.0;
+      float pmin_above = INFINITY, pmax_below = 0.0f;
+      int klo = bstar * 64, khi = klo + 64;
+      auto exact_pass = [&]() {
+        for (int b = lane; b < kWin; b += 32) hist[b] = 0.0f;
+        __syncwarp();
+        ncand = 0;
+        above_x = 0.0;
+        pmin_above = INFINITY;
+        pmax_below = 0.0f;
+        for (int c0 = 0; c0 < a.words * 32; c0 += 32) {
+          const int c = c0 + lane;
+          const float p = c < Nb ? ph[c] : 0.0f;
+          const int k = c < Nb ? value_key(p) : 1 << 30;
+          const bool kept = k < klo;
+          if (kept) {
+            above_x += kCount ? 1.0 : static_cast<double>(p);
+            pmin_above = fminf(pmin_above, p);
+          } else if (k >= khi && c < Nb) {
+            pmax_below = fmaxf(pmax_below, p);
+          }
+          const uint32_t kw = __ballot_sync(0xFFFFFFFFu, kept);
+          if (lane == 0) bits[c0 >> 5] = kw;
+          const bool in = k >= klo && k < khi;
+          if (in && khi - klo == 64) atomicAdd(&hist[k - klo], kCount ? 1.0f : p);
+          const uint32_t m = __ballot_sync(0xFFFFFFFFu, in);
+          if (in) {
+            const int pos = ncand + __popc(m & ((1u << lane) - 1u));
+            if (pos < kCand) {
+              cand_c[pos] = c;
+              cand_t[pos] = srow[c];
+            }
+          }
+          ncand += __popc(m);
         }
-      m = fmax(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-      m = fmax(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-      if (tq == 0) sRed[wm * 32 + mi * 8 + g][wn] = m;
-    }
-    __syncthreads();
-    if (tid < kRT) {
-      const double m = fmax(fmax(sRed[tid][0], sRed[tid][1]), fmax(sRed[tid][2], sRed[tid][3]));
-      sTileMax[tid] = m;
-      if (r0 + tid < a.Nb) tmax[tid * a.ntiles + ct] = m;
-    }
-    __syncthreads();
+        above_x = warp_sum(above_x);
 #pragma unroll
-    for (int mi = 0; mi < 4; ++mi) {
-      const int row = wm * 32 + mi * 8 + g;
-      const double m = sTileMax[row];
+        for (int o = 16; o; o >>= 1) {
+          pmin_above = fminf(pmin_above, __shfl_xor_sync(0xFFFFFFFFu, pmin_above, o));
+          pmax_below = fmaxf(pmax_below, __shfl_xor_sync(0xFFFFFFFFu, pmax_below, o));
+        }
+        __syncwarp();
+      };
+      if (!recheck) {
+        exact_pass();
+        if (ncand > kCand && above_x < target) {
+          klo += first_bin_reaching(hist, above_x, target);
+          khi = klo + 1;
+          exact_pass();
+        }
+        if (ncand == 0 || ncand > kCand || !(above_x < target)) recheck = true;
+      }
+      // 4. sort the cut bin (t desc, index asc) and cut it
+      if (!recheck) {
+        uint64_t key[2];
 #pragma unroll
-      for (int ni = 0; ni < 4; ++ni) {
-        const int col = c0 + wn * 32 + ni * 8 + 2 * tq;
-        if (col < a.Nb && r0 + row < a.Nb) {
-          float2 e;
-          e.x = exp2_split(acc[mi][ni][0] - m);
-          e.y = exp2_split(acc[mi][ni][1] - m);
-          *reinterpret_cast<float2 *>(slab + row * a.ld_slab + col) = e;
+        for (int h = 0; h < 2; ++h) {
+          const int v = 2 * lane + h;
+          if (v < ncand) {
+            uint32_t o = __float_as_uint(cand_t[v]);
+            o = (o & 0x80000000u) ? ~o : (o | 0x80000000u);     // orders like t
+            key[h] = (static_cast<uint64_t>(~o) << 32) | static_cast<uint32_t>(cand_c[v]);
+          } else {
+            key[h] = ~0ull;
+          }
+        }
+        // bitonic sort of 64 keys, ascending, key h of lane l at position 2l + h
+#pragma unroll
+        for (int size = 2; size <= 64; size <<= 1) {
+#pragma unroll
+          for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            if (stride == 1) {
+              const bool up = ((2 * lane) & size) == 0;
+              const uint64_t lo = key[0] < key[1] ? key[0] : key[1];
+              const uint64_t hi = key[0] < key[1] ? key[1] : key[0];
+              key[0] = up ? lo : hi;
+              key[1] = up ? hi : lo;
+            } else {
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int pos = 2 * lane + h;
+                const uint64_t other = __shfl_xor_sync(0xFFFFFFFFu, key[h], stride >> 1);
+                const bool up = (pos & size) == 0;
+                const bool lower = (pos & stride) == 0;
+                const uint64_t lo = key[h] < other ? key[h] : other;
+                const uint64_t hi = key[h] < other ? other : key[h];
+                key[h] = (lower == up) ? lo : hi;
+              }
+            }
+          }
+        }
+        double pp[2];
+        float tt[2];
+        int cc[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const bool vld = key[h] != ~0ull;
+          cc[h] = vld ? static_cast<int>(key[h] & 0xFFFFFFFFu) : -1;
+          tt[h] = vld ? srow[cc[h]] : -INFINITY;
+          pp[h] = vld ? (kCount ? 1.0 : static_cast<double>(ph[cc[h]])) : 0.0;
+        }
+        double incl = pp[0] + pp[1];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const double y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const double ex0 = incl - pp[0] - pp[1];
+        // first position whose inclusive mass (count) reaches the target
+        int first = 1 << 30;
+        if (cc[0] >= 0 && above_x + ex0 + pp[0] >= target) first = 2 * lane;
+        else if (cc[1] >= 0 && above_x + incl >= target) first = 2 * lane + 1;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) first = min(first, __shfl_xor_sync(0xFFFFFFFFu, first, o));
+        if (first >= ncand) {
+          recheck = true;
+        } else {
+          const int keep_n = first + 1;
+          const int la = first >> 1, ha = first & 1;
+          const float ta = __shfl_sync(0xFFFFFFFFu, ha ? tt[1] : tt[0], la);
+          const double pa = __shfl_sync(0xFFFFFFFFu, ha ? pp[1] : pp[0], la);
+          const double mk = above_x + __shfl_sync(0xFFFFFFFFu, ha ? incl : ex0 + pp[0], la);
+          // smallest kept and largest dropped log2-scores, bounded from the
+          // values of the neighbouring bins where they are not in the list
+          double ta_eff = ta, tb_eff = -INFINITY;
+          if (pmin_above < INFINITY) {
+            const double l = log2_of(pmin_above);
+            ta_eff = fmin(ta_eff, R + l - log2_slack(l));
+          }
+          if (keep_n < ncand) {
+            const int lb = keep_n >> 1, hb = keep_n & 1;
+            tb_eff = __shfl_sync(0xFFFFFFFFu, hb ? tt[1] : tt[0], lb);
+          }
+          if (pmax_below > 0.0f) {
+            const double l = log2_of(pmax_below);
+            tb_eff = fmax(tb_eff, R + l + log2_slack(l));
+          } else if (pmax_below == 0.0f && keep_n == ncand) {
+            // dropped blocks whose value underflowed to 0 lie below 2^-126
+            tb_eff = fmax(tb_eff, R - 126.0);
+          }
+          // the kept blocks are apart from the dropped ones by more than the
+          // error of both; the kept mass reaches the target, and falls short
+          // of it without its smallest member, under every admissible error
+          if (!(ta_eff - tb_eff > 2.0 * eps)) recheck = true;
+          if (!kCount) {
+            const double grow2 = exp2(2.0 * eps);
+            if (!(mk >= target * grow2) || !(mk * grow2 - pa < target)) recheck = true;
+          }
+          if (!recheck) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              if (2 * lane + h < keep_n) atomicOr(&bits[cc[h] >> 5], 1u << (cc[h] & 31));
+          }
         }
       }
+      __syncwarp();
     }
-    // sRed / sTileMax and sQ are reused by the next unit
-    __syncthreads();
-  }
-}
-
-// One warp per row of the mask: selection and kept bits.
-// Static-ratio selection of one row (DynamicRad, "Dual-Mode Strategy",
-// Static-Ratio mode; reading: the k most probable blocks, equal probabilities
-// to the lower index, k >= Nb keeps the row).  The probabilities are positive
-// fp32 values, so their bit patterns order like the values: a histogram of
-// the exponent field finds the octave holding the k-th largest, a bisection
-// over that octave's 2^23 patterns (on its members, compacted when there are
-// at most kCand) finds the k-th largest pattern, and equal patterns at the cut
-// are taken in index order.
-template <bool kSmemRow>
-__device__ void select_row_topk(const MaskArgs &a, int64_t grow, int r, const float *slab_row,
-                                const double *tmax_row, float *erow, uint32_t *cand_key,
-                                int32_t *cand_idx, float *tscale, int *hist, uint32_t *wbits) {
-  const int lane = threadIdx.x & 31;
-  const int Nb = a.Nb, k = a.k;
-  double M = -INFINITY;
-  for (int t = lane; t < a.ntiles; t += 32) M = fmax(M, tmax_row[t]);
-  M = warp_max(M);
-  for (int t = lane; t < a.ntiles; t += 32) tscale[t] = static_cast<float>(exp2(tmax_row[t] - M));
-  for (int b = lane; b < kOctaves; b += 32) hist[b] = 0;
-  __syncwarp();
-  using Row = typename std::conditional<kSmemRow, SmemRow, RowView>::type;
-  Row ebuf;
-  if constexpr (kSmemRow) ebuf = SmemRow{erow}; else ebuf = RowView{slab_row, tscale};
-  const bool keep_all = k >= Nb;
-  for (int c = lane; c < Nb; c += 32) {
-    const float e = slab_row[c] * tscale[c / kCT];
-    if constexpr (kSmemRow) erow[c] = e;
-    if (!keep_all) atomicAdd(&hist[__float_as_uint(e) >> 23], 1);
-  }
-  __syncwarp();
-
-  bool bits_done = false;
-  uint32_t vkey = 0;
-  int need_ties = 0;
-  if (!keep_all) {
-    // lane l owns exponent bins 255-8l .. 248-8l: lane order = descending values
-    int loc = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) loc += hist[kOctaves - 1 - 8 * lane - i];
-    int incl = loc;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int run = incl - loc, found = -1, above = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int b = kOctaves - 1 - 8 * lane - i;
-      if (found < 0 && run + hist[b] >= k) {
-        found = b;
-        above = run;
+    if (recheck) {
+      if (lane == 0) {
+        const int pos = atomicAdd(a.nflag, 1);
+        a.flagged[pos] = static_cast<int32_t>(g);
       }
-      run += hist[b];
+      __syncwarp();
+      continue;
     }
-    // the highest such bin (the lowest lane that found one); every entry is
-    // counted, so one exists as k < Nb
-    const uint32_t fm = __ballot_sync(0xFFFFFFFFu, found >= 0);
-    const int src = __ffs(fm) - 1;
-    found = __shfl_sync(0xFFFFFFFFu, found, src);
-    above = __shfl_sync(0xFFFFFFFFu, above, src);
-    const bool compact = hist[found] <= kCand;
-    // entries of higher octaves are kept whatever happens at the cut
-    int pos = 0;
-    for (int c0 = 0; c0 < Nb; c0 += 32) {
-      const int c = c0 + lane;
-      const int ex = c < Nb ? static_cast<int>(__float_as_uint(ebuf(c)) >> 23) : -1;
-      const uint32_t hi_word = __ballot_sync(0xFFFFFFFFu, ex > found);
-      if (lane == 0) wbits[c0 >> 5] = hi_word;
-      if (compact) {
-        const bool in = ex == found;
-        const uint32_t m = __ballot_sync(0xFFFFFFFFu, in);
-        if (in) {
-          const int p = pos + __popc(m & ((1u << lane) - 1u));
-          cand_key[p] = __float_as_uint(ebuf(c));
-          cand_idx[p] = c;
+    if (a.use_sta && !keep_all_rule) {
+      const int hw = a.Hb * a.Wb;
+      const int tr = r / hw, yr = (r / a.Wb) % a.Hb, xr = r % a.Wb;
+      const int nt = 2 * a.rt + 1, ny = 2 * a.rh + 1, nx = 2 * a.rw + 1;
+      for (int v = lane; v < nt * ny * nx; v += 32) {
+        const int t3 = tr - a.rt + v / (ny * nx);
+        const int yy = yr - a.rh + (v / nx) % ny;
+        const int xx = xr - a.rw + v % nx;
+        if (t3 >= 0 && t3 < a.T && yy >= 0 && yy < a.Hb && xx >= 0 && xx < a.Wb) {
+          const int c = (t3 * a.Hb + yy) * a.Wb + xx;
+          atomicOr(&bits[c >> 5], 1u << (c & 31));
         }
-        pos += __popc(m);
       }
     }
     __syncwarp();
-    // k-th largest pattern inside the octave: count(key >= hi) + above < k
-    // <= count(key >= lo) + above
-    uint32_t lo = static_cast<uint32_t>(found) << 23, hi = lo + (1u << 23);
-    int cnt_hi = 0;
-    while (hi - lo > 1) {
-      const uint32_t mid = lo + ((hi - lo) >> 1);
-      int cin = 0;
-      if (compact) {
-        for (int i = lane; i < pos; i += 32) cin += cand_key[i] >= mid && cand_key[i] < hi;
-      } else {
-        for (int c = lane; c < Nb; c += 32) {
-          const uint32_t key = __float_as_uint(ebuf(c));
-          cin += key >= mid && key < hi;
+    int count = 0;
+    for (int w = lane; w < a.words; w += 32) {
+      const uint32_t x = bits[w];
+      a.bits[g * a.words + w] = x;
+      count += __popc(x);
+    }
+    count = warp_sum_i(count);
+    if (lane == 0) a.counts[g] = count;
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------- recheck
+// The oracle's arithmetic for one listed row, a CTA per row: fp64 scores
+// scaled by 1/sqrt(d), softmax against the row maximum, and the kept set of
+// the sort on (probability desc, index asc) -- blocks taken while the mass
+// before them is below 1 - thr (top-p), or the first k (static ratio).  The
+// scores come from 64-key tiles of K staged in SMEM (coalesced loads; the next
+// tile is fetched into registers while the current one is used).  The cut
+// value is found by bisection on the bit patterns of the probabilities
+// (positive doubles order like their patterns) with fp64 mass (count) sums;
+// equal probabilities at the cut go to the lower indices.  Then the STA
+// union, the kept-bit row and its count.
+constexpr int kRcThreads = 256;
+constexpr int kRcTile = 64;       // keys per staged tile
+
+__host__ __device__ inline size_t recheck_smem_bytes(int ldp, int words, int d) {
+  return static_cast<size_t>(kRcTile) * (d + 4) * 8 + static_cast<size_t>(ldp) * 8 +
+         static_cast<size_t>(d) * 8 + ((static_cast<size_t>(words) * 4 + 15) & ~static_cast<size_t>(15));
+}
+
+__global__ void __launch_bounds__(kRcThreads) mask_recheck_kernel(const MaskArgs a, int ldp) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int d = a.d, Nb = a.Nb;
+  // padded tile rows: the 16 threads of a half-warp (4 keys x 4 quarters)
+  // read 16 distinct 8-byte banks
+  const int ldt = d + 4;
+  double *tile = reinterpret_cast<double *>(smem_raw);    // [kRcTile][d + 4]
+  double *pv = tile + kRcTile * ldt;                      // [ldp] scores, then probabilities
+  double *q = pv + ldp;                                   // [d]
+  uint32_t *bits = reinterpret_cast<uint32_t *>(q + d);   // [words]
+  __shared__ double red[kRcThreads / 32];
+  const int nf = *a.nflag;
+  // each thread moves 16-byte pieces: kRcTile * d / 2 pieces per tile,
+  // d / 2 = 2^hs pieces per key row
+  const int hs = d == 128 ? 6 : 5;
+  const int per_thread = (kRcTile << hs) / kRcThreads;    // 16 (d = 128) or 8 (d = 64)
+  for (int64_t fi = blockIdx.x; fi < nf; fi += gridDim.x) {
+    const int64_t g = a.flagged[fi];
+    const int64_t bh = g / Nb;
+    const int r = static_cast<int>(g % Nb);
+    const double *kbase = a.kp + bh * Nb * d;
+    for (int j = tid; j < d; j += kRcThreads) q[j] = a.qp[g * d + j];
+    double2 pre[16];
+    auto fetch = [&](int c0) {
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        if (u < per_thread) {
+          const int piece = tid + u * kRcThreads;
+          const int row = piece >> hs, col = piece & ((1 << hs) - 1);
+          pre[u] = c0 + row < Nb ? reinterpret_cast<const double2 *>(kbase + (c0 + row) * d)[col]
+                                 : make_double2(0.0, 0.0);
         }
       }
-      cin = warp_sum_i(cin);
-      if (above + cnt_hi + cin >= k) {
-        lo = mid;
+    };
+    fetch(0);
+    for (int c0 = 0; c0 < Nb; c0 += kRcTile) {
+      __syncthreads();                 // the previous tile has been used
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        if (u < per_thread) {
+          const int piece = tid + u * kRcThreads;
+          const int row = piece >> hs, col = piece & ((1 << hs) - 1);
+          tile[row * ldt + 2 * col] = pre[u].x;
+          tile[row * ldt + 2 * col + 1] = pre[u].y;
+        }
+      }
+      __syncthreads();
+      if (c0 + kRcTile < Nb) fetch(c0 + kRcTile);
+      // 4 threads per key, a quarter of d each, then a 4-lane reduction
+      const int key = tid >> 2, part = tid & 3;
+      double s = 0.0;
+      const double *kr = tile + key * ldt;
+      for (int j = part; j < d; j += 4) s = fma(q[j], kr[j], s);
+      s += __shfl_xor_sync(0xFFFFFFFFu, s, 1);
+      s += __shfl_xor_sync(0xFFFFFFFFu, s, 2);
+      if (part == 0 && c0 + key < Nb) pv[c0 + key] = s * a.scale;
+    }
+    __syncthreads();
+    // softmax against the row maximum (block reductions)
+    double m = -INFINITY;
+    for (int c = tid; c < Nb; c += kRcThreads) m = fmax(m, pv[c]);
+    m = warp_max(m);
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    m = red[0];
+    for (int w = 1; w < kRcThreads / 32; ++w) m = fmax(m, red[w]);
+    __syncthreads();
+    double z = 0.0;
+    for (int c = tid; c < Nb; c += kRcThreads) {
+      const double e = exp(pv[c] - m);
+      pv[c] = e;
+      z += e;
+    }
+    z = warp_sum(z);
+    if (lane == 0) red[warp] = z;
+    __syncthreads();
+    z = 0.0;
+    for (int w = 0; w < kRcThreads / 32; ++w) z += red[w];
+    for (int c = tid; c < Nb; c += kRcThreads) pv[c] /= z;
+    for (int w = tid; w < a.words; w += kRcThreads) bits[w] = 0u;
+    __syncthreads();
+    // the cut value: bisection over the probabilities' bit patterns with
+    // CTA-wide mass (count) sums
+    auto mass_at_least = [&](uint64_t key) {
+      double sum = 0.0;
+      for (int c = tid; c < Nb; c += kRcThreads) {
+        const uint64_t kc = static_cast<uint64_t>(__double_as_longlong(pv[c]));
+        if (kc >= key) sum += a.topk > 0 ? 1.0 : pv[c];
+      }
+      sum = warp_sum(sum);
+      __syncthreads();                   // red[] is free
+      if (lane == 0) red[warp] = sum;
+      __syncthreads();
+      double tot = 0.0;
+      for (int w = 0; w < kRcThreads / 32; ++w) tot += red[w];
+      return tot;
+    };
+    const double target = a.topk > 0 ? static_cast<double>(a.topk) : 1.0 - static_cast<double>(a.thr);
+    bool keep_all = a.topk > 0 ? a.topk >= Nb : !(a.thr > 0.0f);
+    uint64_t vkey = 0;
+    int need_ties = 0;
+    if (!keep_all) {
+      if (!(mass_at_least(0) >= target)) {
+        keep_all = true;                   // the sums never reach 1 - thr
       } else {
-        cnt_hi += cin;
-        hi = mid;
+        // invariant: mass(p >= lo) >= target > mass(p >= hi)
+        uint64_t lo = 0, hi = 0x7FF0000000000000ull;   // +inf: nothing is >= hi
+        while (hi - lo > 1) {
+          const uint64_t mid = lo + ((hi - lo) >> 1);
+          if (mass_at_least(mid) >= target) lo = mid; else hi = mid;
+        }
+        vkey = lo;                         // the cut value's pattern
+        const double base = mass_at_least(vkey + 1);   // strictly above the cut
+        const double v = a.topk > 0 ? 1.0 : __longlong_as_double(static_cast<long long>(vkey));
+        int j = static_cast<int>(fmin(ceil((target - base) / v), static_cast<double>(Nb)));
+        if (j < 1) j = 1;
+        while (j > 1 && base + (j - 1) * v >= target) --j;
+        while (base + j * v < target && j < Nb) ++j;
+        need_ties = j;
       }
     }
-    vkey = lo;
-    need_ties = k - (above + cnt_hi);   // >= 1 entries equal to vkey
-    if (compact) {
-      // members in ascending index order: patterns above vkey, then the
-      // first need_ties equal to it
+    // kept bits, ties in index order (warp 0 walks the words in order)
+    if (warp == 0) {
       int ties_seen = 0;
-      for (int i0 = 0; i0 < pos; i0 += 32) {
-        const int i = i0 + lane;
-        const uint32_t key = i < pos ? cand_key[i] : 0u;
-        bool kept = i < pos && key > vkey;
-        const bool tie = i < pos && key == vkey;
-        const uint32_t tm = __ballot_sync(0xFFFFFFFFu, tie);
-        if (tie && ties_seen + __popc(tm & ((1u << lane) - 1u)) < need_ties) kept = true;
-        ties_seen += __popc(tm);
-        if (kept) atomicOr(&wbits[cand_idx[i] >> 5], 1u << (cand_idx[i] & 31));
+      for (int w = 0; w < a.words; ++w) {
+        const int c = w * 32 + lane;
+        const bool valid = c < Nb;
+        bool kept;
+        if (keep_all) {
+          kept = valid;
+        } else {
+          const uint64_t kc = valid ? static_cast<uint64_t>(__double_as_longlong(pv[c])) : 0ull;
+          kept = valid && kc > vkey;
+          const bool tie = valid && kc == vkey;
+          const uint32_t tm = __ballot_sync(0xFFFFFFFFu, tie);
+          if (tie && ties_seen + __popc(tm & ((1u << lane) - 1u)) < need_ties) kept = true;
+          ties_seen += __popc(tm);
+        }
+        const uint32_t word = __ballot_sync(0xFFFFFFFFu, kept);
+        if (lane == 0) bits[w] = word;
       }
-      bits_done = true;
     }
-  }
-  if (!bits_done) {
-    int ties_seen = 0;
-    for (int w = 0; w < a.words; ++w) {
-      const int c = w * 32 + lane;
-      const bool valid = c < Nb;
-      const uint32_t key = valid ? __float_as_uint(ebuf(c)) : 0u;
-      bool kept;
-      if (keep_all) {
-        kept = valid;
-      } else {
-        kept = valid && key > vkey;
-        const bool tie = valid && key == vkey;
-        const uint32_t tm = __ballot_sync(0xFFFFFFFFu, tie);
-        if (tie && ties_seen + __popc(tm & ((1u << lane) - 1u)) < need_ties) kept = true;
-        ties_seen += __popc(tm);
+    __syncthreads();
+    if (a.use_sta) {
+      const int hw = a.Hb * a.Wb;
+      const int tr = r / hw, yr = (r / a.Wb) % a.Hb, xr = r % a.Wb;
+      const int nt = 2 * a.rt + 1, ny = 2 * a.rh + 1, nx = 2 * a.rw + 1;
+      for (int v = tid; v < nt * ny * nx; v += kRcThreads) {
+        const int t3 = tr - a.rt + v / (ny * nx);
+        const int yy = yr - a.rh + (v / nx) % ny;
+        const int xx = xr - a.rw + v % nx;
+        if (t3 >= 0 && t3 < a.T && yy >= 0 && yy < a.Hb && xx >= 0 && xx < a.Wb) {
+          const int c = (t3 * a.Hb + yy) * a.Wb + xx;
+          atomicOr(&bits[c >> 5], 1u << (c & 31));
+        }
       }
-      const uint32_t word = __ballot_sync(0xFFFFFFFFu, kept);
-      if (lane == 0) wbits[w] = word;
+      __syncthreads();
     }
-  }
-  __syncwarp();
-  finish_row(a, grow, r, wbits);
-}
-
-// Per-warp SMEM of the top-p selection: candidates, tile factors, the bin
-// histogram and the kept-bit row.
-__host__ __device__ inline size_t select_warp_bytes(int ntiles, int row_floats) {
-  return (static_cast<size_t>(kCand) * 8 + static_cast<size_t>(ntiles) * 8 + 16 + kBins * 8 +
-          kMaxWords * 4 + static_cast<size_t>(row_floats) * 4 + 15) & ~static_cast<size_t>(15);
-}
-
-template <bool kSmemRow>
-__global__ void __launch_bounds__(kThreads) mask_select_kernel(const MaskArgs a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int warp = threadIdx.x >> 5;
-  unsigned char *wbase = smem_raw + warp * select_warp_bytes(a.ntiles, kSmemRow ? a.Nb : 0);
-  uint32_t *cand_key = reinterpret_cast<uint32_t *>(wbase);
-  int32_t *cand_idx = reinterpret_cast<int32_t *>(cand_key + kCand);
-  float *tscale = reinterpret_cast<float *>(
-      (reinterpret_cast<uintptr_t>(cand_idx + kCand) + 15) & ~static_cast<uintptr_t>(15));
-  int *hcnt = reinterpret_cast<int *>(tscale + a.ntiles);
-  float *hmass = reinterpret_cast<float *>(hcnt + kBins);
-  uint32_t *wbits = reinterpret_cast<uint32_t *>(hmass + kBins);
-  float *erow = reinterpret_cast<float *>(wbits + kMaxWords);
-  const int64_t rows = a.BH * a.Nb;
-  for (int64_t g = static_cast<int64_t>(blockIdx.x) * kWarps + warp; g < rows;
-       g += static_cast<int64_t>(gridDim.x) * kWarps) {
-    select_row<kSmemRow>(a, g, static_cast<int>(g % a.Nb), a.slab + g * a.ld_slab,
-                         a.tmax + g * a.ntiles, erow, cand_key, cand_idx, tscale, hcnt, hmass,
-                         wbits);
+    int count = 0;
+    for (int w = tid; w < a.words; w += kRcThreads) {
+      const uint32_t x = bits[w];
+      a.bits[g * a.words + w] = x;
+      count += __popc(x);
+    }
+    count = warp_sum_i(count);
+    if (lane == 0) red[warp] = static_cast<double>(count);
+    __syncthreads();
+    if (tid == 0) {
+      double tot = 0.0;
+      for (int w = 0; w < kRcThreads / 32; ++w) tot += red[w];
+      a.counts[g] = static_cast<int32_t>(tot);
+    }
+    __syncthreads();
   }
 }
 
-// Per-warp SMEM of the static-ratio selection (all 4-byte fields).
-__host__ __device__ inline size_t topk_warp_bytes(int ntiles, int row_floats) {
-  return (static_cast<size_t>(2 * kCand + ntiles + kOctaves + kMaxWords + row_floats) * 4 + 15) &
-         ~static_cast<size_t>(15);
-}
-
-template <bool kSmemRow>
-__global__ void __launch_bounds__(kThreads) mask_select_topk_kernel(const MaskArgs a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int warp = threadIdx.x >> 5;
-  unsigned char *wbase = smem_raw + warp * topk_warp_bytes(a.ntiles, kSmemRow ? a.Nb : 0);
-  uint32_t *cand_key = reinterpret_cast<uint32_t *>(wbase);
-  int32_t *cand_idx = reinterpret_cast<int32_t *>(cand_key + kCand);
-  float *tscale = reinterpret_cast<float *>(cand_idx + kCand);
-  int *hist = reinterpret_cast<int *>(tscale + a.ntiles);
-  uint32_t *wbits = reinterpret_cast<uint32_t *>(hist + kOctaves);
-  float *erow = reinterpret_cast<float *>(wbits + kMaxWords);
-  const int64_t rows = a.BH * a.Nb;
-  for (int64_t g = static_cast<int64_t>(blockIdx.x) * kWarps + warp; g < rows;
-       g += static_cast<int64_t>(gridDim.x) * kWarps) {
-    select_row_topk<kSmemRow>(a, g, static_cast<int>(g % a.Nb), a.slab + g * a.ld_slab,
-                              a.tmax + g * a.ntiles, erow, cand_key, cand_idx, tscale, hist,
-                              wbits);
-  }
-}
-
-// Exclusive scan of n counts into row_ptr[0..n] by one CTA of 1024 threads.
 // Exclusive scan of the kept counts into row_ptr in two launches: per-chunk
 // sums of kScanChunk rows, then every chunk adds up the sums before it (at
 // most a few hundred) and scans its own rows.  Coalesced, no serial walk.
@@ -874,104 +1122,157 @@ __global__ void __launch_bounds__(256) expand_bits_kernel(const uint32_t *__rest
   }
 }
 
-struct MaskLayout {
-  int ld_slab, ntiles, words, grid;
-  size_t slab_off, tmax_off, bits_off, counts_off, total;
-  size_t smem, smem_a, smem_b, smem_k;
-};
-
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-MaskLayout mask_layout(const Geometry &g, int grid) {
+struct MaskLayout {
+  int64_t rows, plane_rows;
+  int words, np2, ld, ldk, ldp;
+  size_t qdig_off, kdig_off, qexp_off, kexp_off, kscale_off, slab_off, rec_off, bits_off,
+      counts_off, flag_off, nflag_off, sums_off, total;
+  int sel_warps;
+  size_t smem_select, smem_recheck;
+};
+
+MaskLayout mask_layout(const Geometry &g) {
   MaskLayout L;
-  L.ld_slab = static_cast<int>((g.Nb + 3) & ~3LL);
-  L.ntiles = static_cast<int>((g.Nb + kCT - 1) / kCT);
+  L.rows = g.BH * g.Nb;
+  // digit planes hold at least one whole 128-row box
+  L.plane_rows = L.rows > kTileRows ? L.rows : kTileRows;
   L.words = static_cast<int>((g.Nb + 31) / 32);
-  L.grid = grid;
+  L.np2 = 1;
+  while (L.np2 < g.Nb) L.np2 <<= 1;
+  L.ld = static_cast<int>((g.Nb + 15) & ~15LL);      // slab row: whole 16-column slices
+  L.ldk = static_cast<int>((g.Nb + 63) & ~63LL);     // per-head K scales: whole chunks
+  L.ldp = static_cast<int>((g.Nb + 31) & ~31LL);
+  const size_t plane = static_cast<size_t>(kDigits) * L.plane_rows * kRowBytes;
   size_t off = 0;
-  L.slab_off = off;
-  off = align256(off + static_cast<size_t>(g.BH * g.Nb) * L.ld_slab * 4);
-  L.tmax_off = off;
-  off = align256(off + static_cast<size_t>(g.BH * g.Nb) * L.ntiles * 8);
-  L.bits_off = off;
-  off = align256(off + static_cast<size_t>(g.BH * g.Nb) * L.words * 4);
-  L.counts_off = off;
-  off = align256(off + static_cast<size_t>(g.BH * g.Nb) * 4);
+  L.qdig_off = off; off = align256(off + plane);
+  L.kdig_off = off; off = align256(off + plane);
+  L.qexp_off = off; off = align256(off + static_cast<size_t>(L.rows) * 4);
+  L.kexp_off = off; off = align256(off + static_cast<size_t>(L.rows) * 4);
+  L.kscale_off = off; off = align256(off + static_cast<size_t>(g.BH) * L.ldk * 4);
+  L.slab_off = off; off = align256(off + static_cast<size_t>(L.rows) * L.ld * 4);
+  L.rec_off = off; off = align256(off + static_cast<size_t>(L.rows) * sizeof(RowRec));
+  L.bits_off = off; off = align256(off + static_cast<size_t>(L.rows) * L.words * 4);
+  L.counts_off = off; off = align256(off + static_cast<size_t>(L.rows) * 4);
+  L.flag_off = off; off = align256(off + static_cast<size_t>(L.rows) * 4);
+  L.nflag_off = off; off = align256(off + 16);
+  L.sums_off = off; off = align256(off + static_cast<size_t>(L.rows / 1024 + 2) * 8);
   L.total = off;
-  L.smem_a = (static_cast<size_t>(kRT) * (g.d + kPad) + 2 * static_cast<size_t>(kCT) * kLdK) * 8;
-  const int row_floats = g.Nb <= kSmemRowMaxNb ? static_cast<int>(g.Nb) : 0;
-  L.smem_b = static_cast<size_t>(kWarps) * select_warp_bytes(L.ntiles, row_floats);
-  L.smem_k = static_cast<size_t>(kWarps) * topk_warp_bytes(L.ntiles, row_floats);
-  L.smem = L.smem_a > L.smem_b ? L.smem_a : L.smem_b;
-  if (L.smem_k > L.smem) L.smem = L.smem_k;
-  if (L.words > kMaxWords) L.smem = ~static_cast<size_t>(0) >> 1;  // reported as unsupported
+  // as many rows per select CTA as 200 KiB of SMEM hold, at most kSelWarps
+  const size_t pw = select_warp_bytes(L.ldp, L.words);
+  L.sel_warps = static_cast<int>(pw <= (200u << 10) / kSelWarps ? kSelWarps : (200u << 10) / pw);
+  if (L.sel_warps < 1) L.sel_warps = 1;
+  L.smem_select = static_cast<size_t>(L.sel_warps) * pw;
+  L.smem_recheck = recheck_smem_bytes(L.ldp, L.words, g.d);
   return L;
+}
+
+// The digit planes [4][plane_rows][128 B] as a 3-D map: one box = a whole
+// row range of all four planes, 128-byte swizzled.
+bool make_map_digits(CUtensorMap *m, const void *base, int64_t plane_rows, int box_rows) {
+  EncodeFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {kRowBytes, static_cast<cuuint64_t>(plane_rows), kDigits};
+  const cuuint64_t strides[2] = {kRowBytes, static_cast<cuuint64_t>(plane_rows) * kRowBytes};
+  const cuuint32_t box[3] = {kRowBytes, static_cast<cuuint32_t>(box_rows), kDigits};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
 }
 
 }  // namespace
 
-size_t block_mask_workspace_bytes(const Geometry &g) { return mask_layout(g, kMaxGrid).total; }
+size_t block_mask_workspace_bytes(const Geometry &g) { return mask_layout(g).total; }
 
-size_t block_mask_smem_bytes(const Geometry &g) { return mask_layout(g, kMaxGrid).smem; }
+size_t block_mask_smem_bytes(const Geometry &g) {
+  if (g.Nb > kMaxNb) return ~static_cast<size_t>(0) >> 1;   // reported as unsupported
+  const MaskLayout L = mask_layout(g);
+  size_t m = static_cast<size_t>(SmemA::kAlloc);
+  if (L.smem_recheck > m) m = L.smem_recheck;
+  if (L.smem_select > m) m = L.smem_select;
+  return m;
+}
 
 cudaError_t launch_block_mask(const double *qp, const double *kp, const Geometry &g,
                               const vsa_mask_params &p, int topk, int64_t *row_ptr,
                               int32_t *col_idx, int32_t *kept_count, void *ws, unsigned *err,
                               cudaStream_t st) {
-  (void)err;
   const int64_t rows = g.BH * g.Nb;
-  if (rows == 0) {
-    return cudaMemsetAsync(row_ptr, 0, sizeof(int64_t), st);
-  }
-  const int64_t tiles_per_head = (g.Nb + kRT - 1) / kRT;
-  const int64_t items = g.BH * tiles_per_head;
-  const int64_t units = items * ((g.Nb + kCT - 1) / kCT);
-  int grid = num_sms();
-  if (grid > kMaxGrid) grid = kMaxGrid;
-  if (units < grid) grid = static_cast<int>(units);
-  MaskLayout L = mask_layout(g, grid);
+  if (rows == 0) return cudaMemsetAsync(row_ptr, 0, sizeof(int64_t), st);
+  const MaskLayout L = mask_layout(g);
   unsigned char *w = static_cast<unsigned char *>(ws);
   MaskArgs a;
-  a.qp = qp; a.kp = kp; a.BH = g.BH; a.Nb = static_cast<int>(g.Nb); a.d = g.d;
-  a.Hb = g.Hb; a.Wb = g.Wb; a.thr = p.thr; a.use_sta = p.use_sta != 0;
-  a.rt = p.sta_t; a.rh = p.sta_h; a.rw = p.sta_w;
-  a.c = 1.4426950408889634 / std::sqrt(static_cast<double>(g.d));
-  a.slab = reinterpret_cast<float *>(w + L.slab_off);
-  a.tmax = reinterpret_cast<double *>(w + L.tmax_off);
-  a.ld_slab = L.ld_slab; a.ntiles = L.ntiles;
+  a.BH = g.BH; a.rows = rows; a.Nb = static_cast<int>(g.Nb); a.d = g.d;
+  a.Hb = g.Hb; a.Wb = g.Wb; a.T = static_cast<int>(g.Nb / (static_cast<int64_t>(g.Hb) * g.Wb));
+  a.thr = p.thr; a.topk = topk;
+  a.use_sta = p.use_sta != 0; a.rt = p.sta_t; a.rh = p.sta_h; a.rw = p.sta_w;
+  a.c_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(g.d)));
+  a.scale = 1.0 / std::sqrt(static_cast<double>(g.d));
+  a.qp = qp; a.kp = kp;
+  int8_t *qdig = reinterpret_cast<int8_t *>(w + L.qdig_off);
+  int8_t *kdig = reinterpret_cast<int8_t *>(w + L.kdig_off);
+  int *qexp = reinterpret_cast<int *>(w + L.qexp_off);
+  int *kexp = reinterpret_cast<int *>(w + L.kexp_off);
+  float *kscale = reinterpret_cast<float *>(w + L.kscale_off);
+  a.qexp = qexp; a.kexp = kexp; a.kscale = kscale; a.ldk = L.ldk;
+  a.slab = reinterpret_cast<float *>(w + L.slab_off); a.ld = L.ld;
+  a.rec = reinterpret_cast<RowRec *>(w + L.rec_off);
   a.bits = reinterpret_cast<uint32_t *>(w + L.bits_off);
   a.words = L.words;
   a.counts = kept_count ? kept_count : reinterpret_cast<int32_t *>(w + L.counts_off);
-  a.items = items; a.tiles_per_head = tiles_per_head;
-  a.k = topk;
-  cudaError_t e = cudaFuncSetAttribute(mask_scores_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(L.smem_a));
-  if (e != cudaSuccess) return e;
-  mask_scores_kernel<<<grid, kThreads, L.smem_a, st>>>(a);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const int64_t sel_blocks = (rows + kWarps - 1) / kWarps;
-  const int sel_grid = static_cast<int>(sel_blocks < 64LL * num_sms() ? sel_blocks : 64LL * num_sms());
-  const bool smem_row = g.Nb <= kSmemRowMaxNb;
-  const void *sel = topk > 0 ? (smem_row ? reinterpret_cast<const void *>(mask_select_topk_kernel<true>)
-                                         : reinterpret_cast<const void *>(mask_select_topk_kernel<false>))
-                             : (smem_row ? reinterpret_cast<const void *>(mask_select_kernel<true>)
-                                         : reinterpret_cast<const void *>(mask_select_kernel<false>));
-  const size_t sel_smem = topk > 0 ? L.smem_k : L.smem_b;
-  if ((e = cudaFuncSetAttribute(sel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(sel_smem))) != cudaSuccess)
-    return e;
-  if (topk > 0) {
-    if (smem_row) mask_select_topk_kernel<true><<<sel_grid, kThreads, sel_smem, st>>>(a);
-    else mask_select_topk_kernel<false><<<sel_grid, kThreads, sel_smem, st>>>(a);
-  } else {
-    if (smem_row) mask_select_kernel<true><<<sel_grid, kThreads, sel_smem, st>>>(a);
-    else mask_select_kernel<false><<<sel_grid, kThreads, sel_smem, st>>>(a);
+  a.flagged = reinterpret_cast<int32_t *>(w + L.flag_off);
+  a.nflag = reinterpret_cast<int *>(w + L.nflag_off);
+  a.tiles_per_head = static_cast<int>((g.Nb + kTileRows - 1) / kTileRows);
+  a.nch = static_cast<int>((g.Nb + kChunk - 1) / kChunk);
+  a.np2 = L.np2;
+  a.units = g.BH * a.tiles_per_head;
+  a.err = err;
+
+  cudaError_t e;
+  {
+    const int64_t threads = 2 * rows * 32;
+    mask_digits_kernel<<<static_cast<int>((threads + 255) / 256), 256, 0, st>>>(
+        qp, kp, rows, L.plane_rows, g.d, a.Nb, L.ldk, qdig, kdig, qexp, kexp, kscale, a.nflag);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  const bool keep_all = topk > 0 ? topk >= g.Nb : p.thr <= 0.0f;
+  if (!keep_all) {
+    CUtensorMap mq, mk;
+    if (!make_map_digits(&mq, qdig, L.plane_rows, kTileRows) ||
+        !make_map_digits(&mk, kdig, L.plane_rows, kChunk))
+      return cudaErrorInvalidValue;
+    int grid = num_sms();
+    if (a.units < grid) grid = static_cast<int>(a.units);
+    if ((e = cudaFuncSetAttribute(mask_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  SmemA::kAlloc)) != cudaSuccess)
+      return e;
+    mask_scores_kernel<<<grid, kThreadsA, SmemA::kAlloc, st>>>(mq, mk, a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  {
+    const void *fn = topk > 0 ? reinterpret_cast<const void *>(mask_select_kernel<true>)
+                              : reinterpret_cast<const void *>(mask_select_kernel<false>);
+    if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(L.smem_select))) != cudaSuccess)
+      return e;
+    const int64_t want = (rows + L.sel_warps - 1) / L.sel_warps;
+    const int sg = static_cast<int>(want < 16LL * num_sms() ? want : 16LL * num_sms());
+    const int threads = L.sel_warps * 32;
+    if (topk > 0) mask_select_kernel<true><<<sg, threads, L.smem_select, st>>>(a, L.ldp);
+    else mask_select_kernel<false><<<sg, threads, L.smem_select, st>>>(a, L.ldp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if ((e = cudaFuncSetAttribute(mask_recheck_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(L.smem_recheck))) != cudaSuccess)
+    return e;
+  // a CTA per listed row, as many as fit on the GPU at once
+  mask_recheck_kernel<<<2 * num_sms(), kRcThreads, L.smem_recheck, st>>>(a, L.ldp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   {
-    // chunk sums go to the start of the slab: the selection is done with it
-    int64_t *sums = reinterpret_cast<int64_t *>(a.slab);
+    int64_t *sums = reinterpret_cast<int64_t *>(w + L.sums_off);
     const int chunks = static_cast<int>((rows + kScanChunk - 1) / kScanChunk);
     chunk_sums_kernel<<<chunks, kScanChunk, 0, st>>>(a.counts, rows, sums);
     chunk_scan_kernel<<<chunks, kScanChunk, 0, st>>>(a.counts, rows, sums, row_ptr);

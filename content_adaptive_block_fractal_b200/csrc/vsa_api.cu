@@ -447,8 +447,21 @@ vsa_status vsa_device_status(void *stream) {
   if ((e = cudaMemcpy(err, &zero, sizeof zero, cudaMemcpyHostToDevice)) != cudaSuccess)
     return cuda_fail(e, "clear device error word");
   return fail(VSA_ERR_DEVICE_TIMEOUT,
-              "device error word 0x%x (1: TMA wait, 2: MMA wait, 4: softmax wait, 8: bad block index, 16: shared memory misaligned)",
+              "device error word 0x%x (1: TMA wait, 2: MMA wait, 4: softmax wait, 8: bad block index, 16: shared memory misaligned, 32: wait probe)",
               v);
+}
+
+vsa_status vsa_wait_probe(int64_t wait_cycles, void *stream) {
+  if (wait_cycles < 1 || wait_cycles > (1LL << 32))
+    return fail(VSA_ERR_INVALID_ARG, "wait_cycles %lld outside [1, 2^32]",
+                static_cast<long long>(wait_cycles));
+  cudaError_t e;
+  unsigned *err = device_error_word(&e);
+  if (!err) return cuda_fail(e, "device error word");
+  if ((e = vsa::launch_wait_probe(wait_cycles, err, static_cast<cudaStream_t>(stream))) !=
+      cudaSuccess)
+    return cuda_fail(e, "wait probe launch");
+  return VSA_OK;
 }
 
 }  // extern "C"

@@ -20,6 +20,7 @@ enum : unsigned {
   kErrWaitSoftmax = 1u << 2, // softmax/epilogue hand-off never arrived
   kErrBadIndex = 1u << 3,    // a block index outside [0, Nb) was skipped
   kErrSmemAlign = 1u << 4,   // dynamic shared memory not 1 KiB aligned
+  kErrWaitProbe = 1u << 5,   // the wait probe gave up (diagnostic entry point)
 };
 
 // ~2 s at 1.9 GHz: far above any legitimate wait inside one kernel.
@@ -71,18 +72,22 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // Waits for the phase with the given parity to complete.  Gives up after
-// kWaitCycles, records `code` in *err and returns false.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned *err,
-                                          unsigned code) {
+// `limit` cycles, records `code` in *err and returns false.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, long long limit,
+                                              unsigned *err, unsigned code) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       atomicOr(err, code);
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned *err,
+                                          unsigned code) {
+  return mbar_wait_for(bar, parity, kWaitCycles, err, code);
 }
 
 // ---------------------------------------------------------------- fences

@@ -68,4 +68,8 @@ cudaError_t launch_cluster_attn(const void *q, const void *k, const void *v, con
                                 const vsa_cluster_state *out_state, void *ws, unsigned *err,
                                 cudaStream_t st, const char **why);
 
+// Diagnostic: one thread waits, with the given cycle limit, on an mbarrier
+// that nothing arrives at; the wait gives up and records kErrWaitProbe.
+cudaError_t launch_wait_probe(int64_t wait_cycles, unsigned *err, cudaStream_t st);
+
 }  // namespace vsa

@@ -294,6 +294,16 @@ const char *vsa_last_error(void);
  * bounded wait since the last call, or VSA_ERR_CUDA if the stream failed. */
 vsa_status vsa_device_status(void *stream);
 
+/* Diagnostic of the failure-detection path (no counterpart on the pages): one
+ * device thread waits, with a limit of `wait_cycles` SM clock cycles, on an
+ * mbarrier that nothing arrives at.  The wait gives up, records code 32 in the
+ * device error word and the kernel returns, exactly as a library kernel whose
+ * expected arrival never comes does.  The next vsa_device_status() on the
+ * stream then returns VSA_ERR_DEVICE_TIMEOUT (and clears the word); later
+ * calls are unaffected.  wait_cycles in [1, 2^32] (VSA_ERR_INVALID_ARG
+ * otherwise); about 2^21 cycles is a millisecond. */
+vsa_status vsa_wait_probe(int64_t wait_cycles, void *stream);
+
 /* Library version, "major.minor.patch". */
 const char *vsa_version(void);
 

@@ -360,6 +360,28 @@ def sparse_attention(qf, kf, vf, row_ptr, col_idx, scale=None, qblocks=None):
     return o, lse
 
 
+def boundary_rows(diag: np.ndarray, thr: float, eps: float = 1e-5) -> np.ndarray:
+    """Rows whose boundary block's cumulative mass lies within eps of 1 - thr:
+    the kept prefix mass, or that mass without its last block.  These are the
+    only rows on which a kept set computed from probabilities accurate to a
+    few 1e-7 may legitimately differ from the exact one; every other row,
+    near ties across the cut included, has one kept set.  thr = 0 keeps every
+    block: never a boundary row."""
+    if thr <= 0.0:
+        return np.zeros(diag.shape[0], dtype=bool)
+    tgt = 1.0 - thr
+    return (np.abs(diag[:, 0] - tgt) <= eps) | (np.abs(tgt - diag[:, 1]) <= eps)
+
+
+def near_tie_rows(diag: np.ndarray, thr: float, eps: float = 1e-5) -> np.ndarray:
+    """Rows whose last kept and first dropped blocks have probabilities within
+    a relative eps of each other (a near tie across the cut)."""
+    if thr <= 0.0:
+        return np.zeros(diag.shape[0], dtype=bool)
+    dropped = diag[:, 3] >= 0
+    return dropped & (diag[:, 2] - diag[:, 3] <= eps * diag[:, 2])
+
+
 def ambiguous_rows(diag: np.ndarray, thr: float, eps: float = 1e-5) -> np.ndarray:
     """Rows whose CDF cut is numerically ambiguous.
 

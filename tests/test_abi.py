@@ -164,3 +164,10 @@ def test_raster_entry_points_accept_an_empty_shape():
     assert L.vsa_pool_qk_raster(None, None, None, None, s, None) == 0
     assert L.vsa_sparse_attn_fwd_raster(None, None, None, None, None, s, 0.0, None, None, None,
                                         0, None) == 0
+
+
+def test_wait_probe_limit_validated_on_the_host():
+    L = _lib.load()
+    assert L.vsa_wait_probe(0, None) == 1
+    assert L.vsa_wait_probe((1 << 32) + 1, None) == 1
+    assert b"wait_cycles" in L.vsa_last_error()

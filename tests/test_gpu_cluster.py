@@ -105,3 +105,32 @@ def test_cluster_attention_p1_is_dense():
     ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt)
     err = (o[0, 0].double().cpu() - ref).abs()
     assert err.max().item() <= O_MAX and err.mean().item() <= O_MEAN
+
+
+@pytest.mark.parametrize("name,C", [("tiny", 16), ("wan1.3b-480p", 128)])
+def test_centroid_update_matches_oracle_on_gpu_labels(name, C):
+    """The GPU's centroid update element by element: with the same initial
+    centroids, a run without iterations returns the first assignment, and a
+    run with one iteration returns the centroids updated from exactly that
+    assignment; the oracle's update of the same labels must give the same
+    fp32 centroids (fp64 member means of bf16 values, rounded once)."""
+    wl, q, k, v = data(name, 1)
+    shape = vsa.Shape(wl.B, 1, wl.T, wl.H, wl.W, wl.d)
+    qd, kd, vd = (x.cuda() for x in (q, k, v))
+    qu, ku = (oracle.as_u16(x)[0, 0] for x in (q, k))
+    init = [oracle.kmeans_init(xu, C) for xu in (qu, ku)]
+    init_d = tuple(torch.from_numpy(c[None, None].copy()).cuda() for c in init)
+    _, _, st0 = vsa.cluster_attention(qd, kd, vd, shape, vsa.ClusterParams(C, C, 0, 0.9),
+                                      init=init_d, want_state=True)
+    _, _, st1 = vsa.cluster_attention(qd, kd, vd, shape, vsa.ClusterParams(C, C, 1, 0.9),
+                                      init=init_d, want_state=True)
+    vsa.device_status()
+    for side, xu, c0 in (("q", qu, init[0]), ("k", ku, init[1])):
+        lab0 = st0[f"{side}_labels"][0, 0].cpu().numpy()
+        np.testing.assert_array_equal(st0[f"{side}_centroids"][0, 0].cpu().numpy(), c0)
+        want, count = oracle.kmeans_update(xu, lab0, c0)
+        got = st1[f"{side}_centroids"][0, 0].cpu().numpy()
+        ulp = np.spacing(np.abs(want).astype(np.float32))
+        assert (np.abs(got - want) <= ulp).all(), f"{side}: max diff {np.abs(got - want).max()}"
+        exact = float((got == want).mean())
+        print(f"\n{name} {side} C={C}: {exact:.5f} of centroid entries bit-identical")

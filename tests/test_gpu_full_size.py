@@ -4,8 +4,8 @@ block mask, sparse attention, unflatten of O, all heads in one launch each).
 
 The oracle cannot run a whole 40-head or 24-head layer in a test, so it checks
 sampled outputs one by one: a few heads in full for flatten and pool (bit
-exact), sampled mask rows (bit exact except rows the classifier reports as
-within rounding of the cut), and sampled query blocks of attention (O and LSE
+exact), sampled mask rows (bit exact except rows whose boundary mass lies
+within 1e-5 of 1 - thr, which are reported), and sampled query blocks of attention (O and LSE
 within tolerance, on the GPU's own CSR).  Properties that hold at any size are
 checked over the whole output: CSR structure, non-empty rows, STA window
 coverage, finite O and LSE, and the unflatten permutation on sampled tokens.
@@ -109,7 +109,7 @@ def test_full_size_sampled(name):
     ci_g = csr.col_idx[:nnz].cpu().numpy()
     cnt_g = csr.kept_count.cpu().numpy()
     thr = thr32(wl.thr)
-    n_amb = n_bad_amb = 0
+    n_amb = n_bad_amb = n_tie = 0
     for h in heads:
         # flatten and pool of this head: bit exact
         qf_o, kf_o, vf_o = (oracle.flatten(x[:, h:h + 1], wl.T, wl.H, wl.W) for x in (q, k, v))
@@ -124,7 +124,8 @@ def test_full_size_sampled(name):
         rows = sample_rows(wl, cnt_g[base:base + Nb], rng)
         keep, diag = oracle.block_mask(qp_o, kp_o, wl.Hb, wl.Wb, thr, wl.use_sta, wl.sta,
                                        rows=rows)
-        amb = oracle.ambiguous_rows(diag, thr, AMBIG_EPS)
+        amb = oracle.boundary_rows(diag, thr, AMBIG_EPS)
+        n_tie += int((oracle.near_tie_rows(diag, thr, AMBIG_EPS) & ~amb).sum())
         for i, r in enumerate(rows):
             g = base + r
             got = ci_g[rp_g[g]:rp_g[g + 1]]
@@ -154,5 +155,5 @@ def test_full_size_sampled(name):
         assert torch.equal(o_raster[0, h, torch.as_tensor(order[tok]).cuda()],
                            layer.o[0, h, torch.as_tensor(tok).cuda()])
     print(f"{name}: nnz {nnz} ({nnz / (wl.heads * Nb * Nb):.4f} kept), "
-          f"{n_amb} sampled rows near the cut, {n_bad_amb} of them differ")
-    assert n_bad_amb <= n_amb
+          f"{n_amb} sampled rows with the boundary mass within {AMBIG_EPS} of 1 - thr, "
+          f"{n_bad_amb} of them differ; {n_tie} near-tie rows matched")

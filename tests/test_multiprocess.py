@@ -1,7 +1,9 @@
 """The N > 1 host logic of bench.py on CPU: world-size-2 gloo ranks reduce
-their device times with a max (the slowest rank sets the job's time), the
-job's per-layer time is that max over the rank count, and the reference
-arm's non-zero ranks leave without work."""
+their device times with a max (the slowest rank sets the job's time); with
+replicas the job's per-layer time is that max over the rank count, with head
+sharding it is the max itself, the ranks' head slices partition the layer and
+their kept-tile counts add up; the reference arm's non-zero ranks leave
+without work."""
 import importlib.util
 import os
 import socket
@@ -36,8 +38,14 @@ def _rank(rank, world, port, out):
     try:
         b = _bench()
         ms, e2e = b.reduce_over_ranks([1.0 + rank, 10.0 * (rank + 1)], "cpu")
+        # head sharding: each rank's slice of a 40-head layer, gathered
+        h0, h1 = b.head_slice(40, rank, world)
+        slices = [None] * world
+        dist.all_gather_object(slices, (h0, h1))
+        kept = b.sum_over_ranks([100.0 * (h1 - h0)], "cpu")[0]
         dist.barrier()
-        out[rank] = (ms, e2e, b.job_ms_per_layer(ms, world))
+        out[rank] = (ms, e2e, b.job_ms_per_layer(ms, world),
+                     b.job_ms_per_layer(ms, world, "heads"), slices, kept)
     finally:
         dist.destroy_process_group()
 
@@ -49,9 +57,13 @@ def test_timings_reduce_to_the_slowest_rank():
         mp.spawn(_rank, args=(world, _free_port(), out), nprocs=world, join=True)
         res = dict(out)
     for rank in range(world):
-        ms, e2e, per_layer = res[rank]
+        ms, e2e, per_layer, per_layer_heads, slices, kept = res[rank]
         assert ms == 2.0 and e2e == 20.0
         assert per_layer == 1.0
+        assert per_layer_heads == 2.0          # one layer, done when the slowest rank is
+        # the ranks' head slices cover the layer once, in order
+        assert [tuple(x) for x in slices] == [(0, 20), (20, 40)]
+        assert kept == 100.0 * 40               # the layer's work, summed over the slices
 
 
 def test_reference_arm_other_ranks_exit_without_work():

@@ -476,6 +476,28 @@ def test_centroid_topp_size_weighting():
     np.testing.assert_array_equal(keep[0], [1, 1, 1])
 
 
+def test_centroid_topp_scale_is_inverse_sqrt_d():
+    """Two equal-size key clusters with opposite centroids: the estimated
+    attention of the first is the logistic function of the score difference
+    2a/sqrt(d) (a = ln 3, d = 4 gives exactly 3/4 in exact arithmetic).  A
+    dropped or doubled scale would give logistic(2a) = 0.9, a factor sqrt(d)
+    in place of 1/sqrt(d) gives 81/82."""
+    d = 4
+    a = np.float32(np.log(3.0))
+    cq = np.zeros((1, d), dtype=np.float32)
+    cq[0, 0] = a
+    ck = np.zeros((2, d), dtype=np.float32)
+    ck[0, 0], ck[1, 0] = 1.0, -1.0
+    nk = np.array([7, 7], dtype=np.int32)
+    p0 = 1.0 / (1.0 + np.exp(-2.0 * float(a) / np.sqrt(d)))       # ~0.75
+    keep, diag = oracle.centroid_topp(cq, ck, nk, 0.74)
+    np.testing.assert_array_equal(keep[0], [1, 0])
+    np.testing.assert_allclose(diag[0, 2], p0, rtol=1e-14)         # last kept probability
+    np.testing.assert_allclose(diag[0, 3], 1.0 - p0, rtol=1e-14)   # first dropped
+    keep, _ = oracle.centroid_topp(cq, ck, nk, 0.76)               # 0.75 < 0.76: both
+    np.testing.assert_array_equal(keep[0], [1, 1])
+
+
 def test_cluster_attention_against_masked_sdpa_and_permutation():
     """Token-level attention over kept clusters equals torch SDPA with the
     boolean mask built from the labels; all clusters kept is dense attention;
