@@ -833,79 +833,88 @@ __global__ void __launch_bounds__(kSelWarps * 32) mask_select_kernel(const MaskA
 // The oracle's arithmetic for one listed row, a CTA per row: fp64 scores
 // scaled by 1/sqrt(d), softmax against the row maximum, and the kept set of
 // the sort on (probability desc, index asc) -- blocks taken while the mass
-// before them is below 1 - thr (top-p), or the first k (static ratio).  The
-// scores come from 64-key tiles of K staged in SMEM (coalesced loads; the next
-// tile is fetched into registers while the current one is used).  The cut
-// value is found by bisection on the bit patterns of the probabilities
-// (positive doubles order like their patterns) with fp64 mass (count) sums;
-// equal probabilities at the cut go to the lower indices.  Then the STA
-// union, the kept-bit row and its count.
+// before them is below 1 - thr (top-p), or the first k (static ratio).
+// Scores: the head's K passes through a ring of three 32-key stages filled by
+// bulk copies (32 consecutive key rows are contiguous), 16 threads per key
+// reading consecutive doubles.  The cut: bisection over the probabilities'
+// bit patterns (positive doubles order like their patterns) with fp64 mass
+// (count) sums until at most 256 values remain between the bounds; those are
+// sorted on (probability desc, index asc) and walked in order from the mass
+// above them, as the oracle walks its sorted row.  Then the STA union, the
+// kept-bit row and its count.
 constexpr int kRcThreads = 256;
-constexpr int kRcTile = 64;       // keys per staged tile
+constexpr int kRcKeys = 32;       // keys per stage
+constexpr int kRcStages = 3;
+constexpr int kRcList = 256;      // values sorted at the end of the bisection
 
 __host__ __device__ inline size_t recheck_smem_bytes(int ldp, int words, int d) {
-  return static_cast<size_t>(kRcTile) * (d + 4) * 8 + static_cast<size_t>(ldp) * 8 +
-         static_cast<size_t>(d) * 8 + ((static_cast<size_t>(words) * 4 + 15) & ~static_cast<size_t>(15));
+  return static_cast<size_t>(kRcStages) * kRcKeys * d * 8 + static_cast<size_t>(ldp) * 8 +
+         static_cast<size_t>(d) * 8 + static_cast<size_t>(kRcList) * 12 +
+         ((static_cast<size_t>(words) * 4 + 15) & ~static_cast<size_t>(15)) + 64;
 }
 
 __global__ void __launch_bounds__(kRcThreads) mask_recheck_kernel(const MaskArgs a, int ldp) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int d = a.d, Nb = a.Nb;
-  // padded tile rows: the 16 threads of a half-warp (4 keys x 4 quarters)
-  // read 16 distinct 8-byte banks
-  const int ldt = d + 4;
-  double *tile = reinterpret_cast<double *>(smem_raw);    // [kRcTile][d + 4]
-  double *pv = tile + kRcTile * ldt;                      // [ldp] scores, then probabilities
-  double *q = pv + ldp;                                   // [d]
-  uint32_t *bits = reinterpret_cast<uint32_t *>(q + d);   // [words]
-  __shared__ double red[kRcThreads / 32];
+  double *stage = reinterpret_cast<double *>(smem_raw);   // [3][32][d]
+  double *pv = stage + kRcStages * kRcKeys * d;            // [ldp] scores, then probabilities
+  double *q = pv + ldp;                                    // [d]
+  double *lp = q + d;                                      // [256] listed values
+  int *li = reinterpret_cast<int *>(lp + kRcList);         // [256] their indices
+  uint32_t *bits = reinterpret_cast<uint32_t *>(li + kRcList);                 // [words]
+  uint64_t *bar = reinterpret_cast<uint64_t *>(
+      (reinterpret_cast<uintptr_t>(bits + a.words) + 15) & ~static_cast<uintptr_t>(15));  // [3]
+  __shared__ double red[kRcThreads / 32], red2[kRcThreads / 32];
+  __shared__ int nlist, ok_sh;
+  const uint32_t stage_s = smem_u32(stage);
+  auto bar_s = [&](int s) { return smem_u32(bar + s); };
+  if (tid == 0) {
+    for (int s = 0; s < kRcStages; ++s) mbar_init(bar_s(s), 1);
+    fence_mbar_init();
+    ok_sh = 1;
+  }
+  __syncthreads();
   const int nf = *a.nflag;
-  // each thread moves 16-byte pieces: kRcTile * d / 2 pieces per tile,
-  // d / 2 = 2^hs pieces per key row
-  const int hs = d == 128 ? 6 : 5;
-  const int per_thread = (kRcTile << hs) / kRcThreads;    // 16 (d = 128) or 8 (d = 64)
+  const int ntiles = (Nb + kRcKeys - 1) / kRcKeys;
+  const uint32_t stage_bytes = static_cast<uint32_t>(kRcKeys * d * 8);
+  int n = 0;                     // stages consumed by this CTA so far (barrier phases)
   for (int64_t fi = blockIdx.x; fi < nf; fi += gridDim.x) {
     const int64_t g = a.flagged[fi];
     const int64_t bh = g / Nb;
     const int r = static_cast<int>(g % Nb);
     const double *kbase = a.kp + bh * Nb * d;
     for (int j = tid; j < d; j += kRcThreads) q[j] = a.qp[g * d + j];
-    double2 pre[16];
-    auto fetch = [&](int c0) {
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        if (u < per_thread) {
-          const int piece = tid + u * kRcThreads;
-          const int row = piece >> hs, col = piece & ((1 << hs) - 1);
-          pre[u] = c0 + row < Nb ? reinterpret_cast<const double2 *>(kbase + (c0 + row) * d)[col]
-                                 : make_double2(0.0, 0.0);
-        }
-      }
+    auto issue = [&](int t) {    // tile t into stage (n + t - done) % 3, by thread 0
+      const int s = (n + t) % kRcStages;
+      const int keys = Nb - t * kRcKeys < kRcKeys ? Nb - t * kRcKeys : kRcKeys;
+      const uint32_t bytes = static_cast<uint32_t>(keys * d * 8);
+      mbar_arrive_expect_tx(bar_s(s), bytes);
+      bulk_load(stage_s + s * stage_bytes, kbase + static_cast<int64_t>(t) * kRcKeys * d, bytes,
+                bar_s(s));
     };
-    fetch(0);
-    for (int c0 = 0; c0 < Nb; c0 += kRcTile) {
-      __syncthreads();                 // the previous tile has been used
+    if (tid == 0)
+      for (int t = 0; t < kRcStages && t < ntiles; ++t) issue(t);
+    __syncthreads();
+    const int key = tid >> 4, part = tid & 15;        // 16 threads per key
+    for (int t = 0; t < ntiles; ++t) {
+      const int s = (n + t) % kRcStages;
+      if (!mbar_wait(bar_s(s), ((n + t) / kRcStages) & 1, a.err, kErrWaitTma)) ok_sh = 0;
+      const double *ks = stage + s * kRcKeys * d;
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        if (u < per_thread) {
-          const int piece = tid + u * kRcThreads;
-          const int row = piece >> hs, col = piece & ((1 << hs) - 1);
-          tile[row * ldt + 2 * col] = pre[u].x;
-          tile[row * ldt + 2 * col + 1] = pre[u].y;
-        }
+      for (int h = 0; h < kRcKeys; h += 16) {
+        const int kk = h + key;
+        double acc = 0.0;
+        for (int j = part; j < d; j += 16) acc = fma(q[j], ks[kk * d + j], acc);
+#pragma unroll
+        for (int o = 8; o; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+        const int c = t * kRcKeys + kk;
+        if (part == 0 && c < Nb) pv[c] = acc * a.scale;
       }
-      __syncthreads();
-      if (c0 + kRcTile < Nb) fetch(c0 + kRcTile);
-      // 4 threads per key, a quarter of d each, then a 4-lane reduction
-      const int key = tid >> 2, part = tid & 3;
-      double s = 0.0;
-      const double *kr = tile + key * ldt;
-      for (int j = part; j < d; j += 4) s = fma(q[j], kr[j], s);
-      s += __shfl_xor_sync(0xFFFFFFFFu, s, 1);
-      s += __shfl_xor_sync(0xFFFFFFFFu, s, 2);
-      if (part == 0 && c0 + key < Nb) pv[c0 + key] = s * a.scale;
+      __syncthreads();            // stage s consumed by every thread
+      if (tid == 0 && t + kRcStages < ntiles) issue(t + kRcStages);
     }
+    n += ntiles;
     __syncthreads();
     // softmax against the row maximum (block reductions)
     double m = -INFINITY;
@@ -930,67 +939,135 @@ __global__ void __launch_bounds__(kRcThreads) mask_recheck_kernel(const MaskArgs
     for (int c = tid; c < Nb; c += kRcThreads) pv[c] /= z;
     for (int w = tid; w < a.words; w += kRcThreads) bits[w] = 0u;
     __syncthreads();
-    // the cut value: bisection over the probabilities' bit patterns with
-    // CTA-wide mass (count) sums
-    auto mass_at_least = [&](uint64_t key) {
-      double sum = 0.0;
+    const bool count_rule = a.topk > 0;
+    // mass (count) of the values with patterns in [lo, hi), and how many
+    auto mass_in = [&](uint64_t lo, uint64_t hi, double &cnt) {
+      double sum = 0.0, k = 0.0;
       for (int c = tid; c < Nb; c += kRcThreads) {
         const uint64_t kc = static_cast<uint64_t>(__double_as_longlong(pv[c]));
-        if (kc >= key) sum += a.topk > 0 ? 1.0 : pv[c];
+        if (kc >= lo && kc < hi) {
+          sum += count_rule ? 1.0 : pv[c];
+          k += 1.0;
+        }
       }
       sum = warp_sum(sum);
-      __syncthreads();                   // red[] is free
-      if (lane == 0) red[warp] = sum;
+      k = warp_sum(k);
+      __syncthreads();
+      if (lane == 0) {
+        red[warp] = sum;
+        red2[warp] = k;
+      }
       __syncthreads();
       double tot = 0.0;
-      for (int w = 0; w < kRcThreads / 32; ++w) tot += red[w];
+      cnt = 0.0;
+      for (int w = 0; w < kRcThreads / 32; ++w) {
+        tot += red[w];
+        cnt += red2[w];
+      }
       return tot;
     };
-    const double target = a.topk > 0 ? static_cast<double>(a.topk) : 1.0 - static_cast<double>(a.thr);
-    bool keep_all = a.topk > 0 ? a.topk >= Nb : !(a.thr > 0.0f);
-    uint64_t vkey = 0;
-    int need_ties = 0;
+    const double target = count_rule ? static_cast<double>(a.topk) : 1.0 - static_cast<double>(a.thr);
+    const uint64_t kInf = 0x7FF0000000000000ull;     // nothing is >= this pattern
+    bool keep_all = count_rule ? a.topk >= Nb : !(a.thr > 0.0f);
+    int kept_listed = 0;
+    uint64_t lo = 0, hi = kInf;
+    double above = 0.0;           // mass (count) of the values >= hi
     if (!keep_all) {
-      if (!(mass_at_least(0) >= target)) {
-        keep_all = true;                   // the sums never reach 1 - thr
+      double cnt;
+      if (!(mass_in(0, kInf, cnt) >= target)) {
+        keep_all = true;                 // the sums never reach 1 - thr
       } else {
-        // invariant: mass(p >= lo) >= target > mass(p >= hi)
-        uint64_t lo = 0, hi = 0x7FF0000000000000ull;   // +inf: nothing is >= hi
-        while (hi - lo > 1) {
+        // invariant: above < target <= above + mass[lo, hi); stops at one
+        // pattern (equal values) at the latest
+        while (cnt > kRcList && hi - lo > 1) {
           const uint64_t mid = lo + ((hi - lo) >> 1);
-          if (mass_at_least(mid) >= target) lo = mid; else hi = mid;
+          double cu;
+          const double up = mass_in(mid, hi, cu);
+          if (above + up >= target) {
+            lo = mid;
+            cnt = cu;
+          } else {
+            above += up;
+            hi = mid;
+            cnt -= cu;
+          }
         }
-        vkey = lo;                         // the cut value's pattern
-        const double base = mass_at_least(vkey + 1);   // strictly above the cut
-        const double v = a.topk > 0 ? 1.0 : __longlong_as_double(static_cast<long long>(vkey));
-        int j = static_cast<int>(fmin(ceil((target - base) / v), static_cast<double>(Nb)));
-        if (j < 1) j = 1;
-        while (j > 1 && base + (j - 1) * v >= target) --j;
-        while (base + j * v < target && j < Nb) ++j;
-        need_ties = j;
-      }
-    }
-    // kept bits, ties in index order (warp 0 walks the words in order)
-    if (warp == 0) {
-      int ties_seen = 0;
-      for (int w = 0; w < a.words; ++w) {
-        const int c = w * 32 + lane;
-        const bool valid = c < Nb;
-        bool kept;
-        if (keep_all) {
-          kept = valid;
+        if (cnt > kRcList) {
+          // more than the list holds, all equal to the pattern lo: the
+          // first `need` of them in index order are kept
+          const double v = count_rule ? 1.0 : __longlong_as_double(static_cast<long long>(lo));
+          int j = static_cast<int>(fmin(ceil((target - above) / v), static_cast<double>(Nb)));
+          if (j < 1) j = 1;
+          while (j > 1 && above + (j - 1) * v >= target) --j;
+          while (above + j * v < target && j < Nb) ++j;
+          if (warp == 0) {
+            int ties_seen = 0;
+            for (int w = 0; w < a.words; ++w) {
+              const int c = w * 32 + lane;
+              const uint64_t kc = c < Nb ? static_cast<uint64_t>(__double_as_longlong(pv[c])) : 0ull;
+              const bool tie = c < Nb && kc == lo;
+              const uint32_t tm = __ballot_sync(0xFFFFFFFFu, tie);
+              const bool kept = tie && ties_seen + __popc(tm & ((1u << lane) - 1u)) < j;
+              const uint32_t word = __ballot_sync(0xFFFFFFFFu, kept);
+              if (lane == 0) bits[w] |= word;
+              ties_seen += __popc(tm);
+            }
+          }
+          __syncthreads();
         } else {
-          const uint64_t kc = valid ? static_cast<uint64_t>(__double_as_longlong(pv[c])) : 0ull;
-          kept = valid && kc > vkey;
-          const bool tie = valid && kc == vkey;
-          const uint32_t tm = __ballot_sync(0xFFFFFFFFu, tie);
-          if (tie && ties_seen + __popc(tm & ((1u << lane) - 1u)) < need_ties) kept = true;
-          ties_seen += __popc(tm);
+        // the values in [lo, hi): list, sort on (value desc, index asc), walk
+        if (tid == 0) nlist = 0;
+        __syncthreads();
+        for (int c = tid; c < Nb; c += kRcThreads) {
+          const uint64_t kc = static_cast<uint64_t>(__double_as_longlong(pv[c]));
+          if (kc >= lo && kc < hi) {
+            const int pos = atomicAdd(&nlist, 1);
+            lp[pos] = pv[c];
+            li[pos] = c;
+          }
         }
-        const uint32_t word = __ballot_sync(0xFFFFFFFFu, kept);
-        if (lane == 0) bits[w] = word;
+        __syncthreads();
+        const int nl = nlist;
+        for (int v = nl + tid; v < kRcList; v += kRcThreads) {
+          lp[v] = -1.0;
+          li[v] = INT_MAX;
+        }
+        __syncthreads();
+        for (int size = 2; size <= kRcList; size <<= 1)
+          for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            const int x = tid, y = x ^ stride;
+            if (y > x) {
+              const bool up = (x & size) == 0;
+              const bool first = lp[x] > lp[y] || (lp[x] == lp[y] && li[x] < li[y]);
+              if (first != up) {
+                const double tp = lp[x]; lp[x] = lp[y]; lp[y] = tp;
+                const int ti = li[x]; li[x] = li[y]; li[y] = ti;
+              }
+            }
+            __syncthreads();
+          }
+        if (tid == 0) {
+          // kept while the mass before the value is below the target
+          double mass = above;
+          int k = 0;
+          while (k < nl && mass < target) {
+            mass += count_rule ? 1.0 : lp[k];
+            ++k;
+          }
+          nlist = k;
+        }
+        __syncthreads();
+        kept_listed = nlist;
+        }
       }
     }
+    // kept bits: every value >= hi, and the first kept_listed of the list
+    for (int c = tid; c < Nb; c += kRcThreads) {
+      const uint64_t kc = static_cast<uint64_t>(__double_as_longlong(pv[c]));
+      if (keep_all || kc >= hi) atomicOr(&bits[c >> 5], 1u << (c & 31));
+    }
+    for (int v = tid; v < kept_listed; v += kRcThreads)
+      atomicOr(&bits[li[v] >> 5], 1u << (li[v] & 31));
     __syncthreads();
     if (a.use_sta) {
       const int hw = a.Hb * a.Wb;
@@ -1022,6 +1099,7 @@ __global__ void __launch_bounds__(kRcThreads) mask_recheck_kernel(const MaskArgs
       a.counts[g] = static_cast<int32_t>(tot);
     }
     __syncthreads();
+    if (!ok_sh) break;           // a stage never arrived: stop (recorded)
   }
 }
 

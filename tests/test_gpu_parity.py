@@ -150,10 +150,12 @@ def test_block_mask_matches_oracle(name, thr, sta):
     vsa.device_status()
 
 
-def test_block_mask_sta_radii_and_exact_ties():
+@pytest.mark.parametrize("T,H,W", [(2, 16, 32), (2, 96, 96)], ids=["Nb16", "Nb288"])
+def test_block_mask_sta_radii_and_exact_ties(T, H, W):
     # constant Q and K: every pooled score is equal, every probability is
     # exactly 1/Nb; the CDF keeps the lowest ceil((1 - thr) * Nb) indices
-    wl = small_shape(T=2, H=16, W=32, d=64)
+    # (Nb = 288 puts more equal values at the cut than the recheck sorts)
+    wl = small_shape(T=T, H=H, W=W, d=64)
     Nb = wl.Nb
     qp = np.full((1, 2, Nb, 64), 0.25)
     kp = np.full((1, 2, Nb, 64), -0.5)
