@@ -164,6 +164,19 @@ __device__ __forceinline__ void load_block(uint32_t dst, const CUtensorMap *m, u
   }
 }
 
+// L2 prefetch of block r of head slice bh (the same box load_block fetches).
+template <bool kRaster>
+__device__ __forceinline__ void prefetch_block(const CUtensorMap *m, const AttnArgs &a, int bh,
+                                               int r) {
+  if constexpr (kRaster) {
+    int t, py, px;
+    block_patch(r, a, t, py, px);
+    tma_prefetch_5d(m, 0, px * 8, 0, py * 8, bh * a.T + t);
+  } else {
+    tma_prefetch_4d(m, 0, 0, 0, static_cast<int>(static_cast<int64_t>(bh) * a.N / 8) + r * 8);
+  }
+}
+
 // Token index within its head of position i (= 8 * patch row + column) of
 // block r.
 template <bool kRaster>
@@ -331,11 +344,53 @@ __global__ void __maxnreg__(168)
       ++m;
       return true;
     };
+    // The next item's header is fetched one dependent load per emitted step
+    // (work counter -> plan entry -> row pointers -> first list windows, and
+    // an L2 prefetch of its Q blocks), so item starts do not stall the
+    // producer on a chain of global round trips.  hs: 0 nothing fetched,
+    // 1 counter value pending, 2 plan entry pending, 3 row pointers pending,
+    // 4 ready, 5 no more work.
+    int hs = 0;
+    int h_raw = 0, h_item = 0, h_bh = 0, h_r0 = 0, h_r1 = -1;
+    int64_t h_rp0 = 0, h_rp1 = 0, h_rp2 = 0, h_rp3 = 0;
+    int h_pre0 = 0, h_pre1 = 0;      // this lane's entry of each list's first window
+    auto advance = [&]() {
+      if (hs == 0) {
+        if (lane == 0) h_raw = atomicAdd(a.counter, 1);
+        hs = 1;
+      } else if (hs == 1) {
+        h_raw = __shfl_sync(0xFFFFFFFFu, h_raw, 0);
+        if (h_raw >= n_items) {
+          hs = 5;
+        } else {
+          h_item = a.order[h_raw];
+          hs = 2;
+        }
+      } else if (hs == 2) {
+        decode_item(h_item, a, h_bh, h_r0, h_r1);
+        const int64_t g0 = static_cast<int64_t>(h_bh) * a.Nb + h_r0;
+        h_rp0 = a.row_ptr[g0];
+        h_rp1 = a.row_ptr[g0 + 1];
+        if (h_r1 >= 0) {
+          const int64_t g1 = static_cast<int64_t>(h_bh) * a.Nb + h_r1;
+          h_rp2 = a.row_ptr[g1];
+          h_rp3 = a.row_ptr[g1 + 1];
+        }
+        hs = 3;
+      } else if (hs == 3) {
+        const int64_t n0 = h_rp1 - h_rp0, n1 = h_r1 >= 0 ? h_rp3 - h_rp2 : 0;
+        h_pre0 = lane < n0 ? a.col_idx[h_rp0 + lane] : 0;
+        h_pre1 = lane < n1 ? a.col_idx[h_rp2 + lane] : 0;
+        if (lane == 0) {
+          prefetch_block<kRaster>(&tq, a, h_bh, h_r0);
+          if (h_r1 >= 0) prefetch_block<kRaster>(&tq, a, h_bh, h_r1);
+        }
+        hs = 4;
+      }
+    };
+    while (hs < 4) advance();
     while (ok) {
-      int item = 0;
-      if (lane == 0) item = atomicAdd(a.counter, 1);
-      item = __shfl_sync(0xFFFFFFFFu, item, 0);
-      if (item >= n_items) {
+      if (hs == 5) {
         // one end record per softmax group (they take alternate steps), then
         // the V blocks still owed
         StepMeta r{};
@@ -343,9 +398,20 @@ __global__ void __maxnreg__(168)
         if (emit(r)) emit(r);
         break;
       }
-      item = a.order[item];
-      int bh, r0, r1;
-      decode_item(item, a, bh, r0, r1);
+      const int bh = h_bh, r0 = h_r0, r1 = h_r1;
+      const int64_t b0 = h_rp0, n0 = h_rp1 - h_rp0;
+      const int64_t b1 = r1 >= 0 ? h_rp2 : 0, n1 = r1 >= 0 ? h_rp3 - h_rp2 : 0;
+      // first windows from the prefetched entries; the next windows' entries
+      // are loaded into registers one window ahead
+      __syncwarp();
+      if (lane < kListWin) {
+        list0[lane] = h_pre0;
+        list1[lane] = h_pre1;
+      }
+      __syncwarp();
+      int nx0 = lane < n0 - kListWin ? a.col_idx[b0 + kListWin + lane] : 0;
+      int nx1 = lane < n1 - kListWin ? a.col_idx[b1 + kListWin + lane] : 0;
+      hs = 0;                          // start on the following item's header
       // Q tile: query block r0 -> rows 0..63, r1 -> rows 64..127
       if (nitems > 0) {
         if (!mbar_wait(q_empty, q_phase, a.err, kErrWaitMma)) break;
@@ -360,14 +426,7 @@ __global__ void __maxnreg__(168)
       }
       // merge the two ascending lists, two union entries per step
       const int64_t g0 = static_cast<int64_t>(bh) * a.Nb + r0;
-      const int64_t b0 = a.row_ptr[g0], n0 = a.row_ptr[g0 + 1] - b0;
-      int64_t b1 = 0, n1 = 0;
-      if (r1 >= 0) {
-        const int64_t g1 = static_cast<int64_t>(bh) * a.Nb + r1;
-        b1 = a.row_ptr[g1];
-        n1 = a.row_ptr[g1 + 1] - b1;
-      }
-      int64_t i0 = 0, i1 = 0, w0 = -kListWin, w1 = -kListWin;
+      int64_t i0 = 0, i1 = 0, w0 = 0, w1 = 0;
       StepMeta pend{};
       pend.bh = bh; pend.r0 = r0; pend.r1 = r1;
       pend.seq = nitems - 1;
@@ -377,16 +436,18 @@ __global__ void __maxnreg__(168)
       cur.nb = 0; cur.flags = 0; cur.blk0 = cur.blk1 = -1;
       while (i0 < n0 || i1 < n1) {
         if (i0 < n0 && i0 >= w0 + kListWin) {
-          w0 = i0;
+          w0 += kListWin;
           __syncwarp();
-          if (lane < kListWin && w0 + lane < n0) list0[lane] = a.col_idx[b0 + w0 + lane];
+          if (lane < kListWin) list0[lane] = nx0;
           __syncwarp();
+          nx0 = lane < n0 - w0 - kListWin ? a.col_idx[b0 + w0 + kListWin + lane] : 0;
         }
         if (i1 < n1 && i1 >= w1 + kListWin) {
-          w1 = i1;
+          w1 += kListWin;
           __syncwarp();
-          if (lane < kListWin && w1 + lane < n1) list1[lane] = a.col_idx[b1 + w1 + lane];
+          if (lane < kListWin) list1[lane] = nx1;
           __syncwarp();
+          nx1 = lane < n1 - w1 - kListWin ? a.col_idx[b1 + w1 + kListWin + lane] : 0;
         }
         const int c0 = i0 < n0 ? list0[i0 - w0] : 0x7FFFFFFF;
         const int c1 = i1 < n1 ? list1[i1 - w1] : 0x7FFFFFFF;
@@ -407,7 +468,10 @@ __global__ void __maxnreg__(168)
           cur.blk1 = c;
           cur.flags |= (f << 2) | (kv << 16);
           cur.nb = 2;
-          if (have_pending && !(ok = emit(pend))) break;
+          if (have_pending) {
+            if (!(ok = emit(pend))) break;
+            advance();
+          }
           pend = cur;
           pend.first_last = have_pending ? 0 : 1;
           have_pending = true;
@@ -416,7 +480,10 @@ __global__ void __maxnreg__(168)
       }
       if (!ok) break;
       if (cur.nb > 0) {
-        if (have_pending && !(ok = emit(pend))) break;
+        if (have_pending) {
+          if (!(ok = emit(pend))) break;
+          advance();
+        }
         const int first = have_pending ? 0 : 1;
         pend = cur;
         pend.first_last = first;
@@ -428,6 +495,7 @@ __global__ void __maxnreg__(168)
       }
       pend.first_last |= 2;
       if (!(ok = emit(pend))) break;
+      while (hs < 4) advance();        // short items: finish the next header now
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ S issuer
@@ -698,30 +766,25 @@ __global__ void __maxnreg__(168)
         const int64_t tok =
             static_cast<int64_t>(m.bh) * a.N + (store ? block_token<kRaster>(a, rblk, row & 63) : 0);
         uint4 *orow = reinterpret_cast<uint4 *>(a.o + tok * D);
-#pragma unroll 1
+        // the whole row of O as packed bf16 first; O is then released to the
+        // next item's PV MMAs before the global stores go out
+        uint32_t pk[D / 2];
+#pragma unroll
         for (int cc = 0; cc < D; cc += 32) {
           float ov[32];
           tmem_ld32(lane_addr + kColO + cc, ov);
-          if (store) {
-            if (!has_keys) {
 #pragma unroll
-              for (int j = 0; j < 32; ++j) ov[j] = 0.0f;
-            }
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              uint4 u;
-              u.x = pack_bf16x2(ov[8 * j + 0] * inv, ov[8 * j + 1] * inv);
-              u.y = pack_bf16x2(ov[8 * j + 2] * inv, ov[8 * j + 3] * inv);
-              u.z = pack_bf16x2(ov[8 * j + 4] * inv, ov[8 * j + 5] * inv);
-              u.w = pack_bf16x2(ov[8 * j + 6] * inv, ov[8 * j + 7] * inv);
-              orow[cc / 8 + j] = u;
-            }
-          }
+          for (int j = 0; j < 16; ++j)
+            pk[cc / 2 + j] = has_keys ? pack_bf16x2(ov[2 * j] * inv, ov[2 * j + 1] * inv) : 0u;
         }
-        if (store)
-          a.lse[tok] = has_keys ? (m_run + log2f(l_run)) * a.lse_scale : -INFINITY;
         tc_fence_before();
         mbar_arrive(o_empty);
+        if (store) {
+#pragma unroll
+          for (int j = 0; j < D / 8; ++j)
+            orow[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          a.lse[tok] = has_keys ? (m_run + log2f(l_run)) * a.lse_scale : -INFINITY;
+        }
       }
     }
   }
