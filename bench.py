@@ -56,6 +56,9 @@ def parse_args():
                          "and write raster o; flat: explicit flatten / unflatten passes")
     ap.add_argument("--cluster", action="store_true",
                     help="only the semantic-aware permutation path at the Wan-14B 720p shape")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run only the first N heads of the workload (small profiling captures; "
+                         "0: all)")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
                     help="N > 1: every rank runs its own layer (replicas, weak scaling), or the "
                          "ranks split one layer's heads (heads, strong scaling)")
@@ -188,6 +191,8 @@ def run_gpu(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     wl = workloads.get(args.workload)
+    if args.heads:
+        wl = wl.replace(heads=min(args.heads, wl.heads))
     params = vsa.MaskParams(wl.thr, wl.use_sta, wl.sta)
     shard = args.shard if world > 1 else "replicas"
     h0, h1 = head_slice(wl.heads, rank, world) if shard == "heads" else (0, wl.heads)
