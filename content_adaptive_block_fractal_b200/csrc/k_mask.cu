@@ -647,30 +647,58 @@ __global__ void __launch_bounds__(kSelWarps * 32) mask_select_kernel(const MaskA
         above_x = 0.0;
         pmin_above = INFINITY;
         pmax_below = 0.0f;
-        for (int c0 = 0; c0 < a.words * 32; c0 += 32) {
-          const int c = c0 + lane;
-          const float p = c < Nb ? ph[c] : 0.0f;
-          const int k = c < Nb ? value_key(p) : 1 << 30;
-          const bool kept = k < klo;
-          if (kept) {
-            above_x += kCount ? 1.0 : static_cast<double>(p);
-            pmin_above = fminf(pmin_above, p);
-          } else if (k >= khi && c < Nb) {
-            pmax_below = fmaxf(pmax_below, p);
-          }
-          const uint32_t kw = __ballot_sync(0xFFFFFFFFu, kept);
-          if (lane == 0) bits[c0 >> 5] = kw;
-          const bool in = k >= klo && k < khi;
-          if (in && khi - klo == 64) atomicAdd(&hist[k - klo], kCount ? 1.0f : p);
-          const uint32_t m = __ballot_sync(0xFFFFFFFFu, in);
-          if (in) {
-            const int pos = ncand + __popc(m & ((1u << lane) - 1u));
-            if (pos < kCand) {
-              cand_c[pos] = c;
-              cand_t[pos] = srow[c];
+        const bool fine = khi - klo == 64;
+        // four consecutive columns per lane: lanes 8j .. 8j+7 cover kept-bit
+        // word j of the 128-column chunk
+        for (int c0 = 0; c0 < a.words * 32; c0 += 128) {
+          const int cb = c0 + 4 * lane;
+          float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          if (cb < Nb) v = *reinterpret_cast<const float4 *>(ph + cb);   // cb + 3 < ldp
+          const float p4[4] = {v.x, v.y, v.z, v.w};
+          uint32_t nib = 0u, inm = 0u;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const bool valid = cb + q < Nb;
+            const int k = valid ? value_key(p4[q]) : 1 << 30;
+            if (k < klo) {
+              above_x += kCount ? 1.0 : static_cast<double>(p4[q]);
+              pmin_above = fminf(pmin_above, p4[q]);
+              nib |= 1u << q;
+            } else if (k >= khi && valid) {
+              pmax_below = fmaxf(pmax_below, p4[q]);
             }
+            const bool in = k >= klo && k < khi;
+            inm |= (in ? 1u : 0u) << q;
+            if (in && fine) atomicAdd(&hist[k - klo], kCount ? 1.0f : p4[q]);
           }
-          ncand += __popc(m);
+          uint32_t wv = nib << (4 * (lane & 7));
+          wv |= __shfl_xor_sync(0xFFFFFFFFu, wv, 1);
+          wv |= __shfl_xor_sync(0xFFFFFFFFu, wv, 2);
+          wv |= __shfl_xor_sync(0xFFFFFFFFu, wv, 4);
+          const int w = (c0 >> 5) + (lane >> 3);
+          if ((lane & 7) == 0 && w < a.words) bits[w] = wv;
+          // the range's blocks, in column order
+          if (__any_sync(0xFFFFFFFFu, inm != 0u)) {
+            const int ni = __popc(inm);
+            int incl = ni;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+              const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+              if (lane >= o) incl += y;
+            }
+            int pos = ncand + incl - ni;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if ((inm >> q) & 1u) {
+                if (pos < kCand) {
+                  cand_c[pos] = cb + q;
+                  cand_t[pos] = srow[cb + q];
+                }
+                ++pos;
+              }
+            }
+            ncand += __shfl_sync(0xFFFFFFFFu, incl, 31);
+          }
         }
         above_x = warp_sum(above_x);
 #pragma unroll
@@ -691,39 +719,61 @@ __global__ void __launch_bounds__(kSelWarps * 32) mask_select_kernel(const MaskA
       }
       // 4. sort the cut bin (t desc, index asc) and cut it
       if (!recheck) {
+        // sort key: t descending (fp32 patterns made to order like t, then
+        // inverted), index ascending
+        auto sort_key = [&](int v) -> uint64_t {
+          uint32_t o = __float_as_uint(cand_t[v]);
+          o = (o & 0x80000000u) ? ~o : (o | 0x80000000u);     // orders like t
+          return (static_cast<uint64_t>(~o) << 32) | static_cast<uint32_t>(cand_c[v]);
+        };
         uint64_t key[2];
+        if (ncand <= 32) {
+          // one key per lane: bitonic sort of 32, then position i to lane i/2
+          uint64_t k1 = lane < ncand ? sort_key(lane) : ~0ull;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int v = 2 * lane + h;
-          if (v < ncand) {
-            uint32_t o = __float_as_uint(cand_t[v]);
-            o = (o & 0x80000000u) ? ~o : (o | 0x80000000u);     // orders like t
-            key[h] = (static_cast<uint64_t>(~o) << 32) | static_cast<uint32_t>(cand_c[v]);
-          } else {
-            key[h] = ~0ull;
+          for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+              const uint64_t other = __shfl_xor_sync(0xFFFFFFFFu, k1, stride);
+              const bool up = (lane & size) == 0;
+              const bool lower = (lane & stride) == 0;
+              const uint64_t lo = k1 < other ? k1 : other;
+              const uint64_t hi = k1 < other ? other : k1;
+              k1 = (lower == up) ? lo : hi;
+            }
           }
-        }
-        // bitonic sort of 64 keys, ascending, key h of lane l at position 2l + h
+          const uint64_t a0 = __shfl_sync(0xFFFFFFFFu, k1, (2 * lane) & 31);
+          const uint64_t a1 = __shfl_sync(0xFFFFFFFFu, k1, (2 * lane + 1) & 31);
+          key[0] = lane < 16 ? a0 : ~0ull;
+          key[1] = lane < 16 ? a1 : ~0ull;
+        } else {
 #pragma unroll
-        for (int size = 2; size <= 64; size <<= 1) {
+          for (int h = 0; h < 2; ++h) {
+            const int v = 2 * lane + h;
+            key[h] = v < ncand ? sort_key(v) : ~0ull;
+          }
+          // bitonic sort of 64 keys, ascending, key h of lane l at position 2l + h
 #pragma unroll
-          for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            if (stride == 1) {
-              const bool up = ((2 * lane) & size) == 0;
-              const uint64_t lo = key[0] < key[1] ? key[0] : key[1];
-              const uint64_t hi = key[0] < key[1] ? key[1] : key[0];
-              key[0] = up ? lo : hi;
-              key[1] = up ? hi : lo;
-            } else {
+          for (int size = 2; size <= 64; size <<= 1) {
 #pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const int pos = 2 * lane + h;
-                const uint64_t other = __shfl_xor_sync(0xFFFFFFFFu, key[h], stride >> 1);
-                const bool up = (pos & size) == 0;
-                const bool lower = (pos & stride) == 0;
-                const uint64_t lo = key[h] < other ? key[h] : other;
-                const uint64_t hi = key[h] < other ? other : key[h];
-                key[h] = (lower == up) ? lo : hi;
+            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+              if (stride == 1) {
+                const bool up = ((2 * lane) & size) == 0;
+                const uint64_t lo = key[0] < key[1] ? key[0] : key[1];
+                const uint64_t hi = key[0] < key[1] ? key[1] : key[0];
+                key[0] = up ? lo : hi;
+                key[1] = up ? hi : lo;
+              } else {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  const int pos = 2 * lane + h;
+                  const uint64_t other = __shfl_xor_sync(0xFFFFFFFFu, key[h], stride >> 1);
+                  const bool up = (pos & size) == 0;
+                  const bool lower = (pos & stride) == 0;
+                  const uint64_t lo = key[h] < other ? key[h] : other;
+                  const uint64_t hi = key[h] < other ? other : key[h];
+                  key[h] = (lower == up) ? lo : hi;
+                }
               }
             }
           }
