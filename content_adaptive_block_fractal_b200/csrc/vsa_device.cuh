@@ -44,18 +44,18 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
 }
-// Suspend-time hint for try_wait (ns): a waiting warp is parked by the
-// hardware until the phase completes or the hint expires, instead of
-// spinning and taking issue slots from the warps it shares a scheduler with.
-constexpr uint32_t kSuspendHintNs = 1000000;
+// try_wait blocks the warp for a hardware-chosen time while the phase is
+// open, then reports; the callers re-poll under their own cycle limit.  No
+// suspend-time hint: with an explicit long hint the attention kernel ran 1-2%
+// slower on B200 (later wake-ups on its chain of barrier hand-offs).
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+      : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
 }
