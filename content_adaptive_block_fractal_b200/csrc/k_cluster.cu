@@ -279,19 +279,23 @@ __global__ void __launch_bounds__(kTile) position_kernel(const int32_t *__restri
   inv[bh * Np + p] = static_cast<int32_t>(t);
 }
 
-// xp[bh][r] = x[bh][inv[r]] (16-byte vectors, a warp per row); padding rows zero.
+// xp[bh][r] = x[bh][inv[r]] (16-byte vectors; vec = d/8 lanes per row, so a
+// warp moves 32/vec rows at a time); padding rows zero.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restrict__ x,
                                                           const int32_t *__restrict__ inv,
                                                           int64_t BH, int64_t N, int64_t Np,
                                                           int vec, uint4 *__restrict__ xp) {
   const int lane = threadIdx.x & 31;
+  const int per = 32 / vec, sub = lane / vec, col = lane % vec;
   const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-       r < BH * Np; r += warps) {
-    const int64_t bh = r / Np;
-    const int32_t t = inv[r];
-    for (int i = lane; i < vec; i += 32)
-      xp[r * vec + i] = t >= 0 ? __ldg(x + (bh * N + t) * vec + i) : make_uint4(0, 0, 0, 0);
+  for (int64_t r0 = ((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5) * per;
+       r0 < BH * Np; r0 += warps * per) {
+    const int64_t r = r0 + sub;
+    if (r < BH * Np) {
+      const int64_t bh = r / Np;
+      const int32_t t = inv[r];
+      xp[r * vec + col] = t >= 0 ? __ldg(x + (bh * N + t) * vec + col) : make_uint4(0, 0, 0, 0);
+    }
   }
 }
 
@@ -319,15 +323,29 @@ __global__ void __launch_bounds__(256)
   double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   const int32_t *members = inv + bh * Np + s0;      // token of each member, in order
   const uint4 *head = x + bh * N * kLanesPerRow + col;
-  for (int32_t m = sub; m < n; m += kRowsPerStep) {
-    const uint4 v = __ldg(head + static_cast<int64_t>(members[m]) * kLanesPerRow);
+  auto add = [&](const uint4 v) {
     const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       acc[2 * e] += static_cast<double>(__uint_as_float(u[e] << 16));
       acc[2 * e + 1] += static_cast<double>(__uint_as_float(u[e] & 0xFFFF0000u));
     }
+  };
+  // four members in flight per lane (index loads, then row loads), added in
+  // member order as one at a time would
+  int32_t m = sub;
+  for (; m + 3 * kRowsPerStep < n; m += 4 * kRowsPerStep) {
+    int32_t t[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) t[k] = members[m + k * kRowsPerStep];
+    uint4 v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[k] = __ldg(head + static_cast<int64_t>(t[k]) * kLanesPerRow);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) add(v[k]);
   }
+  for (; m < n; m += kRowsPerStep)
+    add(__ldg(head + static_cast<int64_t>(members[m]) * kLanesPerRow));
 #pragma unroll
   for (int off = kLanesPerRow; off < 32; off <<= 1)
 #pragma unroll
@@ -547,13 +565,17 @@ __global__ void __launch_bounds__(256) unpermute_kernel(const uint4 *__restrict_
                                                         int vec, uint4 *__restrict__ o,
                                                         float *__restrict__ lse) {
   const int lane = threadIdx.x & 31;
+  const int per = 32 / vec, sub = lane / vec, col = lane % vec;   // 32/vec rows per warp
   const int64_t warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-       r < BH * N; r += warps) {
-    const int64_t bh = r / N;
-    const int64_t src = bh * Np + pos[r];
-    for (int i = lane; i < vec; i += 32) o[r * vec + i] = op[src * vec + i];
-    if (lane == 0) lse[r] = lsep[src];
+  for (int64_t r0 = ((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5) * per;
+       r0 < BH * N; r0 += warps * per) {
+    const int64_t r = r0 + sub;
+    if (r < BH * N) {
+      const int64_t bh = r / N;
+      const int64_t src = bh * Np + pos[r];
+      o[r * vec + col] = op[src * vec + col];
+      if (col == 0) lse[r] = lsep[src];
+    }
   }
 }
 
