@@ -300,10 +300,12 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restric
 }
 
 // Member means in fp64, the members read through the inverse map of the
-// permutation (position -> token); an empty cluster keeps its centroid.  A warp per cluster: d/8
-// lanes read a row's 16-byte vectors, so a warp covers 256/d rows per step,
-// each lane keeping 8 fp64 column sums; the partial sums of the row classes
-// are added at the end.
+// permutation (position -> token); an empty cluster keeps its centroid.  A
+// CTA per cluster: each of its 8 warps sums a contiguous eighth of the
+// members (d/8 lanes read a row's 16-byte vectors, so a warp covers 256/d
+// rows per step, four steps in flight), each lane keeping 8 fp64 column
+// sums; the warps' partial sums are added in warp order, so the result does
+// not depend on scheduling.
 template <int D>
 __global__ void __launch_bounds__(256)
     centroid_update_kernel(const uint4 *__restrict__ x, const int32_t *__restrict__ inv,
@@ -311,15 +313,20 @@ __global__ void __launch_bounds__(256)
                            int64_t BH, int64_t N, int C, int64_t Np, float *__restrict__ cent) {
   constexpr int kLanesPerRow = D / 8;
   constexpr int kRowsPerStep = 32 / kLanesPerRow;
-  const int lane = threadIdx.x & 31;
+  constexpr int kWarps = 8;
+  __shared__ double part[kWarps][D];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int sub = lane / kLanesPerRow, col = lane % kLanesPerRow;
-  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t w = blockIdx.x;                 // cluster bh * C + j
   if (w >= BH * C) return;
   const int64_t bh = w / C;
   const int j = static_cast<int>(w % C);
   const int32_t n = count[w];
   if (n == 0) return;
   const int32_t s0 = start[bh * (C + 1) + j];
+  const int32_t chunk = (n + kWarps - 1) / kWarps;
+  const int32_t lo = warp * chunk < n ? warp * chunk : n;
+  const int32_t hi = lo + chunk < n ? lo + chunk : n;
   double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   const int32_t *members = inv + bh * Np + s0;      // token of each member, in order
   const uint4 *head = x + bh * N * kLanesPerRow + col;
@@ -331,10 +338,8 @@ __global__ void __launch_bounds__(256)
       acc[2 * e + 1] += static_cast<double>(__uint_as_float(u[e] & 0xFFFF0000u));
     }
   };
-  // four members in flight per lane (index loads, then row loads), added in
-  // member order as one at a time would
-  int32_t m = sub;
-  for (; m + 3 * kRowsPerStep < n; m += 4 * kRowsPerStep) {
+  int32_t m = lo + sub;
+  for (; m + 3 * kRowsPerStep < hi; m += 4 * kRowsPerStep) {
     int32_t t[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) t[k] = members[m + k * kRowsPerStep];
@@ -344,16 +349,22 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int k = 0; k < 4; ++k) add(v[k]);
   }
-  for (; m < n; m += kRowsPerStep)
+  for (; m < hi; m += kRowsPerStep)
     add(__ldg(head + static_cast<int64_t>(members[m]) * kLanesPerRow));
 #pragma unroll
   for (int off = kLanesPerRow; off < 32; off <<= 1)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xFFFFFFFFu, acc[e], off);
   if (sub == 0) {
-    float *dst = cent + w * D + col * 8;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) dst[e] = static_cast<float>(acc[e] / n);
+    for (int e = 0; e < 8; ++e) part[warp][col * 8 + e] = acc[e];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < D; i += blockDim.x) {
+    double t = 0.0;
+#pragma unroll
+    for (int k = 0; k < kWarps; ++k) t += part[k][i];
+    cent[w * D + i] = static_cast<float>(t / n);
   }
 }
 
@@ -708,7 +719,7 @@ static cudaError_t run_kmeans(const void *x, const Geometry &g, int C, int iters
     position_kernel<<<static_cast<int>(BH * L.ntile), kTile, 0, st>>>(label, N, C, L.ntile, hist,
                                                                        start, pos, inv, Np);
     if (it < iters) {
-      const int ub = static_cast<int>((BH * C * 32 + 255) / 256);
+      const int ub = static_cast<int>(BH * C);      // a CTA per cluster
       const uint4 *x4 = static_cast<const uint4 *>(x);
       if (d == 128)
         centroid_update_kernel<128><<<ub, 256, 0, st>>>(x4, inv, start, count, BH, N, C, Np,
