@@ -67,8 +67,8 @@ struct AssignSmem {
   static constexpr int kTileBytes = 128 * D * 2;   // 128 rows, K-major, 4-D box layout
   static constexpr int kX = 0;
   static constexpr int kC = kTileBytes;
-  static constexpr int kNorm = 2 * kTileBytes;     // 128 fp32
-  static constexpr int kBar = kNorm + 512;         // x_full, c_full, mma_done
+  static constexpr int kNorm = 2 * kTileBytes;     // [2][128] fp32
+  static constexpr int kBar = kNorm + 1024;        // x_full, c_full, mma_done
   static constexpr int kSlot = kBar + 32;
   static constexpr int kBytes = kSlot + 16;
 };
@@ -123,13 +123,19 @@ __global__ void __launch_bounds__(128)
   int arg = 0;
   bool ok = true;
   const int ntiles = Cpad / 128;
+  // The centroid tile buffer is free once its MMA has completed, so the next
+  // tile's TMA load (and its norms, double-buffered) run under this tile's
+  // argmin; the single TMEM accumulator is reused after the block barrier.
+  s_norm[threadIdx.x] = cnorm[bh * Cpad + threadIdx.x];
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(c_full, L::kTileBytes);
+    const int grp = static_cast<int>((bh * Cpad) / 8);
+    tma_load_4d(sbase + L::kC, &tc, c_full, 0, 0, 0, grp);
+    tma_load_4d(sbase + L::kC + L::kTileBytes / 2, &tc, c_full, 0, 0, 0, grp + 8);
+  }
+  __syncthreads();          // norms of tile 0 visible
   for (int ct = 0; ct < ntiles && ok; ++ct) {
-    s_norm[threadIdx.x] = cnorm[bh * Cpad + ct * 128 + threadIdx.x];
     if (threadIdx.x == 0) {
-      mbar_arrive_expect_tx(c_full, L::kTileBytes);
-      const int grp = static_cast<int>((bh * Cpad + ct * 128) / 8);
-      tma_load_4d(sbase + L::kC, &tc, c_full, 0, 0, 0, grp);
-      tma_load_4d(sbase + L::kC + L::kTileBytes / 2, &tc, c_full, 0, 0, 0, grp + 8);
       bool good = (ct > 0 || mbar_wait(x_full, 0, err, kErrWaitTma)) &&
                   mbar_wait(c_full, ct & 1, err, kErrWaitTma);
       if (good) {
@@ -141,10 +147,20 @@ __global__ void __launch_bounds__(128)
         }
       }
       mma_commit(mma_done);   // arrives even when nothing was issued
+      if (!good) ok = false;
     }
-    __syncthreads();          // s_norm visible
     if (!mbar_wait(mma_done, ct & 1, err, kErrWaitMma)) ok = false;
     tc_fence_after();
+    if (ct + 1 < ntiles) {
+      s_norm[((ct + 1) & 1) * 128 + threadIdx.x] = cnorm[bh * Cpad + (ct + 1) * 128 + threadIdx.x];
+      if (threadIdx.x == 0 && ok) {
+        mbar_arrive_expect_tx(c_full, L::kTileBytes);
+        const int grp = static_cast<int>((bh * Cpad + (ct + 1) * 128) / 8);
+        tma_load_4d(sbase + L::kC, &tc, c_full, 0, 0, 0, grp);
+        tma_load_4d(sbase + L::kC + L::kTileBytes / 2, &tc, c_full, 0, 0, 0, grp + 8);
+      }
+    }
+    const float *nrm = s_norm + (ct & 1) * 128;
     float s[64];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -152,7 +168,7 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
       for (int j = 0; j < 64; ++j) {
         const int c = 64 * h + j;
-        const float dist = fmaf(-2.0f, s[j], s_norm[c]);
+        const float dist = fmaf(-2.0f, s[j], nrm[c]);
         if (dist < best) {
           second = best;
           best = dist;
@@ -163,7 +179,7 @@ __global__ void __launch_bounds__(128)
       }
     }
     tc_fence_before();
-    ok = __syncthreads_and(ok) != 0;   // TMEM, the centroid tile and s_norm are reused
+    ok = __syncthreads_and(ok) != 0;   // TMEM and the next tile's norms
   }
   // always a label in [0, C) (0 after a failed wait, recorded in the error
   // word), so the counting sort that follows never indexes out of range
