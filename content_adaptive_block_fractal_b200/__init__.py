@@ -19,7 +19,8 @@ from . import _lib
 from ._lib import VsaError, vsa_mask_params, vsa_shape
 
 __all__ = ["Shape", "MaskParams", "VsaError", "fractal_flatten", "fractal_unflatten",
-           "flatten_pool_qk", "pool_qk_raster", "sparse_attn_fwd_raster", "Layer",
+           "flatten_pool_qk", "pool_qk_raster", "sparse_attn_fwd_raster",
+           "sparse_attn_fwd_to_raster", "Layer",
            "pool_qk", "block_mask", "block_mask_topk", "sta_mask", "sta_mask_nnz",
            "block_mask_workspace_size", "sparse_attn_fwd", "sparse_attn_fwd_rows",
            "ClusterParams", "cluster_attention", "cluster_attn_workspace_size",
@@ -246,6 +247,24 @@ def sparse_attn_fwd_raster(q, k, v, row_ptr, col_idx, shape: Shape, scale: float
         workspace = _workspace(sparse_attn_workspace_size(shape), q.device)
     _lib.check(_lib.load().vsa_sparse_attn_fwd_raster(
         _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr), _ptr(col_idx), shape.c(), float(scale),
+        _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return o, lse
+
+
+def sparse_attn_fwd_to_raster(qf, kf, vf, row_ptr, col_idx, shape: Shape, scale: float = 0.0,
+                              out=None, workspace=None, stream=None):
+    """sparse_attn_fwd on flattened qf, kf, vf -> raster-order (o, lse): the
+    output unflattening done by the attention's stores.  Equals sparse_attn_fwd
+    followed by fractal_unflatten of o (and the same permutation of lse), bit
+    for bit."""
+    if out is None:
+        out = (torch.empty_like(qf),
+               torch.empty((shape.B, shape.heads, shape.N), dtype=torch.float32, device=qf.device))
+    o, lse = out
+    if workspace is None:
+        workspace = _workspace(sparse_attn_workspace_size(shape), qf.device)
+    _lib.check(_lib.load().vsa_sparse_attn_fwd_to_raster(
+        _ptr(qf), _ptr(kf), _ptr(vf), _ptr(row_ptr), _ptr(col_idx), shape.c(), float(scale),
         _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
     return o, lse
 

@@ -23,7 +23,7 @@ EXPORTS = ("vsa_fractal_flatten", "vsa_fractal_unflatten", "vsa_pool_qk",
            "vsa_sta_mask",
            "vsa_sparse_attn_workspace_size", "vsa_sparse_attn_fwd",
            "vsa_sparse_attn_fwd_noalloc", "vsa_sparse_attn_fwd_rows",
-           "vsa_sparse_attn_fwd_raster",
+           "vsa_sparse_attn_fwd_raster", "vsa_sparse_attn_fwd_to_raster",
            "vsa_cluster_attn_workspace_size", "vsa_cluster_attn_fwd",
            "vsa_last_error", "vsa_device_status", "vsa_wait_probe", "vsa_version")
 
@@ -87,6 +87,7 @@ def load():
                          P, P],
         "vsa_sparse_attn_fwd": [P, P, P, P, P, vsa_shape, F, P, P, P, S, P],
         "vsa_sparse_attn_fwd_raster": [P, P, P, P, P, vsa_shape, F, P, P, P, S, P],
+        "vsa_sparse_attn_fwd_to_raster": [P, P, P, P, P, vsa_shape, F, P, P, P, S, P],
         "vsa_sparse_attn_fwd_noalloc": [P, P, P, P, P, vsa_shape, F, P, P, P],
         "vsa_sparse_attn_fwd_rows": [P, P, P, P, P, vsa_shape, F, P, I64, P, P, P, S, P],
         "vsa_device_status": [P],

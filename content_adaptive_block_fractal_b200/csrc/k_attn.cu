@@ -234,9 +234,11 @@ __device__ __forceinline__ void softmax_chunk(uint32_t (&cur)[32], uint32_t (&nx
 }
 
 // kKeyMask: key blocks may be partial (per-block valid counts in AttnArgs);
-// the plain instantiation carries no masking code.  kRaster: Q, K, V, O and
-// LSE in raster token order (blocks fetched as patches), else flattened.
-template <int D, bool kKeyMask, bool kRaster>
+// the plain instantiation carries no masking code.  kLayout 0: Q, K, V, O and
+// LSE in the flattened (fractal) token order; 1: all in raster order (blocks
+// fetched as patches); 2: Q, K, V flattened, O and LSE stored in raster order
+// (the unflatten of the output folded into the epilogue's row addresses).
+template <int D, bool kKeyMask, int kLayout>
 __global__ void __maxnreg__(168)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tq,
                        const __grid_constant__ CUtensorMap tk,
@@ -337,8 +339,8 @@ __global__ void __maxnreg__(168)
         const uint32_t kf = k_full(s3);
         mbar_arrive_expect_tx(kf, static_cast<uint32_t>(nb * L::kBlockBytes));
         const uint32_t kbase = sbase + L::kKOff + s3 * L::kKVBytes;
-        if (nb > 0) load_block<kRaster>(kbase, &tk, kf, a, r.bh, r.blk0);
-        if (nb > 1) load_block<kRaster>(kbase + L::kBlockBytes, &tk, kf, a, r.bh, r.blk1);
+        if (nb > 0) load_block<kLayout == 1>(kbase, &tk, kf, a, r.bh, r.blk0);
+        if (nb > 1) load_block<kLayout == 1>(kbase + L::kBlockBytes, &tk, kf, a, r.bh, r.blk1);
       }
       __syncwarp();
       ++m;
@@ -382,8 +384,8 @@ __global__ void __maxnreg__(168)
         h_pre0 = lane < n0 ? a.col_idx[h_rp0 + lane] : 0;
         h_pre1 = lane < n1 ? a.col_idx[h_rp2 + lane] : 0;
         if (lane == 0) {
-          prefetch_block<kRaster>(&tq, a, h_bh, h_r0);
-          if (h_r1 >= 0) prefetch_block<kRaster>(&tq, a, h_bh, h_r1);
+          prefetch_block<kLayout == 1>(&tq, a, h_bh, h_r0);
+          if (h_r1 >= 0) prefetch_block<kLayout == 1>(&tq, a, h_bh, h_r1);
         }
         hs = 4;
       }
@@ -422,7 +424,7 @@ __global__ void __maxnreg__(168)
         const int nq = r1 >= 0 ? 2 : 1;
         mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(nq * 64 * D * 2));
         for (int j = 0; j < nq; ++j)
-          load_block<kRaster>(sbase + L::kQOff + j * L::kBlockBytes, &tq, q_full, a, bh, j ? r1 : r0);
+          load_block<kLayout == 1>(sbase + L::kQOff + j * L::kBlockBytes, &tq, q_full, a, bh, j ? r1 : r0);
       }
       // merge the two ascending lists, two union entries per step
       const int64_t g0 = static_cast<int64_t>(bh) * a.Nb + r0;
@@ -608,8 +610,8 @@ __global__ void __maxnreg__(168)
         const uint32_t vf = v_full(b);
         mbar_arrive_expect_tx(vf, static_cast<uint32_t>(nb * L::kBlockBytes));
         const uint32_t vbase = sbase + L::kVOff + b * L::kKVBytes;
-        if (nb > 0) load_block<kRaster>(vbase, &tv, vf, a, r.bh, r.blk0);
-        if (nb > 1) load_block<kRaster>(vbase + L::kBlockBytes, &tv, vf, a, r.bh, r.blk1);
+        if (nb > 0) load_block<kLayout == 1>(vbase, &tv, vf, a, r.bh, r.blk0);
+        if (nb > 1) load_block<kLayout == 1>(vbase + L::kBlockBytes, &tv, vf, a, r.bh, r.blk1);
       }
       __syncwarp();
     }
@@ -764,7 +766,7 @@ __global__ void __maxnreg__(168)
         const bool has_keys = l_run > 0.0f;
         const float inv = has_keys ? 1.0f / l_run : 0.0f;
         const int64_t tok =
-            static_cast<int64_t>(m.bh) * a.N + (store ? block_token<kRaster>(a, rblk, row & 63) : 0);
+            static_cast<int64_t>(m.bh) * a.N + (store ? block_token<kLayout != 0>(a, rblk, row & 63) : 0);
         uint4 *orow = reinterpret_cast<uint4 *>(a.o + tok * D);
         // the whole row of O as packed bf16 first; O is then released to the
         // next item's PV MMAs before the global stores go out
@@ -906,19 +908,21 @@ cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
                                const Geometry &g, float scale, void *o, float *lse, void *ws,
                                unsigned *err, cudaStream_t st, const char **why,
                                const int32_t *qblocks, int64_t n_qblocks,
-                               const int32_t *kvalid, bool raster) {
+                               const int32_t *kvalid, int layout) {
+  const bool raster = layout == 1;          // raster loads
+  const bool raster_out = layout != 0;      // raster O and LSE
   const AttnLayout L = attn_layout(g);
   if (L.items == 0 || (qblocks && n_qblocks == 0)) return cudaSuccess;
   if (L.items > 0x7FFFFFFF || g.BH * g.N > 0x7FFFFFFF) {
     *why = "sparse attention: too many tokens for 32-bit TMA row coordinates";
     return cudaErrorInvalidValue;
   }
-  if (raster && g.Nb * L.HW >= (1LL << 32)) {
+  if (raster_out && g.Nb * L.HW >= (1LL << 32)) {
     *why = "sparse attention: too many blocks per head for the raster layout";
     return cudaErrorInvalidValue;
   }
   const bool masked = kvalid != nullptr;
-  if (raster && masked) {
+  if (raster_out && masked) {
     *why = "sparse attention: key masking is not available in the raster layout";
     return cudaErrorInvalidValue;
   }
@@ -970,32 +974,36 @@ cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
   int grid = num_sms();
   const int64_t max_items = qblocks ? (n_qblocks < L.items ? n_qblocks : L.items) : L.items;
   if (max_items < grid) grid = static_cast<int>(max_items);
-  // three instantiations per d: flattened, flattened with key masking (the
-  // cluster path), raster
+  // four instantiations per d: flattened, flattened with key masking (the
+  // cluster path), raster, flattened in with raster O and LSE out
   const void *fn;
   int smem;
   if (g.d == 128) {
-    fn = masked   ? reinterpret_cast<const void *>(sparse_attn_kernel<128, true, false>)
-         : raster ? reinterpret_cast<const void *>(sparse_attn_kernel<128, false, true>)
-                  : reinterpret_cast<const void *>(sparse_attn_kernel<128, false, false>);
+    fn = masked       ? reinterpret_cast<const void *>(sparse_attn_kernel<128, true, 0>)
+         : raster     ? reinterpret_cast<const void *>(sparse_attn_kernel<128, false, 1>)
+         : raster_out ? reinterpret_cast<const void *>(sparse_attn_kernel<128, false, 2>)
+                      : reinterpret_cast<const void *>(sparse_attn_kernel<128, false, 0>);
     smem = Smem<128>::kAlloc;
   } else {
-    fn = masked   ? reinterpret_cast<const void *>(sparse_attn_kernel<64, true, false>)
-         : raster ? reinterpret_cast<const void *>(sparse_attn_kernel<64, false, true>)
-                  : reinterpret_cast<const void *>(sparse_attn_kernel<64, false, false>);
+    fn = masked       ? reinterpret_cast<const void *>(sparse_attn_kernel<64, true, 0>)
+         : raster     ? reinterpret_cast<const void *>(sparse_attn_kernel<64, false, 1>)
+         : raster_out ? reinterpret_cast<const void *>(sparse_attn_kernel<64, false, 2>)
+                      : reinterpret_cast<const void *>(sparse_attn_kernel<64, false, 0>);
     smem = Smem<64>::kAlloc;
   }
   if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
       cudaSuccess)
     return e;
   if (g.d == 128) {
-    if (masked) sparse_attn_kernel<128, true, false><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
-    else if (raster) sparse_attn_kernel<128, false, true><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
-    else sparse_attn_kernel<128, false, false><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+    if (masked) sparse_attn_kernel<128, true, 0><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+    else if (raster) sparse_attn_kernel<128, false, 1><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+    else if (raster_out) sparse_attn_kernel<128, false, 2><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+    else sparse_attn_kernel<128, false, 0><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
   } else {
-    if (masked) sparse_attn_kernel<64, true, false><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
-    else if (raster) sparse_attn_kernel<64, false, true><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
-    else sparse_attn_kernel<64, false, false><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+    if (masked) sparse_attn_kernel<64, true, 0><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+    else if (raster) sparse_attn_kernel<64, false, 1><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+    else if (raster_out) sparse_attn_kernel<64, false, 2><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
+    else sparse_attn_kernel<64, false, 0><<<grid, kThreads, smem, st>>>(mq, mk, mv, a);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) {

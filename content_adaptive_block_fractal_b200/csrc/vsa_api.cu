@@ -362,7 +362,7 @@ static vsa_status sparse_attn(const void *qf, const void *kf, const void *vf,
                               const int64_t *row_ptr, const int32_t *col_idx, vsa_shape s,
                               float scale, const int32_t *qblocks, int64_t n_qblocks, void *o,
                               float *lse, void *workspace, size_t workspace_bytes, void *stream,
-                              bool raster = false);
+                              int layout = 0);
 
 vsa_status vsa_sparse_attn_fwd(const void *qf, const void *kf, const void *vf,
                                const int64_t *row_ptr, const int32_t *col_idx, vsa_shape s,
@@ -377,7 +377,16 @@ vsa_status vsa_sparse_attn_fwd_raster(const void *q, const void *k, const void *
                                       vsa_shape s, float scale, void *o, float *lse,
                                       void *workspace, size_t workspace_bytes, void *stream) {
   return sparse_attn(q, k, v, row_ptr, col_idx, s, scale, nullptr, 0, o, lse, workspace,
-                     workspace_bytes, stream, true);
+                     workspace_bytes, stream, 1);
+}
+
+vsa_status vsa_sparse_attn_fwd_to_raster(const void *qf, const void *kf, const void *vf,
+                                         const int64_t *row_ptr, const int32_t *col_idx,
+                                         vsa_shape s, float scale, void *o, float *lse,
+                                         void *workspace, size_t workspace_bytes,
+                                         void *stream) {
+  return sparse_attn(qf, kf, vf, row_ptr, col_idx, s, scale, nullptr, 0, o, lse, workspace,
+                     workspace_bytes, stream, 2);
 }
 
 vsa_status vsa_sparse_attn_fwd_rows(const void *qf, const void *kf, const void *vf,
@@ -405,7 +414,7 @@ static vsa_status sparse_attn(const void *qf, const void *kf, const void *vf,
                               const int64_t *row_ptr, const int32_t *col_idx, vsa_shape s,
                               float scale, const int32_t *qblocks, int64_t n_qblocks, void *o,
                               float *lse, void *workspace, size_t workspace_bytes, void *stream,
-                              bool raster) {
+                              int layout) {
   vsa_status st = check_shape(s);
   if (st != VSA_OK) return st;
   if (empty(s)) return VSA_OK;
@@ -427,7 +436,7 @@ static vsa_status sparse_attn(const void *qf, const void *kf, const void *vf,
   const char *why = nullptr;
   e = vsa::launch_sparse_attn(qf, kf, vf, row_ptr, col_idx, g, scale, o, lse, workspace, err,
                               static_cast<cudaStream_t>(stream), &why, qblocks, n_qblocks,
-                              nullptr, raster);
+                              nullptr, layout);
   if (e != cudaSuccess)
     return why ? fail(e == cudaErrorInvalidValue ? VSA_ERR_UNSUPPORTED : VSA_ERR_CUDA, "%s", why)
                : cuda_fail(e, "sparse attention launch");

@@ -58,7 +58,7 @@ cudaError_t launch_sparse_attn(const void *qf, const void *kf, const void *vf,
                                const Geometry &g, float scale, void *o, float *lse, void *ws,
                                unsigned *err, cudaStream_t st, const char **why,
                                const int32_t *qblocks = nullptr, int64_t n_qblocks = 0,
-                               const int32_t *kvalid = nullptr, bool raster = false);
+                               const int32_t *kvalid = nullptr, int layout = 0);
 
 // Semantic-aware permutation attention: workspace and launch.
 size_t cluster_workspace_bytes(const Geometry &g, const vsa_cluster_params &c);

@@ -18,7 +18,9 @@
  *   and vsa_fractal_unflatten    to bring O back to raster order.
  * Steps 1 and 5's unflattening can also be left to the attention's own
  * loads and stores: vsa_pool_qk_raster and vsa_sparse_attn_fwd_raster take
- * raster tensors and give the same results with no permuted copy written.
+ * raster tensors and give the same results with no permuted copy written;
+ * vsa_sparse_attn_fwd_to_raster takes flattened q, k, v and writes o and lse
+ * in raster order.
  *
  * Conventions shared by every entry point
  *   - Pointers marked "device" are CUDA device pointers on the current device;
@@ -130,9 +132,12 @@ vsa_status vsa_pool_qk_raster(const void *q, const void *k, double *qp, double *
  *   kept_count : optional device int32 [B*heads*Nb] (may be NULL).
  *   workspace  : device scratch of at least vsa_block_mask_workspace_size(s)
  *                bytes, 256-byte aligned; its contents need no initialisation.
- * Pooled scores are formed in fp64; probabilities carry a relative error
- * below 1e-6, so only rows whose cut lies within that of 1 - thr (or of a tie
- * across the cut) can differ from exact arithmetic. */
+ * Scores come from exact integer tensor-core products of base-2^7 digits of
+ * the fp64 means, with a proven bound on the dropped low-order products; a
+ * row is decided on them only when that bound cannot change its kept set, and
+ * is otherwise recomputed in fp64 (scores, softmax, sorted prefix mass).  The
+ * kept sets therefore match an fp64 evaluation except where fp64 rounding
+ * order itself decides (a cut mass within rounding of 1 - thr). */
 size_t vsa_block_mask_workspace_size(vsa_shape s);
 vsa_status vsa_block_mask(const double *qp, const double *kp, vsa_shape s,
                           vsa_mask_params p, int64_t *row_ptr, int32_t *col_idx,
@@ -205,6 +210,20 @@ vsa_status vsa_sparse_attn_fwd_raster(const void *q, const void *k, const void *
                                       const int64_t *row_ptr, const int32_t *col_idx,
                                       vsa_shape s, float scale, void *o, float *lse,
                                       void *workspace, size_t workspace_bytes, void *stream);
+
+/* 5. from flattened q, k, v (as vsa_sparse_attn_fwd takes them) to raster o
+ * and lse: the output unflattening (vsa_fractal_unflatten) folded into the
+ * attention's stores, each output row written at its raster position
+ * n = (t*H + y)*W + x.  qf, kf, vf : device bf16 [B,heads,N,d] flattened;
+ * o : device bf16 [B,heads,N,d] and lse : fp32 [B,heads,N] in raster order.
+ * Equals, bit for bit, vsa_sparse_attn_fwd followed by vsa_fractal_unflatten
+ * of o and the same permutation of lse.  Workspace and errors as
+ * vsa_sparse_attn_fwd. */
+vsa_status vsa_sparse_attn_fwd_to_raster(const void *qf, const void *kf, const void *vf,
+                                         const int64_t *row_ptr, const int32_t *col_idx,
+                                         vsa_shape s, float scale, void *o, float *lse,
+                                         void *workspace, size_t workspace_bytes,
+                                         void *stream);
 
 /* Query-subset attention (HSA, arXiv 2605.06892 summary, section 2.2 "KV cache
  * synchronisation": only the active tokens form queries, against the whole

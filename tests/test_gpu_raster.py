@@ -3,7 +3,8 @@ that take Q, K, V in raster token order, fetch each fractal block as one
 patch-shaped TMA box and store O and LSE at raster positions.
 
 Checked bit for bit against the flattened path (flatten, pool, attention,
-unflatten) on the same inputs and mask, and against the oracle on sampled
+unflatten) on the same inputs and mask -- as is the attention that takes the
+flattened tensors and stores O and LSE in raster order -- and against the oracle on sampled
 query blocks: at small shapes (several tiles, odd frame counts that leave a
 query tile half empty, non-square frames, d = 64 and 128, B > 1, thr = 0) and
 at the full 14B 720p and 241-frame sizes in the configuration the layer
@@ -42,8 +43,11 @@ def compare(wl, n_blocks):
     csr = vsa.block_mask(qp, kp, shape, params)
     o_f, l_f = vsa.sparse_attn_fwd(qf, kf, vf, csr.row_ptr, csr.col_idx, shape)
     o_r, l_r = vsa.sparse_attn_fwd_raster(qd, kd, vd, csr.row_ptr, csr.col_idx, shape)
+    # flattened inputs, raster outputs: the unflatten folded into the stores
+    o_t, l_t = vsa.sparse_attn_fwd_to_raster(qf, kf, vf, csr.row_ptr, csr.col_idx, shape)
     vsa.device_status()
-    del qf, kf, vf
+    assert torch.equal(o_t, o_r) and torch.equal(l_t, l_r)
+    del qf, kf, vf, o_t, l_t
     # flattened token i sits at raster position order[i]
     order_np = oracle.fractal_order(wl.T, wl.H, wl.W)
     order = torch.as_tensor(order_np).cuda()
