@@ -151,6 +151,15 @@ def test_raster_pool_and_attention_validation():
     assert attn(lse=(1 << 29) + 2) == 2
     assert attn(ws_bytes=8) == 3                    # workspace too small
     assert len(L.vsa_last_error()) > 0
+    # flattened inputs, raster outputs: the same checks before any launch
+    def to_raster(ws_bytes=1 << 20, q=1 << 12, lse=1 << 29):
+        return L.vsa_sparse_attn_fwd_to_raster(P(q), P(1 << 16), P(1 << 20), P(1 << 24),
+                                               P(1 << 26), s.c(), 0.0, P(1 << 28), P(lse),
+                                               P(1 << 30), ws_bytes, None)
+    assert to_raster(q=0) == 1
+    assert to_raster(q=(1 << 12) + 8) == 2
+    assert to_raster(lse=(1 << 29) + 2) == 2
+    assert to_raster(ws_bytes=8) == 3
 
 
 def test_layer_layout_is_checked_before_allocating():
@@ -164,6 +173,8 @@ def test_raster_entry_points_accept_an_empty_shape():
     assert L.vsa_pool_qk_raster(None, None, None, None, s, None) == 0
     assert L.vsa_sparse_attn_fwd_raster(None, None, None, None, None, s, 0.0, None, None, None,
                                         0, None) == 0
+    assert L.vsa_sparse_attn_fwd_to_raster(None, None, None, None, None, s, 0.0, None, None,
+                                           None, 0, None) == 0
 
 
 def test_wait_probe_limit_validated_on_the_host():
